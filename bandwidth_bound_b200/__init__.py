@@ -1,0 +1,265 @@
+"""Python binding of libmk.so, the B200 decode-step megakernel.
+
+Argument marshalling only: every step of the decode path runs inside the CUDA
+kernel behind the C ABI declared in include/mk.h.  torch is used for device
+memory and streams.  There is no CPU fallback: if libmk.so is missing or cannot
+be loaded, importing the binding's entry points raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmk.so")
+
+MK_OK = 0
+MK_ERR_INVALID_ARG = -1
+MK_ERR_UNSUPPORTED_CFG = -2
+MK_ERR_SCHEDULE_INVALID = -3
+MK_ERR_CUDA = -4
+MK_ERR_DEVICE_TIMEOUT = -5
+MK_ERR_BOUNDS = -6
+MK_ERR_NO_DEVICE = -7
+
+MK_CREATE_SKIP_VALIDATE = 1
+
+MK_FAULT_DROP_WAIT = 1
+MK_FAULT_RAISE_TARGET = 2
+MK_FAULT_REORDER = 3
+MK_FAULT_DUP_UNIT = 4
+MK_FAULT_OVERSIZE_STAGE = 5
+
+
+class MkError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"mk error {code}: {msg}")
+        self.code = code
+
+
+class ModelCfg(ctypes.Structure):
+    _fields_ = [("n_layers", ctypes.c_int32), ("hidden", ctypes.c_int32), ("n_heads", ctypes.c_int32),
+                ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("ffn", ctypes.c_int32),
+                ("vocab", ctypes.c_int32), ("tied", ctypes.c_int32), ("rope_theta", ctypes.c_float),
+                ("rms_eps", ctypes.c_float), ("max_batch", ctypes.c_int32), ("max_ctx", ctypes.c_int32),
+                ("page_size", ctypes.c_int32)]
+
+
+_PP = ctypes.POINTER(ctypes.c_void_p)
+
+
+class WeightPtrs(ctypes.Structure):
+    _fields_ = [("embed", ctypes.c_void_p), ("final_norm", ctypes.c_void_p), ("lm_head", ctypes.c_void_p),
+                ("attn_norm", _PP), ("wq", _PP), ("wk", _PP), ("wv", _PP), ("wo", _PP),
+                ("mlp_norm", _PP), ("w_gate", _PP), ("w_up", _PP), ("w_down", _PP)]
+
+
+class KvCache(ctypes.Structure):
+    _fields_ = [("k_pool", ctypes.c_void_p), ("v_pool", ctypes.c_void_p), ("page_table", ctypes.c_void_p),
+                ("num_pages", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32)]
+
+
+class PlanOpts(ctypes.Structure):
+    _fields_ = [("num_sms", ctypes.c_int32), ("attn_slots_per_sm", ctypes.c_int32),
+                ("max_blocks", ctypes.c_int32)]
+
+
+class PlanInfo(ctypes.Structure):
+    _fields_ = [("n_tasks", ctypes.c_int64), ("n_stages", ctypes.c_int64), ("max_tasks_per_sm", ctypes.c_int64),
+                ("weight_bytes_min_sm", ctypes.c_int64), ("weight_bytes_max_sm", ctypes.c_int64),
+                ("attn_slots", ctypes.c_int64), ("n_counters", ctypes.c_int64)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libmk.so (built by bandwidth_bound_b200/build.py); raises if absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with `python bandwidth_bound_b200/build.py`")
+    lib = ctypes.CDLL(path)
+    vp, i32, u64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint64
+    sig = {
+        "mk_create": (ctypes.c_int, [ctypes.POINTER(ModelCfg), ctypes.POINTER(WeightPtrs), ctypes.POINTER(vp)]),
+        "mk_create_from_plan": (ctypes.c_int, [vp, ctypes.POINTER(WeightPtrs), i32, ctypes.POINTER(vp)]),
+        "mk_decode_step": (ctypes.c_int, [vp, vp, vp, vp, i32, ctypes.POINTER(KvCache), vp, vp, vp]),
+        "mk_decode_step_host": (ctypes.c_int, [vp, vp, vp, vp, i32, ctypes.POINTER(KvCache), vp, vp, vp]),
+        "mk_get_status": (ctypes.c_int, [vp]),
+        "mk_reset": (ctypes.c_int, [vp]),
+        "mk_set_debug": (ctypes.c_int, [vp, vp]),
+        "mk_set_timeout_ns": (ctypes.c_int, [vp, u64]),
+        "mk_launches_per_step": (ctypes.c_int, [vp]),
+        "mk_destroy": (ctypes.c_int, [vp]),
+        "mk_last_error": (ctypes.c_char_p, [vp]),
+        "mk_plan_create": (ctypes.c_int, [ctypes.POINTER(ModelCfg), ctypes.POINTER(PlanOpts), ctypes.POINTER(vp)]),
+        "mk_plan_validate": (ctypes.c_int, [vp, ctypes.c_char_p, ctypes.c_size_t]),
+        "mk_plan_stats": (ctypes.c_int, [vp, ctypes.POINTER(PlanInfo)]),
+        "mk_plan_inject_fault": (ctypes.c_int, [vp, i32, i32]),
+        "mk_plan_destroy": (None, [vp]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = lib
+    return lib
+
+
+def model_cfg(m, max_batch: int, max_ctx: int) -> ModelCfg:
+    """ModelCfg from any object with the synth.ModelConfig fields."""
+    return ModelCfg(m.n_layers, m.hidden, m.n_heads, m.n_kv_heads, m.head_dim, m.ffn, m.vocab, int(m.tied),
+                    float(m.rope_theta), float(m.rms_eps), int(max_batch), int(max_ctx), int(m.page_size))
+
+
+def _check(rc: int, handle=None, what: str = ""):
+    if rc != MK_OK:
+        lib = load_library()
+        msg = lib.mk_last_error(handle)
+        raise MkError(rc, f"{what}: {msg.decode() if msg else ''}")
+
+
+class Plan:
+    """The per-SM task schedule (host only)."""
+
+    def __init__(self, cfg: ModelCfg, num_sms: int = 0, attn_slots_per_sm: int = 0, max_blocks: int = 0):
+        self.lib = load_library()
+        self.ptr = ctypes.c_void_p()
+        opts = PlanOpts(num_sms, attn_slots_per_sm, max_blocks)
+        _check(self.lib.mk_plan_create(ctypes.byref(cfg), ctypes.byref(opts), ctypes.byref(self.ptr)),
+               None, "mk_plan_create")
+
+    def validate(self) -> tuple[int, str]:
+        buf = ctypes.create_string_buffer(512)
+        rc = self.lib.mk_plan_validate(self.ptr, buf, 512)
+        return rc, buf.value.decode()
+
+    def stats(self) -> dict:
+        info = PlanInfo()
+        _check(self.lib.mk_plan_stats(self.ptr, ctypes.byref(info)), None, "mk_plan_stats")
+        return {k: getattr(info, k) for k, _ in PlanInfo._fields_}
+
+    def inject_fault(self, kind: int, arg: int = 0) -> int:
+        return self.lib.mk_plan_inject_fault(self.ptr, kind, arg)
+
+    def close(self):
+        if self.ptr:
+            self.lib.mk_plan_destroy(self.ptr)
+            self.ptr = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def _ptr(t) -> int:
+    return 0 if t is None else int(t.data_ptr())
+
+
+class Megakernel:
+    """A handle of the decode megakernel bound to one model's device weights.
+
+    ``weights`` is a dict as built by ``synth.make_weights`` (bf16 CUDA tensors);
+    the tensors must stay alive while the handle is used.
+    """
+
+    def __init__(self, m, weights: dict, max_batch: int, max_ctx: int, plan: Optional[Plan] = None,
+                 skip_validate: bool = False):
+        import torch  # plumbing only: device pointers and streams
+
+        self.lib = load_library()
+        self.m = m
+        self.cfg = model_cfg(m, max_batch, max_ctx)
+        self.weights = weights
+        L = m.n_layers
+        arr = {}
+        for name in ("attn_norm", "wq", "wk", "wv", "wo", "mlp_norm", "w_gate", "w_up", "w_down"):
+            a = (ctypes.c_void_p * L)(*[_ptr(weights["layers"][i][name]) for i in range(L)])
+            arr[name] = a
+        self._arrays = arr
+        w = WeightPtrs(_ptr(weights["embed"]), _ptr(weights["final_norm"]), _ptr(weights["lm_head"]),
+                       *[ctypes.cast(arr[n], _PP) for n in ("attn_norm", "wq", "wk", "wv", "wo", "mlp_norm",
+                                                             "w_gate", "w_up", "w_down")])
+        self.handle = ctypes.c_void_p()
+        if plan is None:
+            rc = self.lib.mk_create(ctypes.byref(self.cfg), ctypes.byref(w), ctypes.byref(self.handle))
+        else:
+            rc = self.lib.mk_create_from_plan(plan.ptr, ctypes.byref(w),
+                                              MK_CREATE_SKIP_VALIDATE if skip_validate else 0,
+                                              ctypes.byref(self.handle))
+        _check(rc, None, "mk_create")
+        self._torch = torch
+
+    @staticmethod
+    def kv_struct(kv) -> KvCache:
+        return KvCache(_ptr(kv.k_pool), _ptr(kv.v_pool), _ptr(kv.page_table), int(kv.num_pages),
+                       int(kv.max_pages_per_seq))
+
+    def step(self, token_ids, positions, seq_lens, kv, logits, argmax=None, stream=None, check: bool = True) -> int:
+        """One decode step on device tensors (int32 token_ids/positions/seq_lens, fp32 logits)."""
+        if stream is None:
+            stream = self._torch.cuda.current_stream()
+        kvs = self.kv_struct(kv)
+        rc = self.lib.mk_decode_step(self.handle, _ptr(token_ids), _ptr(positions), _ptr(seq_lens),
+                                     int(token_ids.numel()), ctypes.byref(kvs), _ptr(logits), _ptr(argmax),
+                                     ctypes.c_void_p(stream.cuda_stream))
+        if check:
+            _check(rc, self.handle, "mk_decode_step")
+        return rc
+
+    def step_host(self, token_ids, positions, seq_lens, kv, logits_host=None, argmax_host=None, stream=None,
+                  check: bool = True) -> int:
+        """One decode step from host (CPU, ideally pinned) tensors; synchronises the stream."""
+        if stream is None:
+            stream = self._torch.cuda.current_stream()
+        kvs = self.kv_struct(kv)
+        rc = self.lib.mk_decode_step_host(self.handle, _ptr(token_ids), _ptr(positions), _ptr(seq_lens),
+                                          int(token_ids.numel()), ctypes.byref(kvs), _ptr(logits_host),
+                                          _ptr(argmax_host), ctypes.c_void_p(stream.cuda_stream))
+        if check:
+            _check(rc, self.handle, "mk_decode_step_host")
+        return rc
+
+    def status(self) -> int:
+        return self.lib.mk_get_status(self.handle)
+
+    def reset(self):
+        _check(self.lib.mk_reset(self.handle), self.handle, "mk_reset")
+
+    def set_debug(self, layer_hidden):
+        _check(self.lib.mk_set_debug(self.handle, _ptr(layer_hidden)), self.handle, "mk_set_debug")
+
+    def set_timeout_ns(self, ns: int):
+        _check(self.lib.mk_set_timeout_ns(self.handle, int(ns)), self.handle, "mk_set_timeout_ns")
+
+    def launches_per_step(self) -> int:
+        return self.lib.mk_launches_per_step(self.handle)
+
+    def last_error(self) -> str:
+        msg = self.lib.mk_last_error(self.handle)
+        return msg.decode() if msg else ""
+
+    def close(self):
+        if self.handle:
+            self.lib.mk_destroy(self.handle)
+            self.handle = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def header_functions(header: Optional[str] = None) -> list[str]:
+    """Names of the entry points include/mk.h declares (MK_API lines)."""
+    import re
+
+    header = header or os.path.join(os.path.dirname(HERE), "include", "mk.h")
+    src = open(header).read()
+    return re.findall(r"MK_API\s+[\w\s\*]*?\b(mk_\w+)\s*\(", src)

@@ -1,0 +1,313 @@
+// C ABI of the decode megakernel: handle creation, the decode step, status.
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "mk_kernel.h"
+#include "mk_plan.h"
+
+using mk::KParams;
+using mk::LayerW;
+
+struct mk_handle_s {
+  mk_plan_s plan;
+  int device = 0;
+  KParams kp{};                 // everything but the per-step fields
+  void* arena = nullptr;        // all device scratch in one allocation
+  int* host_status = nullptr;   // mapped pinned word
+  int32_t* h_stage = nullptr;   // pinned staging for the host-buffer step
+  int32_t* d_stage = nullptr;   // device copy of token ids / positions / lengths
+  float* d_logits = nullptr;    // device logits for the host-buffer step
+  int32_t* d_argmax = nullptr;
+  uint32_t epoch = 0;
+  std::string err;
+};
+
+static thread_local std::string g_err;
+extern "C" const char* mk_internal_plan_error();
+
+static int fail(mk_handle_t h, int code, const std::string& msg) {
+  if (h) h->err = msg;
+  else g_err = msg;
+  return code;
+}
+
+static int cuda_fail(mk_handle_t h, cudaError_t e, const char* what) {
+  return fail(h, MK_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+#define MK_CUDA(h, call)                                   \
+  do {                                                     \
+    cudaError_t e_ = (call);                               \
+    if (e_ != cudaSuccess) return cuda_fail(h, e_, #call); \
+  } while (0)
+
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+static void release(mk_handle_t h) {
+  if (!h) return;
+  if (h->arena) cudaFree(h->arena);
+  if (h->host_status) cudaFreeHost(h->host_status);
+  if (h->h_stage) cudaFreeHost(h->h_stage);
+  delete h;
+}
+
+extern "C" {
+
+MK_API int mk_create_from_plan(mk_plan_t plan, const mk_weight_ptrs* w, int32_t flags, mk_handle_t* out) {
+  if (!plan || !w || !out) return fail(nullptr, MK_ERR_INVALID_ARG, "mk_create: null argument");
+  const mk_model_cfg& c = plan->cfg;
+  std::string e;
+  if (!(flags & MK_CREATE_SKIP_VALIDATE)) {
+    int rc = mk::validate_plan(*plan, &e);
+    if (rc) return fail(nullptr, rc, "schedule rejected: " + e);
+  }
+  // weights
+  if (!w->embed || !w->final_norm || !w->lm_head || !w->attn_norm || !w->wq || !w->wk || !w->wv || !w->wo ||
+      !w->mlp_norm || !w->w_gate || !w->w_up || !w->w_down)
+    return fail(nullptr, MK_ERR_INVALID_ARG, "mk_create: null weight pointer");
+  std::vector<LayerW> lw(c.n_layers);
+  const void* all[3] = {w->embed, w->final_norm, w->lm_head};
+  for (const void* p : all)
+    if (!aligned16(p)) return fail(nullptr, MK_ERR_INVALID_ARG, "mk_create: weights must be 16-byte aligned");
+  for (int l = 0; l < c.n_layers; ++l) {
+    const void* ps[9] = {w->attn_norm[l], w->wq[l], w->wk[l], w->wv[l], w->wo[l],
+                         w->mlp_norm[l], w->w_gate[l], w->w_up[l], w->w_down[l]};
+    for (const void* p : ps)
+      if (!p || !aligned16(p))
+        return fail(nullptr, MK_ERR_INVALID_ARG, "mk_create: layer weight null or not 16-byte aligned");
+    lw[l] = LayerW{(const __nv_bfloat16*)ps[0], (const __nv_bfloat16*)ps[1], (const __nv_bfloat16*)ps[2],
+                   (const __nv_bfloat16*)ps[3], (const __nv_bfloat16*)ps[4], (const __nv_bfloat16*)ps[5],
+                   (const __nv_bfloat16*)ps[6], (const __nv_bfloat16*)ps[7], (const __nv_bfloat16*)ps[8]};
+  }
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(nullptr, MK_ERR_NO_DEVICE, "no CUDA device");
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return fail(nullptr, MK_ERR_NO_DEVICE, "no CUDA device");
+  if (prop.major != 10) return fail(nullptr, MK_ERR_NO_DEVICE, "the kernel is built for sm_100a (B200)");
+  if (!prop.cooperativeLaunch) return fail(nullptr, MK_ERR_NO_DEVICE, "device lacks cooperative launch");
+  if (plan->num_sms != prop.multiProcessorCount)
+    return fail(nullptr, MK_ERR_INVALID_ARG,
+                "plan built for " + std::to_string(plan->num_sms) + " SMs, device has " +
+                    std::to_string(prop.multiProcessorCount));
+
+  mk_handle_t h = new mk_handle_s();
+  h->plan = *plan;
+  h->device = dev;
+  int regs = 0, lmem = 0, maxthr = 0;
+  cudaError_t ce = mk::kernel_attributes(&regs, &lmem, &maxthr);
+  if (ce != cudaSuccess) { release(h); return cuda_fail(nullptr, ce, "kernel attributes"); }
+  if (maxthr < mk::kThreads) { release(h); return fail(nullptr, MK_ERR_CUDA, "kernel cannot run 288 threads"); }
+
+  const mk::Geometry G = mk::geometry(c);
+  const int S = plan->num_sms * plan->attn_slots_per_sm;
+  const int mb = c.max_batch;
+  // device arena layout (256-byte aligned pieces)
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off += (bytes + 255) & ~size_t(255); return o; };
+  std::vector<mk::TaskDesc> flat;
+  std::vector<uint32_t> offs(plan->num_sms + 1, 0);
+  for (int s = 0; s < plan->num_sms; ++s) {
+    flat.insert(flat.end(), plan->streams[s].begin(), plan->streams[s].end());
+    offs[s + 1] = (uint32_t)flat.size();
+  }
+  const size_t o_layers = take(sizeof(LayerW) * c.n_layers);
+  const size_t o_tasks = take(sizeof(mk::TaskDesc) * flat.size());
+  const size_t o_offs = take(sizeof(uint32_t) * offs.size());
+  const size_t o_x = take(sizeof(float) * mb * G.d);
+  const size_t o_q = take(sizeof(float) * mb * G.qdim);
+  const size_t o_attn = take(sizeof(float) * mb * G.qdim);
+  const size_t o_h = take(sizeof(float) * mb * G.F);
+  const int ssq_stride = plan->max_phase_tasks * mb;
+  const size_t o_ssq = take(sizeof(float) * mk::num_ssq_inst(G.L) * ssq_stride);
+  const size_t o_part = take(sizeof(float) * (size_t)S * G.g * (G.hd + 2));
+  const size_t o_lm = take(sizeof(float2) * (size_t)plan->n_lm_tasks * mb);
+  const size_t o_ctr = take(sizeof(uint32_t) * mk::num_counters(G.L));
+  const size_t o_cmb = take(sizeof(uint32_t) * (size_t)G.L * mb * G.nkv);
+  const size_t o_ctl = take(sizeof(uint32_t) * 2);
+  const size_t o_rope = take(sizeof(float2) * (size_t)c.max_ctx * (G.hd / 2));
+  const size_t o_stage = take(sizeof(int32_t) * 3 * mb);
+  const size_t o_logits = take(sizeof(float) * (size_t)mb * G.V);
+  const size_t o_argmax = take(sizeof(int32_t) * mb);
+  const size_t total = off;
+
+  ce = cudaMalloc(&h->arena, total);
+  if (ce != cudaSuccess) { release(h); return cuda_fail(nullptr, ce, "cudaMalloc(scratch)"); }
+  ce = cudaMemset(h->arena, 0, total);
+  if (ce == cudaSuccess) ce = cudaHostAlloc((void**)&h->host_status, sizeof(int), cudaHostAllocMapped);
+  if (ce == cudaSuccess) ce = cudaHostAlloc((void**)&h->h_stage, sizeof(int32_t) * 3 * mb, cudaHostAllocDefault);
+  if (ce != cudaSuccess) { release(h); return cuda_fail(nullptr, ce, "scratch allocation"); }
+  *h->host_status = 0;
+  int* dev_status = nullptr;
+  ce = cudaHostGetDevicePointer((void**)&dev_status, h->host_status, 0);
+  if (ce != cudaSuccess) { release(h); return cuda_fail(nullptr, ce, "cudaHostGetDevicePointer"); }
+
+  char* A = (char*)h->arena;
+  ce = cudaMemcpy(A + o_layers, lw.data(), sizeof(LayerW) * c.n_layers, cudaMemcpyHostToDevice);
+  if (ce == cudaSuccess)
+    ce = cudaMemcpy(A + o_tasks, flat.data(), sizeof(mk::TaskDesc) * flat.size(), cudaMemcpyHostToDevice);
+  if (ce == cudaSuccess)
+    ce = cudaMemcpy(A + o_offs, offs.data(), sizeof(uint32_t) * offs.size(), cudaMemcpyHostToDevice);
+  if (ce == cudaSuccess) ce = mk::launch_rope_table((float2*)(A + o_rope), c.max_ctx, G.hd, c.rope_theta, 0);
+  if (ce == cudaSuccess) ce = cudaDeviceSynchronize();
+  if (ce != cudaSuccess) { release(h); return cuda_fail(nullptr, ce, "upload"); }
+
+  KParams& k = h->kp;
+  k.L = G.L; k.d = G.d; k.nq = G.nq; k.nkv = G.nkv; k.hd = G.hd; k.F = G.F; k.V = G.V; k.g = G.g;
+  k.qdim = G.qdim; k.max_b = mb; k.max_ctx = c.max_ctx; k.eps = c.rms_eps;
+  k.layers = (const LayerW*)(A + o_layers);
+  k.embed = (const __nv_bfloat16*)w->embed;
+  k.final_norm = (const __nv_bfloat16*)w->final_norm;
+  k.lm_head = (const __nv_bfloat16*)w->lm_head;
+  k.tasks = (const mk::TaskDesc*)(A + o_tasks);
+  k.task_off = (const uint32_t*)(A + o_offs);
+  k.num_sms = plan->num_sms;
+  k.n_slots = S;
+  k.n_lm_tasks = plan->n_lm_tasks;
+  k.x = (float*)(A + o_x); k.q = (float*)(A + o_q); k.attn = (float*)(A + o_attn); k.hbuf = (float*)(A + o_h);
+  k.ssq = (float*)(A + o_ssq); k.ssq_stride = ssq_stride; k.part = (float*)(A + o_part);
+  k.lmpart = (float2*)(A + o_lm);
+  k.ctr = (uint32_t*)(A + o_ctr); k.cmb = (uint32_t*)(A + o_cmb); k.ctl = (uint32_t*)(A + o_ctl);
+  k.host_status = dev_status;
+  k.rope = (const float2*)(A + o_rope);
+  k.timeout_ns = 1000000000ull;
+  k.dbg = nullptr;
+  h->d_stage = (int32_t*)(A + o_stage);
+  h->d_logits = (float*)(A + o_logits);
+  h->d_argmax = (int32_t*)(A + o_argmax);
+  // bookkeeping for mk_reset
+  h->err.clear();
+  *out = h;
+  (void)o_ctl;
+  return MK_OK;
+}
+
+MK_API int mk_create(const mk_model_cfg* cfg, const mk_weight_ptrs* w, mk_handle_t* out) {
+  if (!cfg || !w || !out) return fail(nullptr, MK_ERR_INVALID_ARG, "mk_create: null argument");
+  int dev = 0, nsm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return fail(nullptr, MK_ERR_NO_DEVICE, "no CUDA device");
+  mk_plan_opts o{};
+  o.num_sms = nsm;
+  mk_plan_t plan = nullptr;
+  int rc = mk_plan_create(cfg, &o, &plan);
+  if (rc) return fail(nullptr, rc, std::string("plan: ") + mk_internal_plan_error());
+  rc = mk_create_from_plan(plan, w, 0, out);
+  mk_plan_destroy(plan);
+  return rc;
+}
+
+static int check_step_args(mk_handle_t h, const void* tok, const void* pos, const void* lens, int32_t batch,
+                           const mk_kv_cache* kv, const void* logits) {
+  const mk_model_cfg& c = h->plan.cfg;
+  if (!tok || !pos || !lens || !kv || !logits) return fail(h, MK_ERR_INVALID_ARG, "mk_decode_step: null argument");
+  if (batch < 1 || batch > c.max_batch)
+    return fail(h, MK_ERR_INVALID_ARG, "mk_decode_step: batch must be in [1, max_batch]");
+  if (!kv->k_pool || !kv->v_pool || !kv->page_table || kv->num_pages < 1 || kv->max_pages_per_seq < 1)
+    return fail(h, MK_ERR_INVALID_ARG, "mk_decode_step: bad kv cache description");
+  if (!aligned16(kv->k_pool) || !aligned16(kv->v_pool))
+    return fail(h, MK_ERR_INVALID_ARG, "mk_decode_step: kv pools must be 16-byte aligned");
+  int st = *(volatile int*)h->host_status;
+  if (st != 0) return fail(h, st, "mk_decode_step: a previous step failed on the device; call mk_reset");
+  return MK_OK;
+}
+
+static int launch_step(mk_handle_t h, const int32_t* tok, const int32_t* pos, const int32_t* lens, int32_t batch,
+                       const mk_kv_cache* kv, float* logits, int32_t* argmax, cudaStream_t s) {
+  KParams p = h->kp;
+  p.tok = tok; p.pos = pos; p.lens = lens; p.b = batch;
+  p.kpool = (__nv_bfloat16*)kv->k_pool; p.vpool = (__nv_bfloat16*)kv->v_pool;
+  p.ptable = kv->page_table; p.num_pages = kv->num_pages; p.mpps = kv->max_pages_per_seq;
+  p.logits = logits; p.argmax = argmax;
+  p.epoch = ++h->epoch;
+  cudaError_t e = mk::launch_decode(p, s);
+  if (e != cudaSuccess) {
+    --h->epoch;
+    return cuda_fail(h, e, "megakernel launch");
+  }
+  return MK_OK;
+}
+
+MK_API int mk_decode_step(mk_handle_t h, const int32_t* token_ids, const int32_t* positions,
+                          const int32_t* seq_lens, int32_t batch, const mk_kv_cache* kv, float* logits_out,
+                          int32_t* argmax_out, mk_stream_t stream) {
+  if (!h) return fail(nullptr, MK_ERR_INVALID_ARG, "mk_decode_step: null handle");
+  int rc = check_step_args(h, token_ids, positions, seq_lens, batch, kv, logits_out);
+  if (rc) return rc;
+  return launch_step(h, token_ids, positions, seq_lens, batch, kv, logits_out, argmax_out, (cudaStream_t)stream);
+}
+
+MK_API int mk_decode_step_host(mk_handle_t h, const int32_t* token_ids, const int32_t* positions,
+                               const int32_t* seq_lens, int32_t batch, const mk_kv_cache* kv, float* logits_host,
+                               int32_t* argmax_host, mk_stream_t stream) {
+  if (!h) return fail(nullptr, MK_ERR_INVALID_ARG, "mk_decode_step_host: null handle");
+  int rc = check_step_args(h, token_ids, positions, seq_lens, batch, kv, h->d_logits);
+  if (rc) return rc;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int mb = h->plan.cfg.max_batch;
+  // one pinned staging buffer -> one H2D copy of the three int arrays
+  std::memcpy(h->h_stage, token_ids, sizeof(int32_t) * batch);
+  std::memcpy(h->h_stage + mb, positions, sizeof(int32_t) * batch);
+  std::memcpy(h->h_stage + 2 * mb, seq_lens, sizeof(int32_t) * batch);
+  MK_CUDA(h, cudaMemcpyAsync(h->d_stage, h->h_stage, sizeof(int32_t) * 3 * mb, cudaMemcpyHostToDevice, s));
+  rc = launch_step(h, h->d_stage, h->d_stage + mb, h->d_stage + 2 * mb, batch, kv, h->d_logits,
+                   argmax_host ? h->d_argmax : nullptr, s);
+  if (rc) return rc;
+  const size_t V = (size_t)h->plan.cfg.vocab;
+  if (logits_host)
+    MK_CUDA(h, cudaMemcpyAsync(logits_host, h->d_logits, sizeof(float) * V * batch, cudaMemcpyDeviceToHost, s));
+  if (argmax_host)
+    MK_CUDA(h, cudaMemcpyAsync(argmax_host, h->d_argmax, sizeof(int32_t) * batch, cudaMemcpyDeviceToHost, s));
+  MK_CUDA(h, cudaStreamSynchronize(s));
+  int st = *(volatile int*)h->host_status;
+  if (st != 0) return fail(h, st, "mk_decode_step_host: the step failed on the device");
+  return MK_OK;
+}
+
+MK_API int mk_get_status(mk_handle_t h) {
+  if (!h) return MK_ERR_INVALID_ARG;
+  return *(volatile int*)h->host_status;
+}
+
+MK_API int mk_reset(mk_handle_t h) {
+  if (!h) return MK_ERR_INVALID_ARG;
+  MK_CUDA(h, cudaDeviceSynchronize());
+  KParams& k = h->kp;
+  MK_CUDA(h, cudaMemset(k.ctr, 0, sizeof(uint32_t) * mk::num_counters(k.L)));
+  MK_CUDA(h, cudaMemset(k.cmb, 0, sizeof(uint32_t) * (size_t)k.L * k.max_b * k.nkv));
+  MK_CUDA(h, cudaMemset(k.ctl, 0, sizeof(uint32_t) * 2));
+  MK_CUDA(h, cudaDeviceSynchronize());
+  *(volatile int*)h->host_status = 0;
+  h->epoch = 0;
+  return MK_OK;
+}
+
+MK_API int mk_set_debug(mk_handle_t h, float* layer_hidden) {
+  if (!h) return MK_ERR_INVALID_ARG;
+  h->kp.dbg = layer_hidden;
+  return MK_OK;
+}
+
+MK_API int mk_set_timeout_ns(mk_handle_t h, uint64_t ns) {
+  if (!h || ns == 0) return MK_ERR_INVALID_ARG;
+  h->kp.timeout_ns = ns;
+  return MK_OK;
+}
+
+MK_API int mk_launches_per_step(mk_handle_t h) { return h ? 1 : MK_ERR_INVALID_ARG; }
+
+MK_API int mk_destroy(mk_handle_t h) {
+  if (!h) return MK_ERR_INVALID_ARG;
+  cudaDeviceSynchronize();
+  release(h);
+  return MK_OK;
+}
+
+MK_API const char* mk_last_error(mk_handle_t h) { return h ? h->err.c_str() : g_err.c_str(); }
+
+}  // extern "C"

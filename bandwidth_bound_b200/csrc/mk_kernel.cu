@@ -1,0 +1,1080 @@
+// The decode megakernel for B200 (sm_100a): one persistent CTA per SM.
+//
+// Structure (from "ForgeMegakernel: A General Framework for Efficient
+// Auto-Regressive Model Decode Megakernels", §2.1, §2.3 and §4.1, and the
+// "Inside the megakernel serving engine" digest):
+//   * the whole decode step is one launch; each CTA walks its own host-built
+//     stream of task descriptors;
+//   * tasks wait on dependency counters in global memory (acquire loads) and
+//     signal them (release read-modify-writes) instead of grid-wide barriers;
+//   * one producer warp streams every weight tile and every prior KV page of the
+//     CTA's whole stream into a ring of shared-memory slots with cp.async.bulk
+//     (completion on mbarriers), running ahead of the activation dependencies;
+//     eight consumer warps compute from the slots.
+// B200 choices: 1-D bulk copies (no tensor maps, no multicast) of contiguous row
+// segments, evict-first L2 policy for streamed bytes, fp32 accumulation, CUDA-core
+// FMA GEMV at batch 1, mma.sync bf16 tensor cores with hi/lo-split activations
+// at batch >= 2, split-K flash-decode with QK^T on tensor cores.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "mk_kernel.h"
+
+namespace mk {
+
+typedef __nv_bfloat16 bf16;
+
+// ---------------------------------------------------------------------------------------
+// shared memory
+
+struct Smem {
+  alignas(128) uint8_t pool[kNumSlots][kSlotBytes];
+  alignas(16) float red[kRedBytes / 4];                 // GEMV cross-warp partials / attention merge
+  alignas(16) float ep[kMaxBlocks * 8][kMaxBatch];       // per-task results [row][batch]
+  alignas(16) float pw[kConsumerWarps][16 * 8];          // attention probabilities [token][head]
+  float mw[kConsumerWarps][8], lw[kConsumerWarps][8];    // attention merge state per warp
+  float corr[kConsumerWarps][8];
+  float inv_rms[kMaxBatch];
+  alignas(8) uint64_t full[kNumSlots];
+  alignas(8) uint64_t empty[kNumSlots];
+  int attn_ch, attn_n, bad, flag, flag2;
+};
+
+size_t kernel_smem_bytes() { return sizeof(Smem); }
+
+// ---------------------------------------------------------------------------------------
+// PTX helpers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t n) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(n) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, P;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                         uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+      : "memory");
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ uint64_t gtimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_relaxed(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t atom_add_acqrel(uint32_t* p, uint32_t v) {
+  uint32_t o;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(o) : "l"(p), "r"(v) : "memory");
+  return o;
+}
+__device__ __forceinline__ void cbar() {  // the consumer warps only
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+}
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// ---------------------------------------------------------------------------------------
+// errors, waits
+
+__device__ __noinline__ void raise_error(const KParams& p, int code) {
+  if (atomicCAS(reinterpret_cast<int*>(&p.ctl[1]), 0, code) == 0) {
+    *reinterpret_cast<volatile int*>(p.host_status) = code;
+    __threadfence_system();
+  }
+  atomicExch(&p.ctl[0], 1u);
+}
+
+__device__ __forceinline__ bool aborted(const KParams& p) { return ld_relaxed(&p.ctl[0]) != 0; }
+
+// Wait until the mbarrier phase of the given parity completes.  Bounded: gives up
+// (returning false) when the abort flag is set or the time limit passes.
+__device__ bool mbar_wait(const KParams& p, uint64_t* bar, uint32_t parity) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = gtimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try(bar, parity)) return true;
+    if ((it & 15) == 0) {
+      if (aborted(p)) return false;
+      if (gtimer() - t0 > p.timeout_ns) {
+        raise_error(p, -5 /* MK_ERR_DEVICE_TIMEOUT */);
+        return false;
+      }
+    }
+  }
+}
+
+// Warp-uniform variant: lane 0 waits, the result is broadcast.
+__device__ __forceinline__ bool mbar_wait_warp(const KParams& p, uint64_t* bar, uint32_t parity) {
+  int ok = 0;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(p, bar, parity) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// Wait until counter c has received count*epoch signals (wrap-around safe).
+__device__ bool wait_counter(const KParams& p, int c, uint32_t count) {
+  const uint32_t target = count * p.epoch;
+  const uint32_t* ptr = p.ctr + c;
+  if ((int32_t)(ld_acquire(ptr) - target) >= 0) return true;
+  const uint64_t t0 = gtimer();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(64);
+    if ((int32_t)(ld_acquire(ptr) - target) >= 0) return true;
+    if ((it & 15) == 0) {
+      if (aborted(p)) return false;
+      if (gtimer() - t0 > p.timeout_ns) {
+        raise_error(p, -5);
+        return false;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// work-unit geometry
+
+__device__ __forceinline__ int gemv_K_dev(const KParams& p, int op) {
+  return op == OP_OPROJ ? p.qdim : (op == OP_DOWN ? p.F : p.d);
+}
+
+// Device address of row r (0-based within the task) of a GEMV task's weight rows.
+__device__ __forceinline__ const bf16* task_row(const KParams& p, const TaskDesc& t, int r) {
+  const LayerW& w = p.layers[t.layer];
+  switch (t.op) {
+    case OP_QKV: {
+      const int u = t.u0 + (r >> 4), ru = r & 15;
+      const int per_head = p.hd >> 4;
+      const int hh = u / per_head, m = u - hh * per_head;
+      const int row = (ru < 8) ? (8 * m + ru) : (p.hd / 2 + 8 * m + ru - 8);
+      const bf16* base = hh < p.nq ? w.wq + (size_t)hh * p.hd * p.d
+                         : hh < p.nq + p.nkv ? w.wk + (size_t)(hh - p.nq) * p.hd * p.d
+                                             : w.wv + (size_t)(hh - p.nq - p.nkv) * p.hd * p.d;
+      return base + (size_t)row * p.d;
+    }
+    case OP_GATEUP: {
+      const int u = t.u0 + (r >> 4), ru = r & 15;
+      return (ru < 8 ? w.wg : w.wu) + (size_t)(8 * u + (ru & 7)) * p.d;
+    }
+    case OP_OPROJ: return w.wo + (size_t)(8 * t.u0 + r) * p.qdim;
+    case OP_DOWN: return w.wd + (size_t)(8 * t.u0 + r) * p.F;
+    default: return p.lm_head + (size_t)(8 * t.u0 + r) * p.d;
+  }
+}
+
+// Split-K attention: slot w -> (sequence, kv head, chunk), or false for an empty slot.
+struct AttnWork {
+  int i, h, c, nc, n, c0, c1;
+};
+
+__device__ bool attn_work(const KParams& p, int ch, int w, AttnWork& a) {
+  for (int i = 0; i < p.b; ++i) {
+    const int n = p.lens[i];
+    const int nc = (n + ch - 1) / ch;
+    const int cnt = p.nkv * nc;
+    if (w < cnt) {
+      a.i = i;
+      a.h = w / nc;
+      a.c = w - a.h * nc;
+      a.nc = nc;
+      a.n = n;
+      a.c0 = a.c * ch;
+      a.c1 = min(a.c0 + ch, n);
+      return true;
+    }
+    w -= cnt;
+  }
+  return false;
+}
+
+// Chunk length: the smallest multiple of 16 such that all chunks fit the slots and
+// no (sequence, kv head) has more than kMaxChunksPerSeq chunks.
+__device__ void attn_setup(const KParams& p, int* ch_out, int* n_out) {
+  long long sum = 0;
+  int mx = 1;
+  for (int i = 0; i < p.b; ++i) {
+    sum += p.lens[i];
+    mx = max(mx, p.lens[i]);
+  }
+  int ch = ((mx + 16 * kMaxChunksPerSeq - 1) / (16 * kMaxChunksPerSeq)) * 16;
+  ch = max(ch, 16);
+  const long long room = (long long)p.n_slots - (long long)p.nkv * p.b;
+  if (room > 0) {
+    long long lb = ((long long)p.nkv * sum + room - 1) / room;
+    lb = ((lb + 15) / 16) * 16;
+    if (lb > ch) { const long long cap = (long long)((mx + 15) / 16) * 16; ch = (int)(lb < cap ? lb : cap); }
+  }
+  for (;; ch += 16) {
+    long long tot = 0;
+    for (int i = 0; i < p.b; ++i) tot += (long long)p.nkv * ((p.lens[i] + ch - 1) / ch);
+    if (tot <= p.n_slots || ch >= mx) {
+      *ch_out = ch;
+      *n_out = (int)tot;
+      return;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// producer warp: streams weight rows and prior KV pages into the slot ring
+
+__device__ __forceinline__ int attn_stages(const AttnWork& a, int T) { return (a.c1 - a.c0 + T - 1) / T; }
+
+__device__ void producer(const KParams& p, Smem& sm, const TaskDesc* ts, int nt) {
+  const int lane = threadIdx.x & 31;
+  const uint64_t pol = policy_evict_first();
+  uint32_t stage = 0;
+  bool ok = true;
+  const int T = attn_stage_tokens(p.hd);
+  for (int ti = 0; ti < nt && ok; ++ti) {
+    const TaskDesc t = ts[ti];
+    if (t.op == OP_EMBED) continue;
+    if (t.op == OP_ATTN) {
+      AttnWork a;
+      if ((int)t.u0 >= sm.attn_n || !attn_work(p, sm.attn_ch, (int)t.u0, a)) continue;
+      const int newpos = a.n - 1;
+      const int nst = attn_stages(a, T);
+      const size_t head_stride = (size_t)kPage * p.hd;  // elements per (page, kv head) block
+      for (int s = 0; s < nst && ok; ++s, ++stage) {
+        const int slot = stage % kNumSlots;
+        if (!mbar_wait_warp(p, &sm.empty[slot], ((stage / kNumSlots) & 1) ^ 1)) { ok = false; break; }
+        const int t0 = a.c0 + s * T, t1 = min(t0 + T, a.c1);
+        const int tp = min(t1, newpos);  // prior entries only; the new one is read after the wait
+        // bytes of this stage
+        uint32_t bytes = tp > t0 ? (uint32_t)(tp - t0) * p.hd * 2u * 2u : 0u;
+        // validate pages first (every lane checks the same pages)
+        bool bad = false;
+        for (int pg = t0 / kPage; pg * kPage < tp; ++pg) {
+          const int id = p.ptable[a.i * p.mpps + pg];
+          if (id < 0 || id >= p.num_pages) bad = true;
+        }
+        if (bad) {
+          if (lane == 0) raise_error(p, -6 /* MK_ERR_BOUNDS */);
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          if (bytes) mbar_expect_tx(&sm.full[slot], bytes);
+          else mbar_arrive(&sm.full[slot]);
+        }
+        __syncwarp();
+        if (bytes) {
+          uint8_t* kdst = sm.pool[slot];
+          uint8_t* vdst = sm.pool[slot] + (size_t)T * p.hd * 2;
+          const int pg0 = t0 / kPage;
+          const int npg = (tp - 1) / kPage - pg0 + 1;
+          for (int k = lane; k < 2 * npg; k += 32) {
+            const int pg = pg0 + (k >> 1);
+            const int r0 = max(pg * kPage, t0), r1 = min(pg * kPage + kPage, tp);
+            const int id = p.ptable[a.i * p.mpps + pg];
+            const size_t off = (((size_t)t.layer * p.num_pages + id) * p.nkv + a.h) * head_stride +
+                               (size_t)(r0 - pg * kPage) * p.hd;
+            const uint32_t nb = (uint32_t)(r1 - r0) * p.hd * 2u;
+            if (k & 1) bulk_g2s(vdst + (size_t)(r0 - t0) * p.hd * 2, p.vpool + off, nb, &sm.full[slot], pol);
+            else bulk_g2s(kdst + (size_t)(r0 - t0) * p.hd * 2, p.kpool + off, nb, &sm.full[slot], pol);
+          }
+        }
+      }
+      continue;
+    }
+    // GEMV task
+    const int K = gemv_K_dev(p, t.op);
+    const int kc = t.kc;
+    const int R = t.nunits * rows_per_unit(t.op);
+    const uint32_t pitch = stage_pitch(kc);
+    const int nst = (K + kc - 1) / kc;
+    for (int s = 0; s < nst; ++s, ++stage) {
+      const int slot = stage % kNumSlots;
+      if (!mbar_wait_warp(p, &sm.empty[slot], ((stage / kNumSlots) & 1) ^ 1)) { ok = false; break; }
+      const int kc0 = s * kc;
+      const int kcl = min(kc, K - kc0);
+      const uint32_t rb = (uint32_t)kcl * 2u;
+      if (lane == 0) mbar_expect_tx(&sm.full[slot], rb * (uint32_t)R);
+      __syncwarp();
+      for (int r = lane; r < R; r += 32)
+        bulk_g2s(sm.pool[slot] + (size_t)r * pitch, task_row(p, t, r) + kc0, rb, &sm.full[slot], pol);
+    }
+  }
+  if (!ok) {
+    // Drain: let every copy already issued land before the CTA may exit.
+    if (lane == 0) {
+      const uint32_t first = stage > (uint32_t)kNumSlots ? stage - kNumSlots : 0u;
+      for (uint32_t s = first; s < stage; ++s) {
+        const uint64_t t0 = gtimer();
+        while (!mbar_try(&sm.full[s % kNumSlots], (s / kNumSlots) & 1))
+          if (gtimer() - t0 > p.timeout_ns) break;
+      }
+    }
+    __syncwarp();
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// consumer helpers
+
+// 1/rms of each batch row from the partial sums of squares of instance `inst`.
+__device__ void compute_inv_rms(const KParams& p, Smem& sm, int inst, int nparts) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float* base = p.ssq + (size_t)inst * p.ssq_stride;
+  for (int bi = warp; bi < p.b; bi += kConsumerWarps) {
+    float s = 0.f;
+    for (int k = lane; k < nparts; k += 32) s += __ldcg(base + (size_t)k * p.max_b + bi);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) sm.inv_rms[bi] = 1.0f / sqrtf(s / (float)p.d + p.eps);
+  }
+}
+
+// Load 8 consecutive activations [k, k+8) of batch row bi, optionally RMS-normalised.
+__device__ __forceinline__ void load_act8(const float* src, int ld, int bi, int k, const float* inv_rms,
+                                          const bf16* gain, float (&a)[8]) {
+  const float* s = src + (size_t)bi * ld + k;
+  const float4 v0 = __ldcg(reinterpret_cast<const float4*>(s));
+  const float4 v1 = __ldcg(reinterpret_cast<const float4*>(s + 4));
+  a[0] = v0.x; a[1] = v0.y; a[2] = v0.z; a[3] = v0.w;
+  a[4] = v1.x; a[5] = v1.y; a[6] = v1.z; a[7] = v1.w;
+  if (gain) {
+    const uint4 gv = __ldg(reinterpret_cast<const uint4*>(gain + k));
+    const float r = inv_rms[bi];
+    a[0] *= r * bf_lo(gv.x); a[1] *= r * bf_hi(gv.x);
+    a[2] *= r * bf_lo(gv.y); a[3] *= r * bf_hi(gv.y);
+    a[4] *= r * bf_lo(gv.z); a[5] *= r * bf_hi(gv.z);
+    a[6] *= r * bf_lo(gv.w); a[7] *= r * bf_hi(gv.w);
+  }
+}
+
+// Stream the task's stages through the warps and reduce into sm.ep[row][batch].
+// MT = 0: CUDA-core FMA (batch 1); MT = 1, 2: mma.sync with MT tiles of 8 batch rows,
+// each row split into bf16 hi + lo parts (rows 0-7 hi, 8-15 lo of the M = 16 tile).
+template <int MT>
+__device__ void gemv_body(const KParams& p, Smem& sm, const TaskDesc& t, uint32_t& stage, bool& ab,
+                          const float* src, int ld, const bf16* gain) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, tq = lane & 3;
+  const int K = gemv_K_dev(p, t.op);
+  const int kc = t.kc;
+  const int G = t.nunits * rows_per_unit(t.op) / 8;
+  const uint32_t pitch = stage_pitch(kc);
+  const int nst = (K + kc - 1) / kc;
+  const float* inv = sm.inv_rms;
+
+  constexpr int NACC = MT == 0 ? 1 : MT * 4;
+  float acc[kMaxBlocks][NACC];
+#pragma unroll
+  for (int j = 0; j < kMaxBlocks; ++j)
+#pragma unroll
+    for (int e = 0; e < NACC; ++e) acc[j][e] = 0.f;
+
+  for (int s = 0; s < nst; ++s, ++stage) {
+    const int slot = stage % kNumSlots;
+    if (!ab) ab = !mbar_wait_warp(p, &sm.full[slot], (stage / kNumSlots) & 1);
+    if (ab) continue;
+    const uint8_t* tile = sm.pool[slot];
+    const int kc0 = s * kc;
+    const int kcl = min(kc, K - kc0);
+    const int nb = (kcl + 31) >> 5;
+    for (int kb = warp; kb < nb; kb += kConsumerWarps) {
+      const int kofs = kb * 32 + tq * 8;
+      const bool valid = kofs < kcl;
+      const int k = kc0 + kofs;
+      if constexpr (MT == 0) {
+        float a[8];
+        if (valid) load_act8(src, ld, 0, k, inv, gain, a);
+        else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) a[e] = 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < kMaxBlocks; ++j) {
+          if (j < G) {
+            uint4 w = make_uint4(0, 0, 0, 0);
+            if (valid) w = *reinterpret_cast<const uint4*>(tile + (size_t)(8 * j + g) * pitch + kofs * 2);
+            float s0 = acc[j][0];
+            s0 = fmaf(bf_lo(w.x), a[0], s0); s0 = fmaf(bf_hi(w.x), a[1], s0);
+            s0 = fmaf(bf_lo(w.y), a[2], s0); s0 = fmaf(bf_hi(w.y), a[3], s0);
+            s0 = fmaf(bf_lo(w.z), a[4], s0); s0 = fmaf(bf_hi(w.z), a[5], s0);
+            s0 = fmaf(bf_lo(w.w), a[6], s0); s0 = fmaf(bf_hi(w.w), a[7], s0);
+            acc[j][0] = s0;
+          }
+        }
+      } else {
+        uint32_t A[MT][8];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          const int bi = mt * 8 + g;
+          float a[8];
+          if (valid && bi < p.b) load_act8(src, ld, bi, k, inv, gain, a);
+          else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) a[e] = 0.f;
+          }
+          float hi[8], lo[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            hi[e] = __bfloat162float(__float2bfloat16_rn(a[e]));
+            lo[e] = a[e] - hi[e];
+          }
+          // step 0: logical k (2t,2t+1) <- actual +0,+1 ; (2t+8,2t+9) <- +2,+3 ; step 1: +4..+7
+          A[mt][0] = pack_bf16(hi[0], hi[1]); A[mt][1] = pack_bf16(lo[0], lo[1]);
+          A[mt][2] = pack_bf16(hi[2], hi[3]); A[mt][3] = pack_bf16(lo[2], lo[3]);
+          A[mt][4] = pack_bf16(hi[4], hi[5]); A[mt][5] = pack_bf16(lo[4], lo[5]);
+          A[mt][6] = pack_bf16(hi[6], hi[7]); A[mt][7] = pack_bf16(lo[6], lo[7]);
+        }
+#pragma unroll
+        for (int j = 0; j < kMaxBlocks; ++j) {
+          if (j < G) {
+            uint4 w = make_uint4(0, 0, 0, 0);
+            if (valid) w = *reinterpret_cast<const uint4*>(tile + (size_t)(8 * j + g) * pitch + kofs * 2);
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+              float(&d)[4] = *reinterpret_cast<float(*)[4]>(&acc[j][mt * 4]);
+              mma_bf16(d, A[mt][0], A[mt][1], A[mt][2], A[mt][3], w.x, w.y);
+              mma_bf16(d, A[mt][4], A[mt][5], A[mt][6], A[mt][7], w.z, w.w);
+            }
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.empty[slot]);
+  }
+
+  // cross-warp reduction: red[warp][block][batch][8 rows]
+  float* red = sm.red;
+  if (!ab) {
+#pragma unroll
+    for (int j = 0; j < kMaxBlocks; ++j) {
+      if (j < G) {
+        if constexpr (MT == 0) {
+          float v = acc[j][0];
+          v += __shfl_xor_sync(0xffffffffu, v, 1);
+          v += __shfl_xor_sync(0xffffffffu, v, 2);
+          if (tq == 0) red[((warp * kMaxBlocks + j) * kMaxBatch + 0) * 8 + g] = v;
+        } else {
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+            const int bi = mt * 8 + g;
+            float2 y = make_float2(acc[j][mt * 4 + 0] + acc[j][mt * 4 + 2], acc[j][mt * 4 + 1] + acc[j][mt * 4 + 3]);
+            *reinterpret_cast<float2*>(&red[((warp * kMaxBlocks + j) * kMaxBatch + bi) * 8 + 2 * tq]) = y;
+          }
+        }
+      }
+    }
+  }
+  cbar();
+  const int nb_items = G * 8 * p.b;
+  for (int idx = threadIdx.x; idx < nb_items; idx += kConsumerWarps * 32) {
+    const int bi = idx % p.b;
+    const int row = idx / p.b;  // 8*j + r
+    const int j = row >> 3, r = row & 7;
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) s += red[((w * kMaxBlocks + j) * kMaxBatch + bi) * 8 + r];
+    sm.ep[row][bi] = s;
+  }
+  cbar();
+}
+
+__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
+
+// ---------------------------------------------------------------------------------------
+// consumer task bodies
+
+__device__ void gemv_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_t& stage, bool& ab) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const LayerW& W = p.layers[t.layer];
+  const float* src;
+  int ld;
+  const bf16* gain = nullptr;
+  switch (t.op) {
+    case OP_QKV: src = p.x; ld = p.d; gain = W.attn_norm; break;
+    case OP_GATEUP: src = p.x; ld = p.d; gain = W.mlp_norm; break;
+    case OP_LMHEAD: src = p.x; ld = p.d; gain = p.final_norm; break;
+    case OP_OPROJ: src = p.attn; ld = p.qdim; break;
+    default: src = p.hbuf; ld = p.F; break;
+  }
+  if (gain && !ab) {
+    const int inst = t.op == OP_GATEUP ? ssq_inst_oproj(t.layer)
+                     : t.op == OP_QKV  ? (t.layer == 0 ? ssq_inst_embed() : ssq_inst_down(t.layer - 1))
+                                       : ssq_inst_down(p.L - 1);
+    compute_inv_rms(p, sm, inst, (int)t.wait_count);
+  }
+  cbar();
+  if (p.b == 1) gemv_body<0>(p, sm, t, stage, ab, src, ld, gain);
+  else if (p.b <= 8) gemv_body<1>(p, sm, t, stage, ab, src, ld, gain);
+  else gemv_body<2>(p, sm, t, stage, ab, src, ld, gain);
+
+  const int G = t.nunits * rows_per_unit(t.op) / 8;
+  const int nthr = kConsumerWarps * 32;
+  if (t.op == OP_QKV) {
+    if (!ab) {
+      const int half = p.hd / 2, per_head = p.hd >> 4;
+      const int items = t.nunits * 8 * p.b;
+      for (int idx = threadIdx.x; idx < items; idx += nthr) {
+        const int bi = idx % p.b;
+        const int ur = idx / p.b;
+        const int ul = ur >> 3, r = ur & 7;
+        const int u = t.u0 + ul;
+        const int hh = u / per_head, m = u - hh * per_head;
+        const int j = 8 * m + r;
+        const float x1 = sm.ep[(2 * ul) * 8 + r][bi];
+        const float x2 = sm.ep[(2 * ul + 1) * 8 + r][bi];
+        const int pos = p.pos[bi];
+        if (hh < p.nq + p.nkv) {
+          const float2 cs = p.rope[(size_t)pos * half + j];
+          const float o1 = x1 * cs.x - x2 * cs.y;
+          const float o2 = x2 * cs.x + x1 * cs.y;
+          if (hh < p.nq) {
+            float* qd = p.q + (size_t)bi * p.qdim + (size_t)hh * p.hd;
+            qd[j] = o1;
+            qd[j + half] = o2;
+          } else {
+            const int page = p.ptable[bi * p.mpps + pos / kPage];
+            bf16* kd = p.kpool + ((((size_t)t.layer * p.num_pages + page) * p.nkv + (hh - p.nq)) * kPage +
+                                  pos % kPage) * p.hd;
+            kd[j] = __float2bfloat16_rn(o1);
+            kd[j + half] = __float2bfloat16_rn(o2);
+          }
+        } else {
+          const int page = p.ptable[bi * p.mpps + pos / kPage];
+          bf16* vd = p.vpool + ((((size_t)t.layer * p.num_pages + page) * p.nkv + (hh - p.nq - p.nkv)) * kPage +
+                                pos % kPage) * p.hd;
+          vd[j] = __float2bfloat16_rn(x1);
+          vd[j + half] = __float2bfloat16_rn(x2);
+        }
+      }
+    }
+  } else if (t.op == OP_GATEUP) {
+    if (!ab) {
+      const int items = t.nunits * 8 * p.b;
+      for (int idx = threadIdx.x; idx < items; idx += nthr) {
+        const int bi = idx % p.b;
+        const int ur = idx / p.b;
+        const int ul = ur >> 3, r = ur & 7;
+        const float gv = sm.ep[(2 * ul) * 8 + r][bi];
+        const float uv = sm.ep[(2 * ul + 1) * 8 + r][bi];
+        p.hbuf[(size_t)bi * p.F + 8 * (t.u0 + ul) + r] = silu_f(gv) * uv;
+      }
+    }
+  } else if (t.op == OP_OPROJ || t.op == OP_DOWN) {
+    const int inst = t.op == OP_OPROJ ? ssq_inst_oproj(t.layer) : ssq_inst_down(t.layer);
+    if (!ab) {
+      const int items = G * 8 * p.b;
+      float* dbg = (t.op == OP_DOWN && p.dbg) ? p.dbg + (size_t)(t.layer + 1) * p.max_b * p.d : nullptr;
+      for (int idx = threadIdx.x; idx < items; idx += nthr) {
+        const int bi = idx % p.b;
+        const int row = idx / p.b;
+        const int grow = 8 * t.u0 + row;
+        float* xp = p.x + (size_t)bi * p.d + grow;
+        const float xn = __ldcg(xp) + sm.ep[row][bi];
+        *xp = xn;
+        sm.ep[row][bi] = xn;
+        if (dbg) dbg[(size_t)bi * p.d + grow] = xn;
+      }
+    }
+    cbar();
+    if (!ab) {
+      for (int bi = warp; bi < p.b; bi += kConsumerWarps) {
+        float s = 0.f;
+        for (int row = lane; row < G * 8; row += 32) s += sm.ep[row][bi] * sm.ep[row][bi];
+#pragma unroll
+        for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == 0) p.ssq[(size_t)inst * p.ssq_stride + (size_t)t.task_idx * p.max_b + bi] = s;
+      }
+    }
+  } else {  // LM head
+    if (!ab) {
+      const int items = G * 8 * p.b;
+      for (int idx = threadIdx.x; idx < items; idx += nthr) {
+        const int bi = idx % p.b;
+        const int row = idx / p.b;
+        p.logits[(size_t)bi * p.V + 8 * t.u0 + row] = sm.ep[row][bi];
+      }
+      if (p.argmax) {
+        for (int bi = warp; bi < p.b; bi += kConsumerWarps) {
+          float best = -INFINITY;
+          int bidx = 0x7fffffff;
+          for (int row = lane; row < G * 8; row += 32) {
+            const float v = sm.ep[row][bi];
+            if (v > best) { best = v; bidx = 8 * t.u0 + row; }
+          }
+#pragma unroll
+          for (int o = 16; o; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, best, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bidx, o);
+            if (ov > best || (ov == best && oi < bidx)) { best = ov; bidx = oi; }
+          }
+          if (lane == 0) p.lmpart[(size_t)t.task_idx * p.max_b + bi] = make_float2(best, __int_as_float(bidx));
+        }
+      }
+    }
+  }
+}
+
+__device__ void embed_task(const KParams& p, Smem& sm, const TaskDesc& t, bool ab) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (ab) return;
+  const int c0 = 8 * t.u0, nc = 8 * t.nunits;
+  for (int bi = warp; bi < p.b; bi += kConsumerWarps) {
+    const bf16* e = p.embed + (size_t)p.tok[bi] * p.d;
+    float s = 0.f;
+    for (int c = lane; c < nc; c += 32) {
+      const float v = __bfloat162float(e[c0 + c]);
+      p.x[(size_t)bi * p.d + c0 + c] = v;
+      if (p.dbg) p.dbg[(size_t)bi * p.d + c0 + c] = v;
+      s += v * v;
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) p.ssq[(size_t)ssq_inst_embed() * p.ssq_stride + (size_t)t.task_idx * p.max_b + bi] = s;
+  }
+}
+
+// One split-K chunk of GQA decode attention for (sequence i, kv head h): QK^T on
+// tensor cores (A = keys from the slot, B = the g query heads as bf16 hi/lo pairs),
+// an online softmax per warp in the log2 domain, PV on CUDA cores, a merge of the
+// eight warps, and - for the last chunk of (i, h) to finish - the log-sum-exp
+// combine of all chunks into the attention output.
+template <int HD>
+__device__ void attn_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_t& stage, bool& ab) {
+  constexpr int T = HD == 64 ? 128 : 64;   // tokens per stage
+  constexpr int TPW = T / kConsumerWarps;  // tokens per warp per stage: 16 or 8
+  constexpr int NKB = HD / 32;             // 32-dim blocks
+  constexpr int DPL = HD / 32;             // dims per lane in PV
+  constexpr int NT = HD == 64 ? 2 : 1;     // n-tiles of 4 heads
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g_ = lane >> 2, tq = lane & 3;
+  AttnWork a;
+  const bool has = (int)t.u0 < sm.attn_n && attn_work(p, sm.attn_ch, (int)t.u0, a);
+  if (!has) return;  // empty slot: no stages, nothing to merge
+  const int G = p.g;
+  const int newpos = a.n - 1;
+  const float sc = 1.4426950408889634f / sqrtf((float)HD);
+
+  // q fragments (B operand): column g_ = head (g_ & 3) of the n-tile, part g_ >> 2 (hi, lo)
+  uint32_t qf[NT][NKB][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int hq = nt * 4 + (g_ & 3);
+    const bool lo = g_ >= 4;
+#pragma unroll
+    for (int kb = 0; kb < NKB; ++kb) {
+      float v[8];
+      if (hq < G && !ab) {
+        const float* qs = p.q + (size_t)a.i * p.qdim + (size_t)(a.h * G + hq) * HD + kb * 32 + tq * 8;
+        const float4 v0 = __ldcg(reinterpret_cast<const float4*>(qs));
+        const float4 v1 = __ldcg(reinterpret_cast<const float4*>(qs + 4));
+        v[0] = v0.x; v[1] = v0.y; v[2] = v0.z; v[3] = v0.w; v[4] = v1.x; v[5] = v1.y; v[6] = v1.z; v[7] = v1.w;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = 0.f;
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float hi = __bfloat162float(__float2bfloat16_rn(v[e]));
+        v[e] = lo ? v[e] - hi : hi;
+      }
+      qf[nt][kb][0] = pack_bf16(v[0], v[1]);
+      qf[nt][kb][1] = pack_bf16(v[2], v[3]);
+      qf[nt][kb][2] = pack_bf16(v[4], v[5]);
+      qf[nt][kb][3] = pack_bf16(v[6], v[7]);
+    }
+  }
+
+  float m_st[NT][2], l_st[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    m_st[nt][0] = m_st[nt][1] = -INFINITY;
+    l_st[nt][0] = l_st[nt][1] = 0.f;
+  }
+  float acc[8][DPL];
+#pragma unroll
+  for (int h = 0; h < 8; ++h)
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) acc[h][e] = 0.f;
+
+  const int nst = attn_stages(a, T);
+  for (int s = 0; s < nst; ++s, ++stage) {
+    const int slot = stage % kNumSlots;
+    const int t0 = a.c0 + s * T, t1 = min(t0 + T, a.c1);
+    const int ntok = t1 - t0;
+    const bool has_new = newpos >= t0 && newpos < t1;
+    if (!ab) ab = !mbar_wait_warp(p, &sm.full[slot], (stage / kNumSlots) & 1);
+    uint8_t* kreg = sm.pool[slot];
+    uint8_t* vreg = sm.pool[slot] + (size_t)T * HD * 2;
+    if (has_new) {
+      // the new token's K/V were written by this layer's QKV tasks: read them now
+      if (warp == 0 && !ab) {
+        const int page = p.ptable[a.i * p.mpps + newpos / kPage];
+        const size_t off = ((((size_t)t.layer * p.num_pages + page) * p.nkv + a.h) * kPage + newpos % kPage) * HD;
+        constexpr int CH = HD * 2 / 16;  // 16-byte chunks per row
+        if (lane < 2 * CH) {
+          const int c = lane % CH;
+          const bf16* srcp = (lane < CH ? p.kpool : p.vpool) + off + c * 8;
+          const uint4 v = __ldcg(reinterpret_cast<const uint4*>(srcp));
+          uint8_t* dst = (lane < CH ? kreg : vreg) + (size_t)(newpos - t0) * HD * 2 + c * 16;
+          *reinterpret_cast<uint4*>(dst) = v;
+        }
+        fence_proxy_async_smem();
+      }
+      cbar();
+    }
+    if (!ab) {
+      const int tokA = warp * TPW + g_;
+      const int tokB = warp * TPW + 8 + g_;
+      const bool vA = tokA < ntok;
+      const bool vB = TPW == 16 && tokB < ntok;
+      const int nw = max(0, min(TPW, ntok - warp * TPW));  // this warp's tokens
+      if (nw > 0) {
+        float sacc[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
+#pragma unroll
+        for (int kb = 0; kb < NKB; ++kb) {
+          uint4 ka = make_uint4(0, 0, 0, 0), kbv = make_uint4(0, 0, 0, 0);
+          if (vA) ka = *reinterpret_cast<const uint4*>(kreg + (size_t)tokA * HD * 2 + kb * 64 + tq * 16);
+          if (vB) kbv = *reinterpret_cast<const uint4*>(kreg + (size_t)tokB * HD * 2 + kb * 64 + tq * 16);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            mma_bf16(sacc[nt], ka.x, kbv.x, ka.y, kbv.y, qf[nt][kb][0], qf[nt][kb][1]);
+            mma_bf16(sacc[nt], ka.z, kbv.z, ka.w, kbv.w, qf[nt][kb][2], qf[nt][kb][3]);
+          }
+        }
+        // scores: lanes tq<2 hold hi columns, tq>=2 the lo columns of the same heads
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          float sv[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sv[e] = sacc[nt][e] + __shfl_xor_sync(0xffffffffu, sacc[nt][e], 2);
+#pragma unroll
+          for (int hs = 0; hs < 2; ++hs) {
+            const int hq = nt * 4 + 2 * (tq & 1) + hs;
+            const bool hv = hq < G;
+            float sA = (vA && hv) ? sv[hs] * sc : -INFINITY;
+            float sB = (vB && hv) ? sv[2 + hs] * sc : -INFINITY;
+            float mx = fmaxf(sA, sB);
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            const float mo = m_st[nt][hs];
+            const float mn = fmaxf(mo, mx);
+            float corr = 1.f, pA = 0.f, pB = 0.f;
+            if (mn != -INFINITY) {
+              corr = exp2f(mo - mn);
+              pA = exp2f(sA - mn);
+              pB = exp2f(sB - mn);
+            }
+            float ls = pA + pB;
+            ls += __shfl_xor_sync(0xffffffffu, ls, 4);
+            ls += __shfl_xor_sync(0xffffffffu, ls, 8);
+            ls += __shfl_xor_sync(0xffffffffu, ls, 16);
+            m_st[nt][hs] = mn;
+            l_st[nt][hs] = l_st[nt][hs] * corr + ls;
+            if (tq < 2 && hq < 8) {
+              sm.pw[warp][g_ * 8 + hq] = pA;
+              if (TPW == 16) sm.pw[warp][(8 + g_) * 8 + hq] = pB;
+              if (g_ == 0) sm.corr[warp][hq] = corr;
+            }
+          }
+        }
+        __syncwarp();
+        // PV: lane owns dims lane*DPL .. +DPL-1
+#pragma unroll
+        for (int h = 0; h < 8; ++h) {
+          if (h < G) {
+            const float c = sm.corr[warp][h];
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) acc[h][e] *= c;
+          }
+        }
+        for (int tk = 0; tk < nw; ++tk) {
+          const uint8_t* vr = vreg + (size_t)(warp * TPW + tk) * HD * 2 + lane * DPL * 2;
+          float vv[DPL];
+          if constexpr (DPL == 4) {
+            const uint2 u = *reinterpret_cast<const uint2*>(vr);
+            vv[0] = bf_lo(u.x); vv[1] = bf_hi(u.x); vv[2] = bf_lo(u.y); vv[3] = bf_hi(u.y);
+          } else {
+            const uint32_t u = *reinterpret_cast<const uint32_t*>(vr);
+            vv[0] = bf_lo(u); vv[1] = bf_hi(u);
+          }
+          const float4 p0 = *reinterpret_cast<const float4*>(&sm.pw[warp][tk * 8]);
+          const float4 p1 = *reinterpret_cast<const float4*>(&sm.pw[warp][tk * 8 + 4]);
+          const float pr[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+          for (int h = 0; h < 8; ++h) {
+            if (h < G) {
+#pragma unroll
+              for (int e = 0; e < DPL; ++e) acc[h][e] = fmaf(pr[h], vv[e], acc[h][e]);
+            }
+          }
+        }
+        __syncwarp();
+      }
+    }
+    __syncwarp();
+    if (!ab && lane == 0) mbar_arrive(&sm.empty[slot]);
+  }
+
+  // merge the eight warps' (m, l, acc) states: red[warp][head][HD]
+  if (!ab) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int hs = 0; hs < 2; ++hs) {
+        const int hq = nt * 4 + 2 * (tq & 1) + hs;
+        if (g_ == 0 && tq < 2 && hq < 8) {
+          sm.mw[warp][hq] = m_st[nt][hs];
+          sm.lw[warp][hq] = l_st[nt][hs];
+        }
+      }
+#pragma unroll
+    for (int h = 0; h < 8; ++h)
+      if (h < G)
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) sm.red[(warp * 8 + h) * HD + lane * DPL + e] = acc[h][e];
+  }
+  cbar();
+  float* part = p.part + (size_t)t.u0 * G * (HD + 2);
+  if (!ab) {
+    for (int idx = threadIdx.x; idx < G * HD; idx += kConsumerWarps * 32) {
+      const int h = idx / HD, dd = idx % HD;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm.mw[w][h]);
+      float A = 0.f, Ls = 0.f;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        const float f = sm.mw[w][h] == -INFINITY ? 0.f : exp2f(sm.mw[w][h] - M);
+        A += f * sm.red[(w * 8 + h) * HD + dd];
+        Ls += f * sm.lw[w][h];
+      }
+      part[h * (HD + 2) + dd] = A;
+      if (dd == 0) {
+        part[h * (HD + 2) + HD] = M;
+        part[h * (HD + 2) + HD + 1] = Ls;
+      }
+    }
+  }
+  cbar();
+  if (threadIdx.x == 0) {
+    int last = 0;
+    if (!ab) {
+      __threadfence();
+      uint32_t* cc = p.cmb + ((size_t)t.layer * p.max_b + a.i) * p.nkv + a.h;
+      const uint32_t old = atom_add_acqrel(cc, 1u);
+      last = (old + 1u == (uint32_t)a.nc) ? 1 : 0;
+      if (last) *cc = 0u;  // ready for the next step (every chunk of (i, h) has arrived)
+    }
+    sm.flag2 = last;
+  }
+  cbar();
+  if (sm.flag2) {
+    // log-sum-exp combine of the nc chunk states of (i, h)
+    const float* base = p.part + (size_t)(t.u0 - a.c) * G * (HD + 2);
+    for (int idx = threadIdx.x; idx < G * HD; idx += kConsumerWarps * 32) {
+      const int h = idx / HD, dd = idx % HD;
+      float M = -INFINITY;
+      for (int c = 0; c < a.nc; ++c) M = fmaxf(M, __ldcg(base + ((size_t)c * G + h) * (HD + 2) + HD));
+      float num = 0.f, den = 0.f;
+      for (int c = 0; c < a.nc; ++c) {
+        const float* pc = base + ((size_t)c * G + h) * (HD + 2);
+        const float f = exp2f(__ldcg(pc + HD) - M);
+        num += f * __ldcg(pc + dd);
+        den += f * __ldcg(pc + HD + 1);
+      }
+      p.attn[(size_t)a.i * p.qdim + (size_t)(a.h * G + h) * HD + dd] = num / den;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// consumer warps: walk the stream
+
+__device__ void consumer(const KParams& p, Smem& sm, const TaskDesc* ts, int nt) {
+  uint32_t stage = 0;
+  bool ab = false;
+  for (int ti = 0; ti < nt; ++ti) {
+    const TaskDesc t = ts[ti];
+    // dependency wait: one thread polls, the others wait at the consumer barrier
+    if (threadIdx.x == 0) {
+      bool ok = !ab;
+      if (ok && t.wait_ctr != kNoCounter) ok = wait_counter(p, t.wait_ctr, t.wait_count);
+      sm.flag = ok ? 0 : 1;
+    }
+    cbar();
+    ab = ab || sm.flag;
+    switch (t.op) {
+      case OP_EMBED: embed_task(p, sm, t, ab); break;
+      case OP_ATTN:
+        if (p.hd == 64) attn_task<64>(p, sm, t, stage, ab);
+        else attn_task<128>(p, sm, t, stage, ab);
+        break;
+      default: gemv_task(p, sm, t, stage, ab); break;
+    }
+    cbar();
+    if (threadIdx.x == 0) {
+      if (!ab) {
+        __threadfence();
+        const uint32_t old = atom_add_acqrel(p.ctr + t.sig_ctr, 1u);
+        sm.flag = (t.op == OP_LMHEAD && p.argmax && old + 1u == (uint32_t)p.n_lm_tasks * p.epoch) ? 1 : 0;
+      } else {
+        sm.flag = 0;
+      }
+    }
+    cbar();
+    if (sm.flag) {
+      // the last LM-head task of the step reduces the per-task argmax candidates
+      const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+      for (int bi = warp; bi < p.b; bi += kConsumerWarps) {
+        float best = -INFINITY;
+        int bidx = 0x7fffffff;
+        for (int k = lane; k < p.n_lm_tasks; k += 32) {
+          const float2 c = __ldcg(p.lmpart + (size_t)k * p.max_b + bi);
+          const int ci = __float_as_int(c.y);
+          if (c.x > best || (c.x == best && ci < bidx)) { best = c.x; bidx = ci; }
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, best, o);
+          const int oi = __shfl_xor_sync(0xffffffffu, bidx, o);
+          if (ov > best || (ov == best && oi < bidx)) { best = ov; bidx = oi; }
+        }
+        if (lane == 0) p.argmax[bi] = bidx;
+      }
+    }
+    cbar();
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// the kernel
+
+__global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_constant__ KParams p) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kNumSlots; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], kConsumerWarps);
+    }
+    fence_mbar_init();
+    // scalar input checks (page ids are checked where they are used)
+    int bad = 0;
+    for (int i = 0; i < p.b; ++i) {
+      const int tk = p.tok[i], ps = p.pos[i], ln = p.lens[i];
+      if (tk < 0 || tk >= p.V || ps < 0 || ps >= p.max_ctx || ln != ps + 1 || ps / kPage >= p.mpps) bad = 1;
+      else {
+        const int pg = p.ptable[i * p.mpps + ps / kPage];
+        if (pg < 0 || pg >= p.num_pages) bad = 1;
+      }
+    }
+    if (bad) raise_error(p, -6 /* MK_ERR_BOUNDS */);
+    sm.bad = bad;
+    if (!bad) attn_setup(p, &sm.attn_ch, &sm.attn_n);
+  }
+  __syncthreads();
+  if (sm.bad) return;
+  const uint32_t o0 = p.task_off[blockIdx.x], o1 = p.task_off[blockIdx.x + 1];
+  if ((threadIdx.x >> 5) == kConsumerWarps) producer(p, sm, p.tasks + o0, (int)(o1 - o0));
+  else consumer(p, sm, p.tasks + o0, (int)(o1 - o0));
+}
+
+// RoPE table: (cos, sin) of pos * theta^(-2j/hd), computed in double, stored as fp32.
+__global__ void rope_table_kernel(float2* table, int max_ctx, int hd, double theta) {
+  const int half = hd / 2;
+  const long long n = (long long)max_ctx * half;
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < n;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const int pos = (int)(idx / half), j = (int)(idx % half);
+    const double inv = pow(theta, -2.0 * j / hd);
+    double sn, cs;
+    sincos((double)pos * inv, &sn, &cs);
+    table[idx] = make_float2((float)cs, (float)sn);
+  }
+}
+
+cudaError_t launch_decode(const KParams& p, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.num_sms);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = sizeof(Smem);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;  // co-residency of all CTAs (no grid sync is used)
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, mk_decode_kernel, p);
+}
+
+cudaError_t launch_rope_table(float2* table, int max_ctx, int hd, double theta, cudaStream_t s) {
+  rope_table_kernel<<<256, 256, 0, s>>>(table, max_ctx, hd, theta);
+  return cudaGetLastError();
+}
+
+cudaError_t kernel_attributes(int* regs, int* local_bytes, int* max_threads) {
+  cudaError_t e = cudaFuncSetAttribute(mk_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)sizeof(Smem));
+  if (e != cudaSuccess) return e;
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, mk_decode_kernel);
+  if (e != cudaSuccess) return e;
+  if (regs) *regs = fa.numRegs;
+  if (local_bytes) *local_bytes = (int)fa.localSizeBytes;
+  if (max_threads) *max_threads = fa.maxThreadsPerBlock;
+  return cudaSuccess;
+}
+
+}  // namespace mk

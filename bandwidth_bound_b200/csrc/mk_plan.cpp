@@ -1,0 +1,557 @@
+// Per-SM instruction streams for the decode megakernel, and their static validator.
+//
+// The pages' structure ("ForgeMegakernel", §4.1: per-SM instruction streams,
+// dependency counters instead of grid-wide barriers; the AutoMegaKernel summary:
+// a static validator proves the schedule deadlock-free and race-free before it
+// runs; "Inside the megakernel serving engine": idle SMs take ready work instead
+// of waiting on a wave) is realised here as plain host code:
+//  * every phase (embed, per layer qkv / attn / oproj / gateup / down, lm head)
+//    is cut into fixed work units; each SM gets a contiguous range of units, and
+//    the SMs that carry the extra unit of a phase are the ones with the least
+//    cumulative weight bytes so far, so that bytes stay balanced over the step;
+//  * each task waits on exactly one counter (all tasks of the phase it reads)
+//    and adds one to its own phase's counter.
+#include "mk_plan.h"
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <numeric>
+
+namespace mk {
+
+Geometry geometry(const mk_model_cfg& c) {
+  Geometry G;
+  G.L = c.n_layers;
+  G.d = c.hidden;
+  G.nq = c.n_heads;
+  G.nkv = c.n_kv_heads;
+  G.hd = c.head_dim;
+  G.F = c.ffn;
+  G.V = c.vocab;
+  G.g = c.n_kv_heads > 0 ? c.n_heads / c.n_kv_heads : 0;
+  G.qdim = c.n_heads * c.head_dim;
+  G.kvdim = c.n_kv_heads * c.head_dim;
+  return G;
+}
+
+int gemv_K(const Geometry& G, int op) {
+  switch (op) {
+    case OP_QKV: case OP_GATEUP: case OP_LMHEAD: return G.d;
+    case OP_OPROJ: return G.qdim;
+    case OP_DOWN: return G.F;
+    default: return 0;
+  }
+}
+
+int phase_units(const Geometry& G, int op) {
+  switch (op) {
+    case OP_EMBED: return G.d / 8;
+    case OP_QKV: return (G.nq + 2 * G.nkv) * (G.hd / 16);
+    case OP_OPROJ: case OP_DOWN: return G.d / 8;
+    case OP_GATEUP: return G.F / 8;
+    case OP_LMHEAD: return G.V / 8;
+    default: return 0;
+  }
+}
+
+long long unit_weight_bytes(const Geometry& G, int op) {
+  if (op == OP_EMBED || op == OP_ATTN) return 0;
+  return (long long)rows_per_unit(op) * gemv_K(G, op) * 2;
+}
+
+uint16_t choose_kc(int rows, int K) {
+  if ((long long)rows * stage_pitch(K) <= kSlotBytes) return (uint16_t)K;
+  int best = 0;
+  for (int kc = 256; kc < K; kc += 256)
+    if ((long long)rows * stage_pitch(kc) <= kSlotBytes) best = kc;
+  if (best == 0)
+    for (int kc = 32; kc < K; kc += 32)
+      if ((long long)rows * stage_pitch(kc) <= kSlotBytes) best = kc;
+  return (uint16_t)best;
+}
+
+static bool set_err(std::string* err, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+static bool set_err(std::string* err, const char* fmt, ...) {
+  if (err) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    *err = buf;
+  }
+  return false;
+}
+
+int check_cfg(const mk_model_cfg& c, std::string* err) {
+  if (c.n_layers < 1 || c.hidden < 8 || c.n_heads < 1 || c.n_kv_heads < 1 || c.ffn < 8 || c.vocab < 8 ||
+      c.max_batch < 1 || c.max_ctx < 1) {
+    set_err(err, "model cfg: sizes must be positive");
+    return MK_ERR_INVALID_ARG;
+  }
+  if (!(c.rms_eps > 0.f) || !(c.rope_theta > 1.f)) {
+    set_err(err, "model cfg: rms_eps must be > 0 and rope_theta > 1");
+    return MK_ERR_INVALID_ARG;
+  }
+  if (c.page_size != kPage) { set_err(err, "page_size must be %d", kPage); return MK_ERR_UNSUPPORTED_CFG; }
+  if (c.head_dim != 64 && c.head_dim != 128) { set_err(err, "head_dim must be 64 or 128"); return MK_ERR_UNSUPPORTED_CFG; }
+  if (c.n_heads % c.n_kv_heads) { set_err(err, "n_heads must be a multiple of n_kv_heads"); return MK_ERR_UNSUPPORTED_CFG; }
+  int g = c.n_heads / c.n_kv_heads;
+  if (g > 8 || (c.head_dim == 128 && g > 4)) {
+    set_err(err, "query heads per kv head: at most 8 (4 at head_dim 128)");
+    return MK_ERR_UNSUPPORTED_CFG;
+  }
+  if (c.hidden % 8 || c.ffn % 8 || c.vocab % 8) {
+    set_err(err, "hidden, ffn and vocab must be multiples of 8");
+    return MK_ERR_UNSUPPORTED_CFG;
+  }
+  if (c.max_batch > kMaxBatch) { set_err(err, "max_batch must be <= %d", kMaxBatch); return MK_ERR_UNSUPPORTED_CFG; }
+  if (c.max_ctx > 65536) { set_err(err, "max_ctx must be <= 65536"); return MK_ERR_UNSUPPORTED_CFG; }
+  if (c.hidden > 65535 * 8 || c.ffn > 65535 || c.hidden > 65535) {
+    set_err(err, "hidden and ffn must fit the descriptor's 16-bit stage width");
+    return MK_ERR_UNSUPPORTED_CFG;
+  }
+  return MK_OK;
+}
+
+// Phase order of one step: embed, per layer qkv attn oproj gateup down, lm head.
+struct PhaseRef {
+  int op, layer;
+};
+
+static std::vector<PhaseRef> phase_order(int L) {
+  std::vector<PhaseRef> v;
+  v.push_back({OP_EMBED, 0});
+  for (int l = 0; l < L; ++l)
+    for (int op : {OP_QKV, OP_ATTN, OP_OPROJ, OP_GATEUP, OP_DOWN}) v.push_back({op, l});
+  v.push_back({OP_LMHEAD, 0});
+  return v;
+}
+
+static int sig_counter(int op, int layer, int L) {
+  switch (op) {
+    case OP_EMBED: return ctr_embed();
+    case OP_QKV: return ctr_layer(layer, 0);
+    case OP_ATTN: return ctr_layer(layer, 1);
+    case OP_OPROJ: return ctr_layer(layer, 2);
+    case OP_GATEUP: return ctr_layer(layer, 3);
+    case OP_DOWN: return ctr_layer(layer, 4);
+    case OP_LMHEAD: return ctr_lm(L);
+  }
+  return -1;
+}
+
+// The counter a phase waits on: the phase whose output it reads first.
+static int wait_counter(int op, int layer, int L) {
+  switch (op) {
+    case OP_EMBED: return kNoCounter;
+    case OP_QKV: return layer == 0 ? ctr_embed() : ctr_layer(layer - 1, 4);
+    case OP_ATTN: return ctr_layer(layer, 0);
+    case OP_OPROJ: return ctr_layer(layer, 1);
+    case OP_GATEUP: return ctr_layer(layer, 2);
+    case OP_DOWN: return ctr_layer(layer, 3);
+    case OP_LMHEAD: return ctr_layer(L - 1, 4);
+  }
+  return kNoCounter;
+}
+
+int build_plan(const mk_model_cfg& c, const mk_plan_opts* opts, mk_plan_s* P, std::string* err) {
+  int rc = check_cfg(c, err);
+  if (rc) return rc;
+  const Geometry G = geometry(c);
+  P->cfg = c;
+  P->num_sms = (opts && opts->num_sms > 0) ? opts->num_sms : 148;
+  P->attn_slots_per_sm = (opts && opts->attn_slots_per_sm > 0) ? opts->attn_slots_per_sm : 4;
+  P->max_blocks = (opts && opts->max_blocks > 0) ? opts->max_blocks : kMaxBlocks;
+  if (P->num_sms > 4096 || P->attn_slots_per_sm > 64 || P->max_blocks > kMaxBlocks) {
+    set_err(err, "plan options out of range");
+    return MK_ERR_INVALID_ARG;
+  }
+  // every (sequence, kv head) needs at least one split-K slot
+  const int need = (c.max_batch * G.nkv + P->num_sms - 1) / P->num_sms;
+  if (P->attn_slots_per_sm < need) P->attn_slots_per_sm = need;
+  const int S = P->num_sms * P->attn_slots_per_sm;
+  if (S > 65535) { set_err(err, "too many attention slots"); return MK_ERR_INVALID_ARG; }
+  const int nsm = P->num_sms;
+  P->streams.assign(nsm, {});
+  P->signalers.assign(num_counters(G.L), 0);
+  P->max_phase_tasks = 0;
+  std::vector<long long> cum(nsm, 0);
+
+  std::vector<PhaseRef> order = phase_order(G.L);
+  std::vector<int> phase_tasks(order.size(), 0);
+  // First pass: place units; wait counts need the task count of the awaited phase,
+  // which always comes earlier in the order, so one pass suffices.
+  std::vector<int> tasks_of_counter(num_counters(G.L), 0);
+  for (size_t pi = 0; pi < order.size(); ++pi) {
+    const int op = order[pi].op, l = order[pi].layer;
+    const int sig = sig_counter(op, l, G.L);
+    const int wc = wait_counter(op, l, G.L);
+    const uint32_t wcount = wc == kNoCounter ? 0u : (uint32_t)tasks_of_counter[wc];
+    int tidx = 0;
+    if (op == OP_ATTN) {
+      for (int sm = 0; sm < nsm; ++sm)
+        for (int s = 0; s < P->attn_slots_per_sm; ++s) {
+          TaskDesc t{};
+          t.op = OP_ATTN;
+          t.nunits = 1;
+          t.layer = (uint16_t)l;
+          t.u0 = (uint32_t)(s * nsm + sm);
+          t.task_idx = (uint16_t)tidx++;
+          t.kc = 0;
+          t.wait_ctr = (uint16_t)wc;
+          t.wait_count = wcount;
+          t.sig_ctr = (uint16_t)sig;
+          P->streams[sm].push_back(t);
+        }
+    } else {
+      const int U = phase_units(G, op);
+      const long long ub = unit_weight_bytes(G, op);
+      const int rpu = op == OP_EMBED ? 8 : rows_per_unit(op);
+      const int max_units = op == OP_EMBED ? 255 : std::max(1, P->max_blocks * 8 / rpu);
+      // units per SM: base, and +1 for the 'extra' SMs with the least bytes so far
+      std::vector<int> cnt(nsm, U / nsm);
+      int extra = U % nsm;
+      if (extra) {
+        std::vector<int> idx(nsm);
+        std::iota(idx.begin(), idx.end(), 0);
+        std::stable_sort(idx.begin(), idx.end(), [&](int a, int b) { return cum[a] < cum[b]; });
+        for (int k = 0; k < extra; ++k) cnt[idx[k]]++;
+      }
+      int u = 0;
+      for (int sm = 0; sm < nsm; ++sm) {
+        int n = cnt[sm];
+        if (n == 0) continue;
+        int ntask = (n + max_units - 1) / max_units;
+        for (int k = 0; k < ntask; ++k) {
+          int nk = n / ntask + (k < n % ntask ? 1 : 0);
+          TaskDesc t{};
+          t.op = (uint8_t)op;
+          t.nunits = (uint8_t)nk;
+          t.layer = (uint16_t)l;
+          t.u0 = (uint32_t)u;
+          t.task_idx = (uint16_t)tidx++;
+          t.kc = op == OP_EMBED ? 0 : choose_kc(nk * rpu, gemv_K(G, op));
+          t.wait_ctr = (uint16_t)wc;
+          t.wait_count = wcount;
+          t.sig_ctr = (uint16_t)sig;
+          P->streams[sm].push_back(t);
+          u += nk;
+        }
+        cum[sm] += (long long)n * ub;
+      }
+    }
+    phase_tasks[pi] = tidx;
+    tasks_of_counter[sig] += tidx;
+    P->signalers[sig] += tidx;
+    if (op != OP_ATTN) P->max_phase_tasks = std::max(P->max_phase_tasks, tidx);
+    if (op == OP_LMHEAD) P->n_lm_tasks = tidx;
+  }
+  return MK_OK;
+}
+
+// ---------------------------------------------------------------------------------------
+// Validator
+
+namespace {
+
+enum Buf { B_X, B_Q, B_ATTN, B_H, B_PART, B_LOGITS, B_LMPART, B_KVNEW, B_SSQ };
+
+struct Access {
+  int buf, inst;   // inst: layer for KVNEW, ssq instance for SSQ, 0 otherwise
+  bool write;
+};
+
+std::vector<Access> accesses(int op, int l, int L) {
+  switch (op) {
+    case OP_EMBED: return {{B_X, 0, true}, {B_SSQ, ssq_inst_embed(), true}};
+    case OP_QKV:
+      return {{B_X, 0, false}, {B_SSQ, l == 0 ? ssq_inst_embed() : ssq_inst_down(l - 1), false},
+              {B_Q, 0, true}, {B_KVNEW, l, true}};
+    case OP_ATTN: return {{B_Q, 0, false}, {B_KVNEW, l, false}, {B_PART, 0, true}, {B_ATTN, 0, true}};
+    case OP_OPROJ: return {{B_ATTN, 0, false}, {B_X, 0, true}, {B_SSQ, ssq_inst_oproj(l), true}};
+    case OP_GATEUP: return {{B_X, 0, false}, {B_SSQ, ssq_inst_oproj(l), false}, {B_H, 0, true}};
+    case OP_DOWN: return {{B_H, 0, false}, {B_X, 0, true}, {B_SSQ, ssq_inst_down(l), true}};
+    case OP_LMHEAD:
+      return {{B_X, 0, false}, {B_SSQ, ssq_inst_down(L - 1), false}, {B_LOGITS, 0, true}, {B_LMPART, 0, true}};
+  }
+  return {};
+}
+
+}  // namespace
+
+int validate_plan(const mk_plan_s& p, std::string* err) {
+  std::string e;
+  if (check_cfg(p.cfg, &e) != MK_OK) { set_err(err, "%s", e.c_str()); return MK_ERR_SCHEDULE_INVALID; }
+  const Geometry G = geometry(p.cfg);
+  const int nsm = (int)p.streams.size();
+  const int nctr = num_counters(G.L);
+  const int S = p.num_sms * p.attn_slots_per_sm;
+  std::vector<PhaseRef> order = phase_order(G.L);
+  auto phase_index = [&](int op, int l) -> int {
+    if (op == OP_EMBED) return 0;
+    if (op == OP_LMHEAD) return (int)order.size() - 1;
+    int k = op == OP_QKV ? 0 : op == OP_ATTN ? 1 : op == OP_OPROJ ? 2 : op == OP_GATEUP ? 3 : 4;
+    return 1 + 5 * l + k;
+  };
+  const int NP = (int)order.size();
+
+  // 1. each task well formed; units covered exactly once; stages fit a slot
+  std::vector<std::vector<int>> cover(NP);
+  for (int pi = 0; pi < NP; ++pi) {
+    int op = order[pi].op;
+    cover[pi].assign(op == OP_ATTN ? S : phase_units(G, op), 0);
+  }
+  std::vector<int> n_sig(nctr, 0);
+  std::vector<int> phase_of_sig(nctr, -1);
+  for (int sm = 0; sm < nsm; ++sm)
+    for (size_t k = 0; k < p.streams[sm].size(); ++k) {
+      const TaskDesc& t = p.streams[sm][k];
+      if (t.op < OP_EMBED || t.op > OP_LMHEAD || t.layer >= G.L) {
+        set_err(err, "sm %d task %zu: bad op %d / layer %d", sm, k, t.op, t.layer);
+        return MK_ERR_SCHEDULE_INVALID;
+      }
+      int pi = phase_index(t.op, t.layer);
+      if (t.nunits < 1 || t.u0 + t.nunits > cover[pi].size()) {
+        set_err(err, "sm %d task %zu (op %d layer %d): units [%u, %u) outside [0, %zu)", sm, k, t.op,
+                t.layer, t.u0, t.u0 + t.nunits, cover[pi].size());
+        return MK_ERR_SCHEDULE_INVALID;
+      }
+      for (uint32_t u = t.u0; u < t.u0 + t.nunits; ++u) cover[pi][u]++;
+      if (t.op != OP_EMBED && t.op != OP_ATTN) {
+        int rows = t.nunits * rows_per_unit(t.op);
+        int K = gemv_K(G, t.op);
+        if (rows > kMaxBlocks * 8) {
+          set_err(err, "sm %d task %zu: %d rows exceed %d", sm, k, rows, kMaxBlocks * 8);
+          return MK_ERR_SCHEDULE_INVALID;
+        }
+        if (t.kc < 8 || t.kc % 8 || (t.kc < K && t.kc % 32) || t.kc > K ||
+            (long long)rows * stage_pitch(t.kc) > kSlotBytes) {
+          set_err(err, "sm %d task %zu: stage of %d rows x %d columns does not fit a %d-byte slot", sm, k,
+                  rows, t.kc, kSlotBytes);
+          return MK_ERR_SCHEDULE_INVALID;
+        }
+      }
+      if (t.sig_ctr >= nctr) { set_err(err, "sm %d task %zu: bad signal counter", sm, k); return MK_ERR_SCHEDULE_INVALID; }
+      if (phase_of_sig[t.sig_ctr] == -1) phase_of_sig[t.sig_ctr] = pi;
+      if (phase_of_sig[t.sig_ctr] != pi) {
+        set_err(err, "counter %d is signalled by two phases", t.sig_ctr);
+        return MK_ERR_SCHEDULE_INVALID;
+      }
+      n_sig[t.sig_ctr]++;
+    }
+  for (int pi = 0; pi < NP; ++pi)
+    for (size_t u = 0; u < cover[pi].size(); ++u)
+      if (cover[pi][u] != 1) {
+        set_err(err, "phase op %d layer %d: unit %zu covered %d times", order[pi].op, order[pi].layer, u,
+                cover[pi][u]);
+        return MK_ERR_SCHEDULE_INVALID;
+      }
+
+  // 2. every wait target is exactly the number of signals its counter gets
+  for (int sm = 0; sm < nsm; ++sm)
+    for (size_t k = 0; k < p.streams[sm].size(); ++k) {
+      const TaskDesc& t = p.streams[sm][k];
+      if (t.wait_ctr == kNoCounter) continue;
+      if (t.wait_ctr >= nctr || t.wait_count != (uint32_t)n_sig[t.wait_ctr] || t.wait_count == 0) {
+        set_err(err, "sm %d task %zu (op %d layer %d): waits for %u signals on counter %d, which gets %d", sm,
+                k, t.op, t.layer, t.wait_count, (int)t.wait_ctr, t.wait_ctr < nctr ? n_sig[t.wait_ctr] : -1);
+        return MK_ERR_SCHEDULE_INVALID;
+      }
+    }
+
+  // 3. deadlock freedom: program order + counter edges must form a DAG (Kahn)
+  {
+    std::vector<int> first(nsm + 1, 0);
+    for (int sm = 0; sm < nsm; ++sm) first[sm + 1] = first[sm] + (int)p.streams[sm].size();
+    const int NT = first[nsm];
+    std::vector<int> indeg(NT + nctr, 0);
+    std::vector<std::vector<int>> waiters(nctr);
+    for (int sm = 0; sm < nsm; ++sm)
+      for (size_t k = 0; k < p.streams[sm].size(); ++k) {
+        int id = first[sm] + (int)k;
+        const TaskDesc& t = p.streams[sm][k];
+        if (k > 0) indeg[id]++;
+        if (t.wait_ctr != kNoCounter) {
+          indeg[id]++;
+          waiters[t.wait_ctr].push_back(id);
+        }
+        indeg[NT + t.sig_ctr]++;
+      }
+    std::vector<int> stack, sm_of(NT);
+    for (int sm = 0; sm < nsm; ++sm)
+      for (int id = first[sm]; id < first[sm + 1]; ++id) sm_of[id] = sm;
+    for (int v = 0; v < NT + nctr; ++v)
+      if (indeg[v] == 0) stack.push_back(v);
+    int done = 0;
+    while (!stack.empty()) {
+      int v = stack.back();
+      stack.pop_back();
+      ++done;
+      if (v < NT) {
+        int sm = sm_of[v];
+        const TaskDesc& t = p.streams[sm][v - first[sm]];
+        if (v + 1 < first[sm + 1] && --indeg[v + 1] == 0) stack.push_back(v + 1);
+        if (--indeg[NT + t.sig_ctr] == 0) stack.push_back(NT + t.sig_ctr);
+      } else {
+        for (int w : waiters[v - NT])
+          if (--indeg[w] == 0) stack.push_back(w);
+      }
+    }
+    if (done != NT + nctr) {
+      for (int sm = 0; sm < nsm; ++sm)
+        for (int id = first[sm]; id < first[sm + 1]; ++id)
+          if (indeg[id] > 0) {
+            const TaskDesc& t = p.streams[sm][id - first[sm]];
+            set_err(err, "deadlock: sm %d task %d (op %d layer %d) can never start", sm, id - first[sm], t.op,
+                    t.layer);
+            return MK_ERR_SCHEDULE_INVALID;
+          }
+      set_err(err, "deadlock: a counter can never reach its target");
+      return MK_ERR_SCHEDULE_INVALID;
+    }
+  }
+
+  // 4. race freedom at phase level.  Phase A happens before phase B when every task
+  // of B waits on the counter that exactly A's tasks signal; take the closure.
+  {
+    std::vector<int> wait_phase(NP, -2);  // -2 unset, -1 no wait, -3 mixed
+    for (int sm = 0; sm < nsm; ++sm)
+      for (const TaskDesc& t : p.streams[sm]) {
+        int pi = phase_index(t.op, t.layer);
+        int wp = t.wait_ctr == kNoCounter ? -1 : phase_of_sig[t.wait_ctr];
+        if (wait_phase[pi] == -2) wait_phase[pi] = wp;
+        else if (wait_phase[pi] != wp) wait_phase[pi] = -3;
+      }
+    std::vector<std::vector<char>> hb(NP, std::vector<char>(NP, 0));
+    for (int b = 0; b < NP; ++b)
+      if (wait_phase[b] >= 0) hb[wait_phase[b]][b] = 1;
+    for (int k = 0; k < NP; ++k)
+      for (int i = 0; i < NP; ++i)
+        if (hb[i][k])
+          for (int j = 0; j < NP; ++j)
+            if (hb[k][j]) hb[i][j] = 1;
+    for (int a = 0; a < NP; ++a)
+      for (int b = a + 1; b < NP; ++b) {
+        auto A = accesses(order[a].op, order[a].layer, G.L);
+        auto B = accesses(order[b].op, order[b].layer, G.L);
+        for (const Access& x : A)
+          for (const Access& y : B)
+            if (x.buf == y.buf && x.inst == y.inst && (x.write || y.write) && !hb[a][b]) {
+              set_err(err, "race: phase op %d layer %d %s buffer %d and phase op %d layer %d %s it without a "
+                      "counter ordering them", order[a].op, order[a].layer, x.write ? "writes" : "reads", x.buf,
+                      order[b].op, order[b].layer, y.write ? "writes" : "reads");
+              return MK_ERR_SCHEDULE_INVALID;
+            }
+      }
+  }
+  return MK_OK;
+}
+
+}  // namespace mk
+
+// ---------------------------------------------------------------------------------------
+// C ABI of the plan
+
+extern "C" {
+
+static thread_local std::string g_plan_err;
+const char* mk_internal_plan_error() { return g_plan_err.c_str(); }
+
+MK_API int mk_plan_create(const mk_model_cfg* cfg, const mk_plan_opts* opts, mk_plan_t* out) {
+  if (!cfg || !out) { g_plan_err = "null argument"; return MK_ERR_INVALID_ARG; }
+  mk_plan_s* p = new mk_plan_s();
+  int rc = mk::build_plan(*cfg, opts, p, &g_plan_err);
+  if (rc) { delete p; return rc; }
+  *out = p;
+  return MK_OK;
+}
+
+MK_API int mk_plan_validate(mk_plan_t plan, char* msg, size_t msg_len) {
+  if (!plan) return MK_ERR_INVALID_ARG;
+  std::string e;
+  int rc = mk::validate_plan(*plan, &e);
+  if (msg && msg_len) {
+    std::snprintf(msg, msg_len, "%s", rc ? e.c_str() : "ok");
+  }
+  return rc;
+}
+
+MK_API int mk_plan_stats(mk_plan_t plan, mk_plan_info* o) {
+  if (!plan || !o) return MK_ERR_INVALID_ARG;
+  std::memset(o, 0, sizeof(*o));
+  const mk::Geometry G = mk::geometry(plan->cfg);
+  o->weight_bytes_min_sm = -1;
+  for (const auto& s : plan->streams) {
+    o->n_tasks += (int64_t)s.size();
+    o->max_tasks_per_sm = std::max<int64_t>(o->max_tasks_per_sm, (int64_t)s.size());
+    int64_t bytes = 0;
+    for (const auto& t : s) {
+      if (t.op == mk::OP_EMBED || t.op == mk::OP_ATTN) continue;
+      int K = mk::gemv_K(G, t.op);
+      o->n_stages += (K + t.kc - 1) / t.kc;
+      bytes += (int64_t)t.nunits * mk::unit_weight_bytes(G, t.op);
+    }
+    o->weight_bytes_max_sm = std::max(o->weight_bytes_max_sm, bytes);
+    if (o->weight_bytes_min_sm < 0 || bytes < o->weight_bytes_min_sm) o->weight_bytes_min_sm = bytes;
+  }
+  o->attn_slots = (int64_t)plan->num_sms * plan->attn_slots_per_sm;
+  o->n_counters = mk::num_counters(G.L);
+  return MK_OK;
+}
+
+MK_API int mk_plan_inject_fault(mk_plan_t plan, int32_t kind, int32_t arg) {
+  if (!plan) return MK_ERR_INVALID_ARG;
+  const int L = plan->cfg.n_layers;
+  int layer = arg < 0 ? 0 : (arg >= L ? L - 1 : arg);
+  switch (kind) {
+    case MK_FAULT_DROP_WAIT: {
+      for (auto& s : plan->streams)
+        for (auto& t : s)
+          if (t.op == mk::OP_DOWN && t.layer == layer) { t.wait_ctr = mk::kNoCounter; t.wait_count = 0; }
+      return MK_OK;
+    }
+    case MK_FAULT_RAISE_TARGET: {
+      for (auto& s : plan->streams)
+        for (auto& t : s)
+          if (t.op == mk::OP_LMHEAD) t.wait_count += 1;
+      return MK_OK;
+    }
+    case MK_FAULT_REORDER: {
+      // move a down task of the layer in front of a gate/up task of the same layer
+      // (on the gate/up task's SM): it then waits on a task that can only run after it
+      int gs = -1, gi = -1, ds = -1, di = -1;
+      for (size_t s = 0; s < plan->streams.size(); ++s)
+        for (size_t k = 0; k < plan->streams[s].size(); ++k) {
+          const auto& t = plan->streams[s][k];
+          if (t.op == mk::OP_GATEUP && t.layer == layer && gs < 0) { gs = (int)s; gi = (int)k; }
+          if (t.op == mk::OP_DOWN && t.layer == layer && ds < 0) { ds = (int)s; di = (int)k; }
+        }
+      if (gs < 0 || ds < 0) return MK_ERR_INVALID_ARG;
+      mk::TaskDesc t = plan->streams[ds][di];
+      plan->streams[ds].erase(plan->streams[ds].begin() + di);
+      if (ds == gs && di < gi) --gi;
+      plan->streams[gs].insert(plan->streams[gs].begin() + gi, t);
+      return MK_OK;
+    }
+    case MK_FAULT_DUP_UNIT: {
+      for (auto& s : plan->streams)
+        for (auto& t : s)
+          if (t.op == mk::OP_OPROJ && t.layer == layer && t.nunits < 255) { t.nunits += 1; return MK_OK; }
+      return MK_ERR_INVALID_ARG;
+    }
+    case MK_FAULT_OVERSIZE_STAGE: {
+      for (auto& s : plan->streams)
+        for (auto& t : s)
+          if (t.op == mk::OP_LMHEAD) { t.kc = 0xFFE0; return MK_OK; }
+      return MK_ERR_INVALID_ARG;
+    }
+  }
+  return MK_ERR_INVALID_ARG;
+}
+
+MK_API void mk_plan_destroy(mk_plan_t plan) { delete plan; }
+
+}  // extern "C"

@@ -1,0 +1,394 @@
+"""Decode-step benchmark: tokens/s and model bandwidth utilisation on B200.
+
+One step = one call of mk_decode_step: the whole decode step (embedding gather,
+all layers, final norm, LM head, argmax) for one batch, as one kernel launch.
+The metric follows "ForgeMegakernel" §2.2: MBU = B(b, S) / (t_step * peak HBM),
+B counting every weight byte, the gathered embedding rows (not the table) and
+the prior KV entries; decode tokens/s = b / t_step.
+
+  python bench.py [--gpus N --steps K --warmup W --workload NAME --impl mk|reference]
+
+Under torchrun (N > 1) every rank runs an independent replica of the workload on
+its own GPU (the step has no data-parallel exchange); value = tokens of all
+ranks / the slowest rank's time.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "decode tokens/s"
+NOMINAL_HBM_GBS = 8000.0  # the pages' "~8 TB/s" B200 peak used for MBU
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="llama3-8b-b8", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="mk", choices=["mk", "reference"])
+    ap.add_argument("--no-secondary", action="store_true", help="skip the batch-1 line of the same model")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def workload_desc(w: synth.Workload, lens) -> dict:
+    m = w.model
+    return {
+        "workload": w.name,
+        "shape": (f"{m.n_layers}L d{m.hidden} {m.n_heads}/{m.n_kv_heads} heads hd{m.head_dim} "
+                  f"F{m.ffn} V{m.vocab} {'tied' if m.tied else 'untied'}"),
+        "batch": w.batch,
+        "context": w.ctx[1] if w.ctx[0] == "fixed" else f"U[{w.ctx[1]},{w.ctx[2]}] seeded: {lens}",
+        "kv": "paged bf16, 16-token pages, shuffled page table",
+    }
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 7:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for n, v in zip(names, r[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": float(rows[0][1]),
+                "power_w_max": max(float(r[2]) for r in rows), "samples": len(rows), "reasons": sorted(reasons)}
+
+
+def setup_dist(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(world, v: float) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def traffic_from_profile(workload: str):
+    """Per-launch DRAM bytes recorded by the committed ncu summary, if it covers this
+    workload and the kernel sources it was taken on are unchanged."""
+    import hashlib
+
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None
+    src = b""
+    for f in ("mk_kernel.cu", "mk_common.h", "mk_kernel.h"):
+        with open(os.path.join(ROOT, "bandwidth_bound_b200", "csrc", f), "rb") as fh:
+            src += fh.read()
+    h = hashlib.sha256(src).hexdigest()[:16]
+    with open(p) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 3 and parts[0] == workload and parts[1] == h:
+                return float(parts[2])
+    return None
+
+
+def cpu_baseline(w: synth.Workload, wts, kv, toks, lens, budget_s: float = 12.0) -> dict:
+    """The float64 oracle on the host cores, on a bounded sample of the same step:
+    whole layers (repeated until ~budget_s of CPU time) and a slice of the LM head,
+    scaled to one full step."""
+    import oracle
+
+    m = w.model
+    cores = torch.get_num_threads()
+    pt = kv.page_table.cpu()
+    kp = kv.k_pool[:1].cpu()
+    vp = kv.v_pool[:1].cpu()
+    one = {"embed": wts["embed"], "final_norm": wts["final_norm"], "lm_head": wts["lm_head"],
+           "layers": [{k: v.cpu() for k, v in wts["layers"][0].items()}]}
+    cfg1 = synth.scaled_model(m, n_layers=1)
+    t_layers = []
+    t0 = time.perf_counter()
+    while True:
+        a = time.perf_counter()
+        oracle.decode_step(cfg1, one, kp, vp, pt, toks, lens, want_logits=False)
+        t_layers.append(time.perf_counter() - a)
+        if time.perf_counter() - t0 > budget_s * 0.8:
+            break
+    rows = min(m.vocab, 16384)
+    head = wts["lm_head"][:rows].cpu()
+    x = torch.randn(len(toks), m.hidden, dtype=torch.float64)
+    a = time.perf_counter()
+    _ = x @ head.to(torch.float64).T
+    t_head = (time.perf_counter() - a) * m.vocab / rows
+    t_step = statistics.median(t_layers) * m.n_layers + t_head
+    return {"value": len(toks) / t_step, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": (f"{len(t_layers)} runs of layer 0 (embedding gather + 1 layer, float64) x {m.n_layers} "
+                       f"layers + {rows} of {m.vocab} LM-head rows scaled; same seeded inputs"),
+            "seconds_per_step": t_step}
+
+
+def run_reference(args, world, rank):
+    """The oracle itself, timed as the reference arm."""
+    if rank != 0:
+        return
+    w = synth.WORKLOADS[args.workload]
+    lens = w.context_lengths()
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    m = w.model
+    wts = synth.make_weights(m, device=dev, layers=[0])
+    kv = synth.make_kv_cache(m, lens, device=dev)
+    toks = synth.token_ids(m, w.batch, tag=w.name)
+    per = []
+    for k in range(args.warmup + args.steps):
+        cb = cpu_baseline(w, wts, kv, toks, lens, budget_s=0.5)
+        if k >= args.warmup:
+            per.append(cb["seconds_per_step"])
+    t = statistics.median(per)
+    value = w.batch / t
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_desc(w, lens),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cb["cores"], "kind": "oracle",
+                             "sample": cb["sample"]},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def time_steps(fn, steps, stream, flush=None):
+    """CUDA-event time of `steps` calls of fn on `stream` (ms total, per-step list)."""
+    per = []
+    if flush is None:
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+        e0.record(stream)
+        ev[0].record(stream)
+        for k in range(steps):
+            fn()
+            ev[k + 1].record(stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        per = [ev[k].elapsed_time(ev[k + 1]) for k in range(steps)]
+        return e0.elapsed_time(e1), per
+    total = 0.0
+    for _ in range(steps):
+        flush()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        per.append(a.elapsed_time(b))
+        total += per[-1]
+    return total, per
+
+
+def run_mk(args, world, rank, local):
+    import bandwidth_bound_b200 as mk
+    import oracle
+
+    w = synth.WORKLOADS[args.workload]
+    m = w.model
+    lens = w.context_lengths()
+    b = w.batch
+    max_ctx = max(lens) + 2
+    wts = synth.make_weights(m, device="cuda")
+    kv = synth.make_kv_cache(m, lens, device="cuda", max_ctx=max_ctx, batch_cap=max(b, 8))
+    toks = synth.token_ids(m, b, tag=w.name)
+    h = mk.Megakernel(m, wts, max(b, 8), max_ctx)
+    stream = torch.cuda.current_stream()
+    tok_d = torch.tensor(toks, dtype=torch.int32, device="cuda")
+    pos_d = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    len_d = pos_d + 1
+    logits = torch.empty((b, m.vocab), dtype=torch.float32, device="cuda")
+    am = torch.empty((b,), dtype=torch.int32, device="cuda")
+    B = oracle.model_bytes(m, lens)
+    l2 = torch.cuda.get_device_properties(local).L2_cache_size
+    flush = None
+    l2_note = f"inputs larger than L2 ({B / 1e9:.2f} GB read per step vs {l2 / 1e6:.0f} MB L2)"
+    if B < 4 * l2:
+        scrub = torch.empty(2 * l2 // 4, dtype=torch.float32, device="cuda")
+        flush = lambda: scrub.zero_()  # noqa: E731
+        l2_note = "L2 flushed between steps (2x L2 buffer written, untimed)"
+
+    def step():
+        h.step(tok_d, pos_d, len_d, kv, logits, am, stream=stream, check=False)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert h.status() == mk.MK_OK, f"device status {h.status()}"
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    total_ms, per = time_steps(step, args.steps, stream, flush)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    assert h.status() == mk.MK_OK, f"device status {h.status()}"
+    ms = max_over_ranks(world, total_ms) / args.steps
+    value = world * b / (ms / 1e3)
+    peaks = measured_peaks()
+    achieved = B / (ms / 1e3) / 1e9
+    traffic = traffic_from_profile(w.name)
+
+    # end to end through the host-buffer entry point (pinned host memory)
+    tok_h = torch.tensor(toks, dtype=torch.int32).pin_memory()
+    pos_h = torch.tensor(lens, dtype=torch.int32).pin_memory()
+    len_h = (pos_h + 1).pin_memory()
+    logits_h = torch.empty((b, m.vocab), dtype=torch.float32).pin_memory()
+    am_h = torch.empty((b,), dtype=torch.int32).pin_memory()
+
+    def step_host():
+        h.step_host(tok_h, pos_h, len_h, kv, logits_h, am_h, stream=stream, check=False)
+
+    for _ in range(3):
+        step_host()
+    barrier(world)
+    e2e_total, _ = time_steps(step_host, min(args.steps, 100), stream, flush)
+    e2e_ms = max_over_ranks(world, e2e_total) / min(args.steps, 100)
+    h2d = 3 * 4 * b
+    d2h = b * m.vocab * 4 + b * 4
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(workload_desc(w, lens), l2=l2_note, parallelism=f"replicas x{world}"),
+        "mbu": B / (ms / 1e3) / (NOMINAL_HBM_GBS * 1e9),
+        "mbu_vs_measured_copy": achieved / peaks["hbm_gbs"],
+        "bytes_per_step": B,
+        "step_ms": {"median": statistics.median(per), "p10": sorted(per)[len(per) // 10],
+                    "p90": sorted(per)[(9 * len(per)) // 10]},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                     "peak_source": peaks["source"], "kernel": "mk_decode_kernel (the whole step)"},
+        "clocks": clk,
+        "e2e": {"value": world * b / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": args.steps * h.launches_per_step(),
+    }
+    if not args.no_secondary and b > 1:
+        # batch 1 of the same model and context on the same handle (first sequence)
+        b1 = lambda: h.step(tok_d[:1], pos_d[:1], len_d[:1], kv, logits[:1], am[:1], stream=stream,  # noqa: E731
+                            check=False)
+        for _ in range(args.warmup):
+            b1()
+        barrier(world)
+        t1, _ = time_steps(b1, min(args.steps, 200), stream, flush)
+        ms1 = max_over_ranks(world, t1) / min(args.steps, 200)
+        B1 = oracle.model_bytes(m, lens[:1])
+        line["secondary"] = {"workload": f"{m.name}-b1 (same handle, context {lens[0]})", "ms_per_step": ms1,
+                             "tokens_per_s": world / (ms1 / 1e3), "mbu": B1 / (ms1 / 1e3) / (NOMINAL_HBM_GBS * 1e9),
+                             "achieved_gbs": B1 / (ms1 / 1e3) / 1e9}
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = {k: v for k, v in cpu_baseline(w, wts, kv, toks, lens).items()
+                                if k != "seconds_per_step"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    h.close()
+
+
+def main():
+    args = parse()
+    world, rank, local = setup_dist(args) if args.impl == "mk" else (
+        int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_mk(args, world, rank, local)
+    finally:
+        if world > 1 and args.impl == "mk":
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

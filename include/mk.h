@@ -1,0 +1,217 @@
+/*
+ * mk.h - C ABI of the B200 (sm_100a) decode-step megakernel.
+ *
+ * One call of mk_decode_step runs one auto-regressive decode step of a
+ * Llama-style transformer for a ragged batch as ONE persistent kernel launch:
+ * embedding-row gather, per layer RMSNorm -> QKV projection -> RoPE -> paged KV
+ * append -> GQA attention over each sequence's prior positions -> O projection
+ * -> RMSNorm -> SwiGLU MLP, then the final RMSNorm and the LM head.
+ *
+ * What is computed: "ForgeMegakernel: A General Framework for Efficient
+ * Auto-Regressive Model Decode Megakernels" (paperlayer.ai digest of arXiv
+ * 2609.12379v1), §2.1 "The decode step" and §2.3 "Megakernels" (the whole step
+ * inside one host launch).  How it is organised: the same page's §4.1 (per-SM
+ * instruction streams, dependency counters instead of grid-wide barriers, a
+ * shared-memory buffer pool), and "Inside the megakernel serving engine for
+ * North Mini Code" (one thread block per SM, task descriptors, counters in
+ * global memory, weights streamed into shared memory before their activation
+ * dependencies are met, paged attention).
+ *
+ * Conventions for every entry point:
+ *   - Return value: MK_OK (0) or a negative mk_status code.  No exceptions cross
+ *     the ABI.  mk_last_error() gives a one-line message for the last failure
+ *     of a handle (or of the library when there is no handle).
+ *   - "device" pointers are CUDA global-memory addresses on the handle's device;
+ *     "host" pointers are ordinary CPU memory.  The caller owns every buffer it
+ *     passes; it must stay valid until the call's stream work has finished.
+ *   - All tensors are dense and row-major.  Weights are bf16 [out][in], the
+ *     layout of a Hugging Face nn.Linear.
+ */
+#ifndef MK_H_
+#define MK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MK_API __attribute__((visibility("default")))
+
+/* A CUDA stream (cudaStream_t / CUstream); NULL is the legacy default stream. */
+typedef struct CUstream_st *mk_stream_t;
+
+typedef enum mk_status {
+  MK_OK = 0,
+  MK_ERR_INVALID_ARG = -1,     /* a null/misaligned pointer, size out of range, bad value */
+  MK_ERR_UNSUPPORTED_CFG = -2, /* model shape outside what the kernel implements */
+  MK_ERR_SCHEDULE_INVALID = -3,/* the static validator rejected the task schedule */
+  MK_ERR_CUDA = -4,            /* a CUDA runtime call failed (message has the CUDA error) */
+  MK_ERR_DEVICE_TIMEOUT = -5,  /* a device-side wait ran past the handle's time limit */
+  MK_ERR_BOUNDS = -6,          /* the device found a token id, position, length or page id out of range */
+  MK_ERR_NO_DEVICE = -7        /* no usable sm_100 device */
+} mk_status;
+
+/* Model shape.  Supported: head_dim 64 or 128; n_heads % n_kv_heads == 0 with
+ * 1 <= n_heads/n_kv_heads <= 8 (<= 4 at head_dim 128); hidden, ffn, vocab and
+ * n_heads*head_dim multiples of 8; page_size 16; 1 <= max_batch <= 16. */
+typedef struct mk_model_cfg {
+  int32_t n_layers, hidden, n_heads, n_kv_heads, head_dim, ffn, vocab;
+  int32_t tied;        /* 1: the LM head is the embedding table (lm_head may equal embed) */
+  float rope_theta;    /* RoPE base: inv_freq_j = theta^(-2j/head_dim), rotate-half pairing */
+  float rms_eps;       /* RMSNorm epsilon, inside the square root */
+  int32_t max_batch;   /* largest batch a step may use */
+  int32_t max_ctx;     /* largest position + 1 a sequence may reach */
+  int32_t page_size;   /* KV tokens per page; must be 16 */
+} mk_model_cfg;
+
+/* Device pointers to bf16 weights.  The per-layer members are HOST arrays of
+ * n_layers device pointers each.  Shapes ([out][in]): embed, lm_head [vocab][hidden];
+ * final_norm, attn_norm[l], mlp_norm[l] [hidden]; wq [n_heads*head_dim][hidden];
+ * wk, wv [n_kv_heads*head_dim][hidden]; wo [hidden][n_heads*head_dim];
+ * w_gate, w_up [ffn][hidden]; w_down [hidden][ffn].  Every pointer 16-byte aligned.
+ * The handle keeps the device pointers (not the host arrays); the weights must
+ * outlive the handle. */
+typedef struct mk_weight_ptrs {
+  const void *embed, *final_norm, *lm_head;
+  const void *const *attn_norm, *const *wq, *const *wk, *const *wv, *const *wo;
+  const void *const *mlp_norm, *const *w_gate, *const *w_up, *const *w_down;
+} mk_weight_ptrs;
+
+/* Paged KV cache (device, caller-owned).  k_pool and v_pool are bf16
+ * [n_layers][num_pages][n_kv_heads][page_size][head_dim]; entry t of sequence i
+ * lives in physical page page_table[i*max_pages_per_seq + t/page_size], slot
+ * t % page_size.  Keys are stored after RoPE.  page_table is device int32
+ * [>= batch][max_pages_per_seq]. */
+typedef struct mk_kv_cache {
+  void *k_pool, *v_pool;
+  const int32_t *page_table;
+  int32_t num_pages, max_pages_per_seq;
+} mk_kv_cache;
+
+typedef struct mk_handle_s *mk_handle_t;
+typedef struct mk_plan_s *mk_plan_t;
+
+/* Options of the per-SM task schedule (zero fields take the defaults). */
+typedef struct mk_plan_opts {
+  int32_t num_sms;           /* CTAs = SMs of the device (default: queried; host-only plans: 148) */
+  int32_t attn_slots_per_sm; /* split-K attention slots per SM and layer (default 4) */
+  int32_t max_blocks;        /* 8-row blocks per GEMV task, 1..8 (default 8) */
+} mk_plan_opts;
+
+typedef struct mk_plan_info {
+  int64_t n_tasks, n_stages;          /* over all SMs */
+  int64_t max_tasks_per_sm;
+  int64_t weight_bytes_min_sm, weight_bytes_max_sm; /* bulk-copied weight bytes per SM */
+  int64_t attn_slots;                 /* split-K attention slots per layer */
+  int64_t n_counters;
+} mk_plan_info;
+
+/* ---- the decode step --------------------------------------------------------------- */
+
+/* Build a handle: derive the per-SM task streams for cfg (mk_plan_create with
+ * default options), run the static validator, allocate the handle's device state
+ * (dependency counters, activation scratch, RoPE table) on the current device and
+ * upload the streams.  Host-synchronous.  Errors: INVALID_ARG, UNSUPPORTED_CFG,
+ * SCHEDULE_INVALID, CUDA, NO_DEVICE.  *out is set only on success. */
+MK_API int mk_create(const mk_model_cfg *cfg, const mk_weight_ptrs *weights, mk_handle_t *out);
+
+/* As mk_create, from a plan built (and possibly altered) by the caller.  flags:
+ * MK_CREATE_SKIP_VALIDATE runs the plan without the static validator (test use:
+ * a plan with an unreachable wait must then come back as MK_ERR_DEVICE_TIMEOUT).
+ * The plan is copied; the caller still destroys it. */
+#define MK_CREATE_SKIP_VALIDATE 1
+MK_API int mk_create_from_plan(mk_plan_t plan, const mk_weight_ptrs *weights, int32_t flags,
+                               mk_handle_t *out);
+
+/* One decode step, stream-ordered and asynchronous (one kernel launch).
+ *   token_ids  device int32 [batch]: the new token of each sequence
+ *   positions  device int32 [batch]: p_i = prior entries of sequence i = the new
+ *              token's position; sequences may all differ (ragged batch)
+ *   seq_lens   device int32 [batch]: keys attended, must equal positions + 1
+ *   batch      1 .. cfg.max_batch
+ *   kv         the cache; the step writes exactly one K and one V entry per
+ *              (layer, sequence, kv head) at position p_i and nothing else
+ *   logits_out device fp32 [batch][vocab]
+ *   argmax_out device int32 [batch] or NULL: greedy next token (lowest index of the max)
+ * Host-side argument errors return before anything is launched.  Device-side
+ * errors (bounds, timeout) are sticky: they are read with mk_get_status after the
+ * stream has been synchronised, and every later step returns that error until
+ * mk_reset.  One handle runs one step at a time: steps on one handle must be
+ * ordered on the GPU (same stream, or synchronised). */
+MK_API int mk_decode_step(mk_handle_t h, const int32_t *token_ids, const int32_t *positions,
+                          const int32_t *seq_lens, int32_t batch, const mk_kv_cache *kv,
+                          float *logits_out, int32_t *argmax_out, mk_stream_t stream);
+
+/* The same step from HOST buffers: copies token_ids/positions/seq_lens (host
+ * int32 [batch]) to the handle's device staging area, runs the step, copies the
+ * logits (host fp32 [batch][vocab], may be NULL) and argmax (host int32 [batch],
+ * may be NULL) back, and synchronises the stream before returning.  Pinned host
+ * memory makes the copies asynchronous DMA.  The KV cache stays on the device. */
+MK_API int mk_decode_step_host(mk_handle_t h, const int32_t *token_ids, const int32_t *positions,
+                               const int32_t *seq_lens, int32_t batch, const mk_kv_cache *kv,
+                               float *logits_host, int32_t *argmax_host, mk_stream_t stream);
+
+/* Sticky device status of the handle's last steps: MK_OK, MK_ERR_DEVICE_TIMEOUT
+ * or MK_ERR_BOUNDS.  Read it after synchronising the stream of the step. */
+MK_API int mk_get_status(mk_handle_t h);
+
+/* Clear the sticky device status and the dependency counters (the step after a
+ * device error starts from a clean state).  Host-synchronous. */
+MK_API int mk_reset(mk_handle_t h);
+
+/* Mid-state capture for checking: when layer_hidden is a device fp32 buffer of
+ * [n_layers+1][max_batch][hidden], each later step writes the residual stream
+ * after the embedding gather (index 0) and after each layer (index l+1) for its
+ * batch rows.  NULL turns capture off. */
+MK_API int mk_set_debug(mk_handle_t h, float *layer_hidden);
+
+/* Device-side wait limit in nanoseconds (default 1e9).  A wait that runs out
+ * sets MK_ERR_DEVICE_TIMEOUT, every CTA leaves after its copies in flight have
+ * landed, and the launch completes. */
+MK_API int mk_set_timeout_ns(mk_handle_t h, uint64_t ns);
+
+/* Number of kernel launches each mk_decode_step makes (1). */
+MK_API int mk_launches_per_step(mk_handle_t h);
+
+MK_API int mk_destroy(mk_handle_t h);
+
+/* Message of the last failure on h (NULL: of the last handle-less call). */
+MK_API const char *mk_last_error(mk_handle_t h);
+
+/* ---- the task schedule (host only; no GPU needed) ----------------------------------- */
+
+/* Derive the per-SM instruction streams for cfg.  Units of work per phase are
+ * spread so that every SM's cumulative weight bytes stay within one unit of the
+ * others; tasks wait only on dependency counters of earlier phases. */
+MK_API int mk_plan_create(const mk_model_cfg *cfg, const mk_plan_opts *opts, mk_plan_t *out);
+
+/* Static validator (runs inside mk_create): every wait target is exactly the
+ * number of signals its counter receives; the graph of per-SM program order plus
+ * counter edges is acyclic (no deadlock with all CTAs co-resident); every work
+ * unit of every phase is covered exactly once; every stage fits a pool slot; and
+ * every pair of phases that touch the same scratch buffer, one of them writing,
+ * is ordered by counters (no race).  Returns MK_OK or MK_ERR_SCHEDULE_INVALID
+ * with the first violation written to msg (msg_len bytes, may be 0). */
+MK_API int mk_plan_validate(mk_plan_t plan, char *msg, size_t msg_len);
+
+MK_API int mk_plan_stats(mk_plan_t plan, mk_plan_info *out);
+
+/* Host-side fault injection for tests of the validator and of device timeouts.
+ * arg selects the layer (or the task for MK_FAULT_DUP_UNIT). */
+typedef enum mk_fault {
+  MK_FAULT_DROP_WAIT = 1,      /* the down projection of layer arg stops waiting for gate/up */
+  MK_FAULT_RAISE_TARGET = 2,   /* the LM head waits for one signal more than it can receive */
+  MK_FAULT_REORDER = 3,        /* on one SM, a down task of layer arg moves before its gate/up task */
+  MK_FAULT_DUP_UNIT = 4,       /* a task of layer arg's O projection also covers its neighbour's unit */
+  MK_FAULT_OVERSIZE_STAGE = 5  /* a task's stage no longer fits a pool slot */
+} mk_fault;
+MK_API int mk_plan_inject_fault(mk_plan_t plan, int32_t kind, int32_t arg);
+
+MK_API void mk_plan_destroy(mk_plan_t plan);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MK_H_ */

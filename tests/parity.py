@@ -1,0 +1,186 @@
+"""Helpers shared by the GPU parity tests: run one step on the device through the
+C ABI, run the float64 oracle on the same inputs, compare mid-states."""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import torch
+
+import bandwidth_bound_b200 as mk
+import oracle
+import synth
+
+# Tolerances (stated on the decode path: hidden-state relative L2 per layer, max |dlogit|,
+# 1 bf16 ulp on stored KV entries; integer state bit-exact).
+HIDDEN_REL_L2 = 1e-2
+LOGIT_ABS = 5e-2
+KV_ULP = 1.0
+
+
+@dataclass
+class Case:
+    m: synth.ModelConfig
+    lens: list            # prior entries S_i per sequence (= positions)
+    tokens: list
+    gain_std: float = 0.0
+    max_batch: int = 0
+    max_ctx: int = 0
+    weights: dict = None
+    kv: synth.KVCache = None
+    extra: dict = field(default_factory=dict)
+
+
+def make_case(m, lens, gain_std=0.0, max_batch=0, max_ctx=0, tag="", weights=None, kv_spare=3) -> Case:
+    b = len(lens)
+    max_batch = max_batch or b
+    max_ctx = max_ctx or (max(lens) + 1)
+    wts = weights if weights is not None else synth.make_weights(m, device="cuda", gain_std=gain_std)
+    kv = synth.make_kv_cache(m, list(lens), device="cuda", max_ctx=max_ctx, spare_pages=kv_spare,
+                             batch_cap=max_batch, tag=tag)
+    toks = synth.token_ids(m, b, tag=tag or m.name)
+    return Case(m, list(lens), toks, gain_std, max_batch, max_ctx, wts, kv)
+
+
+def gpu_step(c: Case, handle=None, batch=None, debug=True, argmax=True):
+    """Run one step; returns dict of device results (CPU copies) and the handle."""
+    b = len(c.lens) if batch is None else batch
+    if handle is None:
+        handle = mk.Megakernel(c.m, c.weights, c.max_batch, c.max_ctx)
+    dev = "cuda"
+    tok = torch.tensor(c.tokens[:b], dtype=torch.int32, device=dev)
+    pos = torch.tensor(c.lens[:b], dtype=torch.int32, device=dev)
+    lens = pos + 1
+    logits = torch.full((b, c.m.vocab), float("nan"), dtype=torch.float32, device=dev)
+    am = torch.full((b,), -1, dtype=torch.int32, device=dev) if argmax else None
+    dbg = None
+    if debug:
+        dbg = torch.full((c.m.n_layers + 1, c.max_batch, c.m.hidden), float("nan"), dtype=torch.float32,
+                         device=dev)
+        handle.set_debug(dbg)
+    handle.step(tok, pos, lens, c.kv, logits, am)
+    torch.cuda.synchronize()
+    st = handle.status()
+    out = {"status": st, "logits": logits.cpu(), "argmax": am.cpu() if am is not None else None,
+           "hidden": dbg[:, :b].cpu() if dbg is not None else None}
+    return out, handle
+
+
+def run_oracle(c: Case, k_before, v_before, batch=None, layers=None):
+    b = len(c.lens) if batch is None else batch
+    return oracle.decode_step(c.m, c.weights, k_before, v_before, c.kv.page_table[:b].cpu(), c.tokens[:b],
+                              c.lens[:b], layers=layers)
+
+
+def rel_l2(a: torch.Tensor, b: torch.Tensor) -> float:
+    a = a.to(torch.float64)
+    b = b.to(torch.float64)
+    return float((a - b).norm() / b.norm().clamp_min(1e-300))
+
+
+def bf16_ulp_error(gpu: torch.Tensor, ref: torch.Tensor) -> torch.Tensor:
+    """|gpu - ref| in units of the bf16 spacing at |ref|, per element.
+
+    ref: float64 values already rounded to bf16 (oracle), shape [..., hd].  The
+    magnitude is floored at 2^-8 times the RMS of its head vector, so that entries
+    near zero are not counted in ulps of a tiny number.
+    """
+    g = gpu.to(torch.float64)
+    r = ref.to(torch.float64)
+    rms = torch.sqrt((r * r).mean(-1, keepdim=True))
+    mag = torch.maximum(r.abs(), rms * 2.0 ** -8).clamp_min(1e-30)
+    ulp = torch.exp2(torch.floor(torch.log2(mag)) - 7)
+    return (g - r).abs() / ulp
+
+
+def check_step(c: Case, out: dict, ref: dict, k_before, v_before, batch=None, check_pool=True,
+               logit_tol=LOGIT_ABS) -> dict:
+    """Compare one GPU step with the oracle; returns the measured errors."""
+    b = len(c.lens) if batch is None else batch
+    m = c.m
+    P = m.page_size
+    errs = {}
+    assert out["status"] == mk.MK_OK, f"device status {out['status']}"
+    # per-layer hidden states, whole batch and per sequence
+    if out["hidden"] is not None:
+        worst = 0.0
+        hidden_fail = None
+        for li in range(m.n_layers + 1):
+            e = rel_l2(out["hidden"][li], ref["hidden"][li])
+            worst = max(worst, e)
+            for i in range(b):
+                ei = rel_l2(out["hidden"][li, i], ref["hidden"][li, i])
+                worst = max(worst, ei)
+                if ei > HIDDEN_REL_L2 and hidden_fail is None:
+                    hidden_fail = f"sequence {i} hidden after layer {li - 1}: rel L2 {ei}"
+        errs["hidden_rel_l2"] = worst
+        errs["hidden_rel_l2_per_layer"] = [round(rel_l2(out["hidden"][li], ref["hidden"][li]), 8)
+                                           for li in range(m.n_layers + 1)]
+    # KV: new entries within 1 ulp; everything else bit-identical (canaries included)
+    k_after = c.kv.k_pool
+    v_after = c.kv.v_pool
+    worst_ulp = 0.0
+    strict_fail = 0
+    for i in range(b):
+        page, slot = ref["slots"][i]
+        assert page == int(c.kv.page_table[i, c.lens[i] // P]) and slot == c.lens[i] % P
+        kg = k_after[:, page, :, slot, :].cpu()
+        vg = v_after[:, page, :, slot, :].cpu()
+        ek = bf16_ulp_error(kg, ref["k_new"][:, i])
+        ev = bf16_ulp_error(vg, ref["v_new"][:, i])
+        for name, e, gv, rv, ex in (("k", ek, kg, ref["k_new"][:, i], ref["k_new_exact"][:, i]),
+                                    ("v", ev, vg, ref["v_new"][:, i], ref["v_new_exact"][:, i])):
+            if float(e.max()) > worst_ulp:
+                worst_ulp = float(e.max())
+                at = [int(v) for v in torch.nonzero(e == e.max())[0]]
+                errs["kv_worst"] = {"which": name, "seq": i, "layer_head_dim": at,
+                                    "gpu": float(gv[tuple(at)]), "oracle_bf16": float(rv[tuple(at)]),
+                                    "oracle_exact": float(ex[tuple(at)]),
+                                    "head_rms": float(ex[at[0], at[1]].pow(2).mean().sqrt())}
+        strict_fail += int((kg.to(torch.float64) != ref["k_new"][:, i]).sum())
+    errs["kv_max_ulp"] = worst_ulp
+    errs["kv_entries_not_bit_equal"] = strict_fail
+    errs["kv_entries"] = 2 * b * ref["k_new"][:, 0].numel()
+    if "logits" in ref:
+        errs["logit_max_abs"] = (out["logits"].to(torch.float64) - ref["logits"]).abs().max().item()
+    print("parity:", errs)
+    if out["hidden"] is not None:
+        assert hidden_fail is None, hidden_fail
+    assert worst_ulp <= KV_ULP, f"new KV entry off by {worst_ulp} bf16 ulp"
+    if check_pool:
+        mask = torch.ones(k_after.shape[1:4], dtype=torch.bool)  # [P][nkv][page]
+        for i in range(b):
+            page, slot = ref["slots"][i]
+            mask[page, :, slot] = False
+        kb = k_before.view(torch.int16)
+        vb = v_before.view(torch.int16)
+        ka = k_after.cpu().view(torch.int16)
+        va = v_after.cpu().view(torch.int16)
+        mm = mask[None, :, :, :, None].expand_as(ka)
+        assert torch.equal(ka[mm], kb[mm]), "the step wrote KV outside the new slots"
+        assert torch.equal(va[mm], vb[mm]), "the step wrote KV outside the new slots"
+    # logits and argmax
+    if "logits" in ref:
+        dl = (out["logits"].to(torch.float64) - ref["logits"]).abs().max().item()
+        errs["logit_max_abs"] = dl
+        assert math.isfinite(dl) and dl <= logit_tol, f"max |dlogit| {dl}"
+        # mean log-prob error of the greedy token (reported, not gated)
+        lp_g = torch.log_softmax(out["logits"].to(torch.float64), -1)
+        lp_r = torch.log_softmax(ref["logits"], -1)
+        idx = torch.tensor(ref["argmax"])
+        errs["logprob_err"] = float((lp_g.gather(1, idx[:, None]) - lp_r.gather(1, idx[:, None])).abs().mean())
+        if out["argmax"] is not None:
+            for i in range(b):
+                got, want = int(out["argmax"][i]), ref["argmax"][i]
+                if got != want:
+                    # only a true numerical tie may differ: the oracle's top-2 gap below the error
+                    top = torch.topk(ref["logits"][i], 2).values
+                    gap = float(top[0] - top[1])
+                    assert gap < dl and abs(float(ref["logits"][i, got]) - float(top[0])) <= 2 * dl, \
+                        f"sequence {i}: argmax {got} != oracle {want} (gap {gap})"
+                    errs.setdefault("argmax_ties", 0)
+                    errs["argmax_ties"] += 1
+            # the device argmax is the argmax of the device logits
+            assert [int(v) for v in out["argmax"]] == [oracle.argmax_lowest(out["logits"][i].to(torch.float64))
+                                                       for i in range(b)]
+    return errs
