@@ -92,6 +92,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "mk_reset": (ctypes.c_int, [vp]),
         "mk_set_debug": (ctypes.c_int, [vp, vp]),
         "mk_set_timeout_ns": (ctypes.c_int, [vp, u64]),
+        "mk_set_trace": (ctypes.c_int, [vp, vp, ctypes.c_int64]),
+        "mk_num_tasks": (ctypes.c_int64, [vp]),
         "mk_launches_per_step": (ctypes.c_int, [vp]),
         "mk_destroy": (ctypes.c_int, [vp]),
         "mk_last_error": (ctypes.c_char_p, [vp]),
@@ -233,6 +235,14 @@ class Megakernel:
 
     def set_debug(self, layer_hidden):
         _check(self.lib.mk_set_debug(self.handle, _ptr(layer_hidden)), self.handle, "mk_set_debug")
+
+    def num_tasks(self) -> int:
+        return int(self.lib.mk_num_tasks(self.handle))
+
+    def set_trace(self, records):
+        """records: device uint64 tensor [>= num_tasks()][4], or None."""
+        n = 0 if records is None else records.shape[0]
+        _check(self.lib.mk_set_trace(self.handle, _ptr(records), n), self.handle, "mk_set_trace")
 
     def set_timeout_ns(self, ns: int):
         _check(self.lib.mk_set_timeout_ns(self.handle, int(ns)), self.handle, "mk_set_timeout_ns")

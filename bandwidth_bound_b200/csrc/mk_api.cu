@@ -1,4 +1,6 @@
 // C ABI of the decode megakernel: handle creation, the decode step, status.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <cstdio>
@@ -53,6 +55,62 @@ static void release(mk_handle_t h) {
   if (h->host_status) cudaFreeHost(h->host_status);
   if (h->h_stage) cudaFreeHost(h->h_stage);
   delete h;
+}
+
+// TMA descriptors of every weight matrix (bf16, 128-byte swizzle, boxes of 64 columns x
+// 8n rows for n = 1..8).  wq/wk/wv are viewed as [heads*2 halves][head_dim/2][hidden]
+// so that one box holds rows 8m..8m+8n-1 of both halves of a head (the RoPE pairs).
+static std::string build_tensor_maps(const mk_model_cfg& c, const mk_weight_ptrs* w, std::vector<CUtensorMap>& maps) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  if (!encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess || !fn)
+      return "cuTensorMapEncodeTiled is not available";
+    encode = (PFN_cuTensorMapEncodeTiled_v12000)fn;
+  }
+  const mk::Geometry G = mk::geometry(c);
+  maps.assign((size_t)(G.L + 1) * mk::kNumMats * mk::kMaxBlocks, CUtensorMap{});
+  auto enc2d = [&](CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {(cuuint32_t)mk::kBoxCols, box_rows};
+    cuuint32_t es[2] = {1, 1};
+    return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  };
+  auto enc3d = [&](CUtensorMap* m, const void* ptr, uint64_t heads, uint32_t box_rows) {
+    cuuint64_t dims[3] = {(cuuint64_t)G.d, (cuuint64_t)G.hd / 2, heads * 2};
+    cuuint64_t strides[2] = {(cuuint64_t)G.d * 2, (cuuint64_t)(G.hd / 2) * G.d * 2};
+    cuuint32_t box[3] = {(cuuint32_t)mk::kBoxCols, box_rows, 2};
+    cuuint32_t es[3] = {1, 1, 1};
+    return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  };
+  for (int l = 0; l < G.L; ++l) {
+    for (int n = 1; n <= mk::kMaxBlocks; ++n) {
+      const uint32_t br = 8u * n;
+      CUresult r = CUDA_SUCCESS;
+      if (n <= mk::max_units(mk::OP_QKV) && 8 * n <= G.hd / 2) {
+        r = enc3d(&maps[mk::tmap_index(l, 0, n)], w->wq[l], G.nq, br);
+        if (r == CUDA_SUCCESS) r = enc3d(&maps[mk::tmap_index(l, 1, n)], w->wk[l], G.nkv, br);
+        if (r == CUDA_SUCCESS) r = enc3d(&maps[mk::tmap_index(l, 2, n)], w->wv[l], G.nkv, br);
+      }
+      if (r == CUDA_SUCCESS && n <= mk::max_units(mk::OP_GATEUP)) {
+        r = enc2d(&maps[mk::tmap_index(l, 4, n)], w->w_gate[l], G.F, G.d, br);
+        if (r == CUDA_SUCCESS) r = enc2d(&maps[mk::tmap_index(l, 5, n)], w->w_up[l], G.F, G.d, br);
+      }
+      if (r == CUDA_SUCCESS) r = enc2d(&maps[mk::tmap_index(l, 3, n)], w->wo[l], G.d, G.qdim, br);
+      if (r == CUDA_SUCCESS) r = enc2d(&maps[mk::tmap_index(l, 6, n)], w->w_down[l], G.d, G.F, br);
+      if (r != CUDA_SUCCESS) return "cuTensorMapEncodeTiled failed for layer " + std::to_string(l);
+    }
+  }
+  for (int n = 1; n <= mk::kMaxBlocks; ++n)
+    if (enc2d(&maps[mk::tmap_index(G.L, 0, n)], w->lm_head, G.V, G.d, 8u * n) != CUDA_SUCCESS)
+      return "cuTensorMapEncodeTiled failed for the LM head";
+  return "";
 }
 
 extern "C" {
@@ -118,10 +176,19 @@ MK_API int mk_create_from_plan(mk_plan_t plan, const mk_weight_ptrs* w, int32_t 
   const size_t o_layers = take(sizeof(LayerW) * c.n_layers);
   const size_t o_tasks = take(sizeof(mk::TaskDesc) * flat.size());
   const size_t o_offs = take(sizeof(uint32_t) * offs.size());
+  std::vector<CUtensorMap> maps;
+  std::string merr = build_tensor_maps(c, w, maps);
+  if (!merr.empty()) { release(h); return fail(nullptr, MK_ERR_CUDA, merr); }
+  const size_t o_maps = take(sizeof(CUtensorMap) * maps.size());
   const size_t o_x = take(sizeof(float) * mb * G.d);
   const size_t o_q = take(sizeof(float) * mb * G.qdim);
-  const size_t o_attn = take(sizeof(float) * mb * G.qdim);
-  const size_t o_h = take(sizeof(float) * mb * G.F);
+  const int ld_x = mk::round_up(G.d, mk::kBoxCols), ld_a = mk::round_up(G.qdim, mk::kBoxCols),
+            ld_h = mk::round_up(G.F, mk::kBoxCols);
+  // operands: bf16 hi/lo tiles of 8 batch rows (operand_index layout) and the fp32 batch row 0,
+  // zero padded to whole 64-column boxes
+  const int ntiles = (mb + 7) / 8;
+  auto opbytes = [&](int ld) { return (size_t)ntiles * 2 * ld * 8 * 2 + (size_t)ld * 4; };
+  const size_t o_ax = take(opbytes(ld_x)), o_aa = take(opbytes(ld_a)), o_ah = take(opbytes(ld_h));
   const int ssq_stride = plan->max_phase_tasks * mb;
   const size_t o_ssq = take(sizeof(float) * mk::num_ssq_inst(G.L) * ssq_stride);
   const size_t o_part = take(sizeof(float) * (size_t)S * G.g * (G.hd + 2));
@@ -152,6 +219,8 @@ MK_API int mk_create_from_plan(mk_plan_t plan, const mk_weight_ptrs* w, int32_t 
     ce = cudaMemcpy(A + o_tasks, flat.data(), sizeof(mk::TaskDesc) * flat.size(), cudaMemcpyHostToDevice);
   if (ce == cudaSuccess)
     ce = cudaMemcpy(A + o_offs, offs.data(), sizeof(uint32_t) * offs.size(), cudaMemcpyHostToDevice);
+  if (ce == cudaSuccess)
+    ce = cudaMemcpy(A + o_maps, maps.data(), sizeof(CUtensorMap) * maps.size(), cudaMemcpyHostToDevice);
   if (ce == cudaSuccess) ce = mk::launch_rope_table((float2*)(A + o_rope), c.max_ctx, G.hd, c.rope_theta, 0);
   if (ce == cudaSuccess) ce = cudaDeviceSynchronize();
   if (ce != cudaSuccess) { release(h); return cuda_fail(nullptr, ce, "upload"); }
@@ -168,7 +237,16 @@ MK_API int mk_create_from_plan(mk_plan_t plan, const mk_weight_ptrs* w, int32_t 
   k.num_sms = plan->num_sms;
   k.n_slots = S;
   k.n_lm_tasks = plan->n_lm_tasks;
-  k.x = (float*)(A + o_x); k.q = (float*)(A + o_q); k.attn = (float*)(A + o_attn); k.hbuf = (float*)(A + o_h);
+  k.tmaps = A + o_maps;
+  k.x = (float*)(A + o_x); k.q = (float*)(A + o_q);
+  auto carve = [&](size_t o, int ld, __nv_bfloat16** t, float** f) {
+    *t = (__nv_bfloat16*)(A + o);
+    *f = (float*)(*t + (size_t)ntiles * 2 * ld * 8);
+  };
+  carve(o_ax, ld_x, &k.ax_t, &k.ax_f);
+  carve(o_aa, ld_a, &k.aa_t, &k.aa_f);
+  carve(o_ah, ld_h, &k.ah_t, &k.ah_f);
+  k.ld_x = ld_x; k.ld_a = ld_a; k.ld_h = ld_h;
   k.ssq = (float*)(A + o_ssq); k.ssq_stride = ssq_stride; k.part = (float*)(A + o_part);
   k.lmpart = (float2*)(A + o_lm);
   k.ctr = (uint32_t*)(A + o_ctr); k.cmb = (uint32_t*)(A + o_cmb); k.ctl = (uint32_t*)(A + o_ctl);
@@ -176,6 +254,7 @@ MK_API int mk_create_from_plan(mk_plan_t plan, const mk_weight_ptrs* w, int32_t 
   k.rope = (const float2*)(A + o_rope);
   k.timeout_ns = 1000000000ull;
   k.dbg = nullptr;
+  k.trace = nullptr;
   h->d_stage = (int32_t*)(A + o_stage);
   h->d_logits = (float*)(A + o_logits);
   h->d_argmax = (int32_t*)(A + o_argmax);
@@ -291,6 +370,22 @@ MK_API int mk_set_debug(mk_handle_t h, float* layer_hidden) {
   if (!h) return MK_ERR_INVALID_ARG;
   h->kp.dbg = layer_hidden;
   return MK_OK;
+}
+
+MK_API int mk_set_trace(mk_handle_t h, uint64_t* records, int64_t capacity) {
+  if (!h) return MK_ERR_INVALID_ARG;
+  int64_t n = 0;
+  for (const auto& s : h->plan.streams) n += (int64_t)s.size();
+  if (records && capacity < n) return fail(h, MK_ERR_INVALID_ARG, "mk_set_trace: capacity below the task count");
+  h->kp.trace = (unsigned long long*)records;
+  return MK_OK;
+}
+
+MK_API int64_t mk_num_tasks(mk_handle_t h) {
+  if (!h) return MK_ERR_INVALID_ARG;
+  int64_t n = 0;
+  for (const auto& s : h->plan.streams) n += (int64_t)s.size();
+  return n;
 }
 
 MK_API int mk_set_timeout_ns(mk_handle_t h, uint64_t ns) {

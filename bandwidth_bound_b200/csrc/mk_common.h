@@ -22,15 +22,19 @@ namespace mk {
 
 // ---- launch geometry -------------------------------------------------------------------
 constexpr int kConsumerWarps = 8;                       // compute warps per CTA
-constexpr int kThreads = (kConsumerWarps + 1) * 32;     // + one producer (bulk-copy) warp
-constexpr int kSlotBytes = 36 * 1024;                   // one pool stage
-constexpr int kNumSlots = 5;                            // pool depth (180 KB)
+constexpr int kThreads = (kConsumerWarps + 1) * 32;     // + one producer (TMA) warp
+constexpr int kWeightBytes = 32 * 1024;                 // weight (or KV) part of a pool stage
+constexpr int kOperandBytes = 16 * 1024;                // GEMV operand part of a pool stage
+constexpr int kSlotBytes = kWeightBytes + kOperandBytes; // one pool stage (1024-byte aligned)
+constexpr int kNumSlots = 4;                            // pool depth (192 KB)
 constexpr int kMaxBatch = 16;
 constexpr int kMaxBlocks = 8;                           // 8-row blocks per GEMV task (64 rows)
 constexpr int kPage = 16;                               // tokens per KV page
 constexpr int kMaxChunksPerSeq = 32;                    // split-K chunks per (sequence, kv head)
-constexpr int kRedBytes = kConsumerWarps * kMaxBlocks * 8 * kMaxBatch * 4;   // 32 KB
+constexpr int kRedBytes = kConsumerWarps * kMaxBlocks * 8 * 8 * 4;   // 16 KB: one 8-row batch tile at a time
 constexpr int kNoCounter = 0xFFFF;
+constexpr int kBoxCols = 64;                            // weight columns per TMA box (128 bytes, 128B swizzle)
+constexpr int kNumMats = 7;                             // wq wk wv wo w_gate w_up w_down
 
 // ---- task descriptors -------------------------------------------------------------------
 enum Op : uint8_t {
@@ -71,19 +75,36 @@ MK_HD int num_ssq_inst(int L) { return 1 + 2 * L; }
 
 // ---- units ------------------------------------------------------------------------------
 MK_HD int rows_per_unit(int op) { return (op == OP_QKV || op == OP_GATEUP) ? 16 : 8; }
+MK_HD int max_units(int op) { return (op == OP_QKV || op == OP_GATEUP) ? kMaxBlocks / 2 : kMaxBlocks; }
 
-// Row pitch of a GEMV stage in shared memory: 2*kc bytes rounded to 16, then padded
-// to 64 mod 128 so that the 8 lanes of a quarter warp (two rows, four 16-byte
-// chunks each) hit eight distinct bank groups.
-MK_HD uint32_t stage_pitch(uint32_t kc) {
-  uint32_t p = (2u * kc + 15u) & ~15u;
-  p += (64u + 128u - (p & 127u)) & 127u;
-  return p;
+MK_HD uint32_t ceil_div(uint32_t a, uint32_t b) { return (a + b - 1) / b; }
+MK_HD int round_up(int a, int b) { return (a + b - 1) / b * b; }
+
+// K columns per pool stage of a GEMV task with `blocks` 8-row blocks: the weights fit
+// kWeightBytes, the operand slice (2 bf16 parts x 8-row batch tiles x 16 bytes per 8
+// columns) fits kOperandBytes, and every consumer warp gets whole 32-column blocks.
+MK_HD int stage_cols(int blocks, int K, int max_batch) {
+  const int tiles = (max_batch + 7) / 8;
+  int kc = blocks >= 5 ? 256 : 512;
+  while (kc > 256 && tiles * 2 * kc * 16 > kOperandBytes) kc -= 256;
+  const int kp = round_up(K, kBoxCols);
+  return kp <= kc ? kp : kc;
 }
+
+// Operand tile layout in global memory (written by the producing epilogues, copied
+// into a pool stage with one bulk copy per tile and part): for batch tile mt (rows
+// 8mt..8mt+7) and part (0 hi, 1 lo), groups of 8 columns; group kg holds 8 rows of 16
+// bytes, row g stored in slot g ^ (2 * ((kg >> 1) & 3)) so that a quarter warp's
+// reads (two rows, four column groups) hit eight distinct bank groups.
+MK_HD size_t operand_index(int mt, int part, int kg, int g, int e, int ld) {
+  return ((((size_t)(mt * 2 + part) * (ld / 8) + kg) * 8 + (g ^ (2 * ((kg >> 1) & 3)))) * 8 + e);
+}
+
+// Index of the TMA descriptor of weight matrix `mat` (0 wq .. 6 w_down) of a layer for
+// boxes of 8*n rows; the LM head's maps follow the layers' (mat 0 of layer L).
+MK_HD int tmap_index(int layer, int mat, int n) { return (layer * kNumMats + mat) * kMaxBlocks + (n - 1); }
 
 // Tokens per attention stage: K rows then V rows of the same tokens, 32 KB total.
 MK_HD int attn_stage_tokens(int head_dim) { return head_dim == 64 ? 128 : 64; }
-
-MK_HD uint32_t ceil_div(uint32_t a, uint32_t b) { return (a + b - 1) / b; }
 
 }  // namespace mk

@@ -23,21 +23,26 @@
 namespace mk {
 
 typedef __nv_bfloat16 bf16;
+struct alignas(64) CUtensorMapLike {  // the driver's opaque 128-byte TMA descriptor
+  unsigned long long v[16];
+};
 
 // ---------------------------------------------------------------------------------------
 // shared memory
 
 struct Smem {
-  alignas(128) uint8_t pool[kNumSlots][kSlotBytes];
+  alignas(1024) uint8_t pool[kNumSlots][kSlotBytes];  // per slot: weights/KV, then GEMV operands
   alignas(16) float red[kRedBytes / 4];                 // GEMV cross-warp partials / attention merge
   alignas(16) float ep[kMaxBlocks * 8][kMaxBatch];       // per-task results [row][batch]
   alignas(16) float pw[kConsumerWarps][16 * 8];          // attention probabilities [token][head]
   float mw[kConsumerWarps][8], lw[kConsumerWarps][8];    // attention merge state per warp
   float corr[kConsumerWarps][8];
   float inv_rms[kMaxBatch];
-  alignas(8) uint64_t full[kNumSlots];
-  alignas(8) uint64_t empty[kNumSlots];
+  alignas(8) uint64_t full[kNumSlots];                   // weight/KV bytes of the stage landed
+  alignas(8) uint64_t ofull[kNumSlots];                  // operand bytes of the stage landed
+  alignas(8) uint64_t empty[kNumSlots];                  // all consumer warps done with the stage
   int attn_ch, attn_n, bad, flag, flag2;
+  unsigned long long wait_ns;  // time warp 0 spent waiting for pool slots in the current task (tracing)
 };
 
 size_t kernel_smem_bytes() { return sizeof(Smem); }
@@ -79,6 +84,27 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
       : "memory");
+}
+// Tiled TMA loads of a box of a weight matrix (128-byte swizzle), completion on an mbarrier.
+__device__ __forceinline__ void tma_2d(void* dst, const void* map, int c0, int c1, uint64_t* bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(c0), "r"(c1), "r"(smem_u32(bar)), "l"(pol)
+      : "memory");
+}
+__device__ __forceinline__ void tma_3d(void* dst, const void* map, int c0, int c1, int c2, uint64_t* bar,
+                                       uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar)), "l"(pol)
+      : "memory");
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
 }
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
@@ -156,9 +182,18 @@ __device__ bool mbar_wait(const KParams& p, uint64_t* bar, uint32_t parity) {
 }
 
 // Warp-uniform variant: lane 0 waits, the result is broadcast.
-__device__ __forceinline__ bool mbar_wait_warp(const KParams& p, uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_warp(const KParams& p, uint64_t* bar, uint32_t parity,
+                                               unsigned long long* wait_acc = nullptr) {
   int ok = 0;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(p, bar, parity) ? 1 : 0;
+  if ((threadIdx.x & 31) == 0) {
+    if (wait_acc && !mbar_try(bar, parity)) {
+      const uint64_t t0 = gtimer();
+      ok = mbar_wait(p, bar, parity) ? 1 : 0;
+      *wait_acc += gtimer() - t0;
+    } else {
+      ok = mbar_wait(p, bar, parity) ? 1 : 0;
+    }
+  }
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
@@ -188,27 +223,29 @@ __device__ __forceinline__ int gemv_K_dev(const KParams& p, int op) {
   return op == OP_OPROJ ? p.qdim : (op == OP_DOWN ? p.F : p.d);
 }
 
-// Device address of row r (0-based within the task) of a GEMV task's weight rows.
-__device__ __forceinline__ const bf16* task_row(const KParams& p, const TaskDesc& t, int r) {
-  const LayerW& w = p.layers[t.layer];
+// Issue the TMA box(es) of 64-column chunk c of one GEMV stage.  Chunk layout in the
+// slot: rows of the task, 128 bytes each, swizzled; QKV: first-half rows then the
+// matching second-half rows of one head; gate/up: gate rows then up rows.
+__device__ __forceinline__ void issue_gemv_chunk(const KParams& p, const TaskDesc& t, int k, uint8_t* dst,
+                                                 uint64_t* bar, uint64_t pol) {
+  const CUtensorMapLike* maps = reinterpret_cast<const CUtensorMapLike*>(p.tmaps);
+  const int n = t.nunits;
   switch (t.op) {
     case OP_QKV: {
-      const int u = t.u0 + (r >> 4), ru = r & 15;
       const int per_head = p.hd >> 4;
-      const int hh = u / per_head, m = u - hh * per_head;
-      const int row = (ru < 8) ? (8 * m + ru) : (p.hd / 2 + 8 * m + ru - 8);
-      const bf16* base = hh < p.nq ? w.wq + (size_t)hh * p.hd * p.d
-                         : hh < p.nq + p.nkv ? w.wk + (size_t)(hh - p.nq) * p.hd * p.d
-                                             : w.wv + (size_t)(hh - p.nq - p.nkv) * p.hd * p.d;
-      return base + (size_t)row * p.d;
+      const int hh = (int)t.u0 / per_head, m0 = (int)t.u0 - hh * per_head;
+      const int mat = hh < p.nq ? 0 : (hh < p.nq + p.nkv ? 1 : 2);
+      const int lh = mat == 0 ? hh : (mat == 1 ? hh - p.nq : hh - p.nq - p.nkv);
+      tma_3d(dst, maps + tmap_index(t.layer, mat, n), k, 8 * m0, 2 * lh, bar, pol);
+      break;
     }
-    case OP_GATEUP: {
-      const int u = t.u0 + (r >> 4), ru = r & 15;
-      return (ru < 8 ? w.wg : w.wu) + (size_t)(8 * u + (ru & 7)) * p.d;
-    }
-    case OP_OPROJ: return w.wo + (size_t)(8 * t.u0 + r) * p.qdim;
-    case OP_DOWN: return w.wd + (size_t)(8 * t.u0 + r) * p.F;
-    default: return p.lm_head + (size_t)(8 * t.u0 + r) * p.d;
+    case OP_GATEUP:
+      tma_2d(dst, maps + tmap_index(t.layer, 4, n), k, 8 * (int)t.u0, bar, pol);
+      tma_2d(dst + 8 * n * 128, maps + tmap_index(t.layer, 5, n), k, 8 * (int)t.u0, bar, pol);
+      break;
+    case OP_OPROJ: tma_2d(dst, maps + tmap_index(t.layer, 3, n), k, 8 * (int)t.u0, bar, pol); break;
+    case OP_DOWN: tma_2d(dst, maps + tmap_index(t.layer, 6, n), k, 8 * (int)t.u0, bar, pol); break;
+    default: tma_2d(dst, maps + tmap_index(p.L, 0, n), k, 8 * (int)t.u0, bar, pol); break;
   }
 }
 
@@ -268,90 +305,199 @@ __device__ void attn_setup(const KParams& p, int* ch_out, int* n_out) {
 // ---------------------------------------------------------------------------------------
 // producer warp: streams weight rows and prior KV pages into the slot ring
 
+struct Operand {
+  const bf16* tiles;
+  const float* f;
+  int ld;
+};
+
+__device__ __forceinline__ Operand operand_of(const KParams& p, int op) {
+  switch (op) {
+    case OP_OPROJ: return {p.aa_t, p.aa_f, p.ld_a};
+    case OP_DOWN: return {p.ah_t, p.ah_f, p.ld_h};
+    default: return {p.ax_t, p.ax_f, p.ld_x};
+  }
+}
+
 __device__ __forceinline__ int attn_stages(const AttnWork& a, int T) { return (a.c1 - a.c0 + T - 1) / T; }
 
+// Stages (pool slots) a task occupies: K / kc for a GEMV, its pages for an attention slot.
+__device__ __forceinline__ int task_stages(const KParams& p, const Smem& sm, const TaskDesc& t, AttnWork& a) {
+  if (t.op == OP_EMBED) return 0;
+  if (t.op == OP_ATTN) {
+    if ((int)t.u0 >= sm.attn_n || !attn_work(p, sm.attn_ch, (int)t.u0, a)) return 0;
+    return attn_stages(a, attn_stage_tokens(p.hd));
+  }
+  const int K = gemv_K_dev(p, t.op);
+  return (K + t.kc - 1) / t.kc;
+}
+
+// Weights (or KV pages) of stage s of task t into slot `slot`.  Returns false on a bad page id.
+__device__ bool issue_weights(const KParams& p, Smem& sm, const TaskDesc& t, const AttnWork& a, int s, int slot,
+                              uint64_t pol) {
+  const int lane = threadIdx.x & 31;
+  if (t.op == OP_ATTN) {
+    const int T = attn_stage_tokens(p.hd);
+    const int newpos = a.n - 1;
+    const int t0 = a.c0 + s * T, t1 = min(t0 + T, a.c1);
+    const int tp = min(t1, newpos);  // prior entries only; the new one is read after the wait
+    bool bad = false;
+    for (int pg = t0 / kPage; pg * kPage < tp; ++pg) {
+      const int id = p.ptable[a.i * p.mpps + pg];
+      if (id < 0 || id >= p.num_pages) bad = true;
+    }
+    if (bad) return false;
+    const uint32_t bytes = tp > t0 ? (uint32_t)(tp - t0) * p.hd * 2u * 2u : 0u;
+    if (lane == 0) {
+      if (bytes) mbar_expect_tx(&sm.full[slot], bytes);
+      else mbar_arrive(&sm.full[slot]);
+    }
+    __syncwarp();
+    if (bytes) {
+      const size_t head_stride = (size_t)kPage * p.hd;
+      uint8_t* kdst = sm.pool[slot];
+      uint8_t* vdst = sm.pool[slot] + (size_t)T * p.hd * 2;
+      const int pg0 = t0 / kPage;
+      const int npg = (tp - 1) / kPage - pg0 + 1;
+      for (int k = lane; k < 2 * npg; k += 32) {
+        const int pg = pg0 + (k >> 1);
+        const int r0 = max(pg * kPage, t0), r1 = min(pg * kPage + kPage, tp);
+        const int id = p.ptable[a.i * p.mpps + pg];
+        const size_t off = (((size_t)t.layer * p.num_pages + id) * p.nkv + a.h) * head_stride +
+                           (size_t)(r0 - pg * kPage) * p.hd;
+        const uint32_t nb = (uint32_t)(r1 - r0) * p.hd * 2u;
+        if (k & 1) bulk_g2s(vdst + (size_t)(r0 - t0) * p.hd * 2, p.vpool + off, nb, &sm.full[slot], pol);
+        else bulk_g2s(kdst + (size_t)(r0 - t0) * p.hd * 2, p.kpool + off, nb, &sm.full[slot], pol);
+      }
+    }
+    return true;
+  }
+  const int K = gemv_K_dev(p, t.op);
+  const int R = t.nunits * rows_per_unit(t.op);
+  const int kc0 = s * t.kc;
+  const int nch = (min((int)t.kc, K - kc0) + kBoxCols - 1) / kBoxCols;
+  if (lane == 0) mbar_expect_tx(&sm.full[slot], (uint32_t)(nch * R * 128));
+  __syncwarp();
+  for (int c = lane; c < nch; c += 32)
+    issue_gemv_chunk(p, t, kc0 + c * kBoxCols, sm.pool[slot] + (size_t)c * R * 128, &sm.full[slot], pol);
+  return true;
+}
+
+// Operand slice of GEMV stage s of task t into the operand part of slot `slot`: one bulk
+// copy per batch tile and bf16 part (batch >= 2), or the fp32 row (batch 1).
+__device__ void issue_operand(const KParams& p, Smem& sm, const TaskDesc& t, int s, int slot) {
+  const int lane = threadIdx.x & 31;
+  const Operand op = operand_of(p, t.op);
+  const int K = gemv_K_dev(p, t.op);
+  const int kc0 = s * t.kc;
+  const int cols = ((min((int)t.kc, K - kc0) + kBoxCols - 1) / kBoxCols) * kBoxCols;
+  uint8_t* dst = sm.pool[slot] + kWeightBytes;
+  // one lane issues: it is the lane whose acquire of the dependency counter ordered the reads
+  if (lane == 0) {
+    const uint64_t pol = policy_evict_last();
+    if (p.b == 1) {
+      mbar_expect_tx(&sm.ofull[slot], (uint32_t)cols * 4u);
+      bulk_g2s(dst, op.f + kc0, (uint32_t)cols * 4u, &sm.ofull[slot], pol);
+    } else {
+      const int nt = (p.b + 7) >> 3;
+      mbar_expect_tx(&sm.ofull[slot], (uint32_t)(nt * 2 * cols * 16));
+      for (int q = 0; q < 2 * nt; ++q) {
+        const bf16* src = op.tiles + operand_index(q >> 1, q & 1, kc0 / 8, 0, 0, op.ld);
+        bulk_g2s(dst + (size_t)q * t.kc * 16, src, (uint32_t)cols * 16u, &sm.ofull[slot], pol);
+      }
+    }
+  }
+  __syncwarp();
+}
+
+// The producer warp: one event loop with two cursors over the CTA's stream of stages.
+// The weight cursor streams weights and prior KV pages as far ahead as free slots
+// allow - weights do not depend on this step's activations.  The operand cursor
+// follows it and fills a GEMV stage's operand part as soon as the task's dependency
+// counter is met (other stages get a bare arrival so every slot's phases stay aligned).
 __device__ void producer(const KParams& p, Smem& sm, const TaskDesc* ts, int nt) {
   const int lane = threadIdx.x & 31;
   const uint64_t pol = policy_evict_first();
-  uint32_t stage = 0;
-  bool ok = true;
-  const int T = attn_stage_tokens(p.hd);
-  for (int ti = 0; ti < nt && ok; ++ti) {
-    const TaskDesc t = ts[ti];
-    if (t.op == OP_EMBED) continue;
-    if (t.op == OP_ATTN) {
-      AttnWork a;
-      if ((int)t.u0 >= sm.attn_n || !attn_work(p, sm.attn_ch, (int)t.u0, a)) continue;
-      const int newpos = a.n - 1;
-      const int nst = attn_stages(a, T);
-      const size_t head_stride = (size_t)kPage * p.hd;  // elements per (page, kv head) block
-      for (int s = 0; s < nst && ok; ++s, ++stage) {
-        const int slot = stage % kNumSlots;
-        if (!mbar_wait_warp(p, &sm.empty[slot], ((stage / kNumSlots) & 1) ^ 1)) { ok = false; break; }
-        const int t0 = a.c0 + s * T, t1 = min(t0 + T, a.c1);
-        const int tp = min(t1, newpos);  // prior entries only; the new one is read after the wait
-        // bytes of this stage
-        uint32_t bytes = tp > t0 ? (uint32_t)(tp - t0) * p.hd * 2u * 2u : 0u;
-        // validate pages first (every lane checks the same pages)
-        bool bad = false;
-        for (int pg = t0 / kPage; pg * kPage < tp; ++pg) {
-          const int id = p.ptable[a.i * p.mpps + pg];
-          if (id < 0 || id >= p.num_pages) bad = true;
+  uint32_t wk = 0, ok = 0;  // stages issued by the weight / operand cursor
+  int wt = 0, ws = 0, wn = -1, ot = 0, os = 0, on = -1;
+  bool odep = false, fail = false;
+  AttnWork wa, oa;
+  uint64_t idle_since = 0;
+  while (!fail && (wt < nt || ot < nt)) {
+    bool prog = false;
+    if (wt < nt) {
+      const TaskDesc t = ts[wt];
+      if (wn < 0) wn = task_stages(p, sm, t, wa);
+      if (ws >= wn) {
+        ++wt; ws = 0; wn = -1; prog = true;
+      } else {
+        const int slot = wk % kNumSlots;
+        int ready = 0;
+        if (lane == 0) ready = mbar_try(&sm.empty[slot], ((wk / kNumSlots) & 1) ^ 1) ? 1 : 0;
+        if (__shfl_sync(0xffffffffu, ready, 0)) {
+          if (!issue_weights(p, sm, t, wa, ws, slot, pol)) {
+            if (lane == 0) raise_error(p, -6 /* MK_ERR_BOUNDS */);
+            fail = true;
+            break;
+          }
+          ++wk; ++ws; prog = true;
         }
-        if (bad) {
-          if (lane == 0) raise_error(p, -6 /* MK_ERR_BOUNDS */);
-          ok = false;
-          break;
-        }
-        if (lane == 0) {
-          if (bytes) mbar_expect_tx(&sm.full[slot], bytes);
-          else mbar_arrive(&sm.full[slot]);
-        }
-        __syncwarp();
-        if (bytes) {
-          uint8_t* kdst = sm.pool[slot];
-          uint8_t* vdst = sm.pool[slot] + (size_t)T * p.hd * 2;
-          const int pg0 = t0 / kPage;
-          const int npg = (tp - 1) / kPage - pg0 + 1;
-          for (int k = lane; k < 2 * npg; k += 32) {
-            const int pg = pg0 + (k >> 1);
-            const int r0 = max(pg * kPage, t0), r1 = min(pg * kPage + kPage, tp);
-            const int id = p.ptable[a.i * p.mpps + pg];
-            const size_t off = (((size_t)t.layer * p.num_pages + id) * p.nkv + a.h) * head_stride +
-                               (size_t)(r0 - pg * kPage) * p.hd;
-            const uint32_t nb = (uint32_t)(r1 - r0) * p.hd * 2u;
-            if (k & 1) bulk_g2s(vdst + (size_t)(r0 - t0) * p.hd * 2, p.vpool + off, nb, &sm.full[slot], pol);
-            else bulk_g2s(kdst + (size_t)(r0 - t0) * p.hd * 2, p.kpool + off, nb, &sm.full[slot], pol);
+      }
+    }
+    if (ot < nt) {
+      const TaskDesc t = ts[ot];
+      if (on < 0) { on = task_stages(p, sm, t, oa); odep = false; }
+      if (os >= on) {
+        ++ot; os = 0; on = -1; prog = true;
+      } else if (ok < wk) {  // a stage's operand part follows its weights into the slot
+        const int slot = ok % kNumSlots;
+        if (t.op == OP_ATTN) {
+          if (lane == 0) mbar_arrive(&sm.ofull[slot]);
+          __syncwarp();
+          ++ok; ++os; prog = true;
+        } else {
+          if (!odep) {
+            int met = 1;
+            if (lane == 0 && t.wait_ctr != kNoCounter)
+              met = (int32_t)(ld_acquire(p.ctr + t.wait_ctr) - t.wait_count * p.epoch) >= 0 ? 1 : 0;
+            odep = __shfl_sync(0xffffffffu, met, 0) != 0;
+            if (odep) asm volatile("fence.proxy.async.global;" ::: "memory");
+          }
+          if (odep) {
+            issue_operand(p, sm, t, os, slot);
+            ++ok; ++os; prog = true;
           }
         }
       }
-      continue;
     }
-    // GEMV task
-    const int K = gemv_K_dev(p, t.op);
-    const int kc = t.kc;
-    const int R = t.nunits * rows_per_unit(t.op);
-    const uint32_t pitch = stage_pitch(kc);
-    const int nst = (K + kc - 1) / kc;
-    for (int s = 0; s < nst; ++s, ++stage) {
-      const int slot = stage % kNumSlots;
-      if (!mbar_wait_warp(p, &sm.empty[slot], ((stage / kNumSlots) & 1) ^ 1)) { ok = false; break; }
-      const int kc0 = s * kc;
-      const int kcl = min(kc, K - kc0);
-      const uint32_t rb = (uint32_t)kcl * 2u;
-      if (lane == 0) mbar_expect_tx(&sm.full[slot], rb * (uint32_t)R);
-      __syncwarp();
-      for (int r = lane; r < R; r += 32)
-        bulk_g2s(sm.pool[slot] + (size_t)r * pitch, task_row(p, t, r) + kc0, rb, &sm.full[slot], pol);
+    if (prog) {
+      idle_since = 0;
+    } else {
+      __nanosleep(32);
+      if (lane == 0) {
+        const uint64_t now = gtimer();
+        if (idle_since == 0) idle_since = now;
+        int stop = 0;
+        if (aborted(p)) stop = 1;
+        else if (now - idle_since > p.timeout_ns) { raise_error(p, -5 /* MK_ERR_DEVICE_TIMEOUT */); stop = 1; }
+        fail = stop;
+      }
+      fail = __shfl_sync(0xffffffffu, fail ? 1 : 0, 0) != 0;
     }
   }
-  if (!ok) {
+  if (fail) {
     // Drain: let every copy already issued land before the CTA may exit.
     if (lane == 0) {
-      const uint32_t first = stage > (uint32_t)kNumSlots ? stage - kNumSlots : 0u;
-      for (uint32_t s = first; s < stage; ++s) {
+      const uint32_t first = wk > (uint32_t)kNumSlots ? wk - kNumSlots : 0u;
+      for (uint32_t s = first; s < wk; ++s) {
         const uint64_t t0 = gtimer();
         while (!mbar_try(&sm.full[s % kNumSlots], (s / kNumSlots) & 1))
+          if (gtimer() - t0 > p.timeout_ns) break;
+      }
+      const uint32_t ofirst = ok > (uint32_t)kNumSlots ? ok - kNumSlots : 0u;
+      for (uint32_t s = ofirst; s < ok; ++s) {
+        const uint64_t t0 = gtimer();
+        while (!mbar_try(&sm.ofull[s % kNumSlots], (s / kNumSlots) & 1))
           if (gtimer() - t0 > p.timeout_ns) break;
       }
     }
@@ -375,112 +521,81 @@ __device__ void compute_inv_rms(const KParams& p, Smem& sm, int inst, int nparts
   }
 }
 
-// Load 8 consecutive activations [k, k+8) of batch row bi, optionally RMS-normalised.
-__device__ __forceinline__ void load_act8(const float* src, int ld, int bi, int k, const float* inv_rms,
-                                          const bf16* gain, float (&a)[8]) {
-  const float* s = src + (size_t)bi * ld + k;
-  const float4 v0 = __ldcg(reinterpret_cast<const float4*>(s));
-  const float4 v1 = __ldcg(reinterpret_cast<const float4*>(s + 4));
-  a[0] = v0.x; a[1] = v0.y; a[2] = v0.z; a[3] = v0.w;
-  a[4] = v1.x; a[5] = v1.y; a[6] = v1.z; a[7] = v1.w;
-  if (gain) {
-    const uint4 gv = __ldg(reinterpret_cast<const uint4*>(gain + k));
-    const float r = inv_rms[bi];
-    a[0] *= r * bf_lo(gv.x); a[1] *= r * bf_hi(gv.x);
-    a[2] *= r * bf_lo(gv.y); a[3] *= r * bf_hi(gv.y);
-    a[4] *= r * bf_lo(gv.z); a[5] *= r * bf_hi(gv.z);
-    a[6] *= r * bf_lo(gv.w); a[7] *= r * bf_hi(gv.w);
-  }
+// Store one GEMV operand value (batch row bi, column k): bf16 hi part and bf16 lo part
+// (the remainder) into the tile layout, and fp32 for batch row 0.
+__device__ __forceinline__ void put_operand(bf16* tiles, float* f, int ld, int bi, int k, float v) {
+  const bf16 h = __float2bfloat16_rn(v);
+  const int mt = bi >> 3, g = bi & 7, kg = k >> 3, e = k & 7;
+  tiles[operand_index(mt, 0, kg, g, e, ld)] = h;
+  tiles[operand_index(mt, 1, kg, g, e, ld)] = __float2bfloat16_rn(v - __bfloat162float(h));
+  if (bi == 0) f[k] = v;
 }
 
-// Stream the task's stages through the warps and reduce into sm.ep[row][batch].
-// MT = 0: CUDA-core FMA (batch 1); MT = 1, 2: mma.sync with MT tiles of 8 batch rows,
-// each row split into bf16 hi + lo parts (rows 0-7 hi, 8-15 lo of the M = 16 tile).
-template <int MT>
-__device__ void gemv_body(const KParams& p, Smem& sm, const TaskDesc& t, uint32_t& stage, bool& ab,
-                          const float* src, int ld, const bf16* gain) {
+// Stream the task's stages through the eight warps and reduce into sm.ep[row][batch].
+// Weight stage layout (per 64-column chunk): 8*G rows of 128 bytes, 16-byte chunks
+// swizzled (chunk c of row r at c ^ (r & 7)).  Warp w takes 32-column k blocks w, w+8,
+// ...; a k block is the even (h = 0) or odd (h = 1) 16-byte chunks of a 64-column
+// chunk, so lane (g, tq) reads chunk 2*tq + h of row 8j + g - conflict-free - which
+// holds columns 16*tq + 8*h .. +7.  The operand of those columns sits in the stage's
+// operand part: column group kg = 8*chunk + 2*tq + h, row g at slot g ^ 2tq.
+// MT = 0: CUDA-core FMA (batch 1, fp32 operand); MT = 1, 2: mma.sync with MT tiles of
+// 8 batch rows, rows 0-7 of the M = 16 tile the bf16 hi parts, rows 8-15 the lo parts.
+template <int MT, int G>
+__device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDesc t, uint32_t& stage, bool& ab) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, tq = lane & 3;
   const int K = gemv_K_dev(p, t.op);
   const int kc = t.kc;
-  const int G = t.nunits * rows_per_unit(t.op) / 8;
-  const uint32_t pitch = stage_pitch(kc);
   const int nst = (K + kc - 1) / kc;
-  const float* inv = sm.inv_rms;
-
-  constexpr int NACC = MT == 0 ? 1 : MT * 4;
-  float acc[kMaxBlocks][NACC];
+  constexpr int R = 8 * G;
+  constexpr int NMT = MT == 0 ? 1 : MT;
+  float acc[G][NMT][4];
 #pragma unroll
-  for (int j = 0; j < kMaxBlocks; ++j)
+  for (int j = 0; j < G; ++j)
 #pragma unroll
-    for (int e = 0; e < NACC; ++e) acc[j][e] = 0.f;
+    for (int mt = 0; mt < NMT; ++mt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[j][mt][e] = 0.f;
+  const int opart = kc * 16;  // bytes of one (tile, part) slice in the operand area
 
   for (int s = 0; s < nst; ++s, ++stage) {
     const int slot = stage % kNumSlots;
-    if (!ab) ab = !mbar_wait_warp(p, &sm.full[slot], (stage / kNumSlots) & 1);
+    const uint32_t par = (stage / kNumSlots) & 1;
+    if (!ab) ab = !mbar_wait_warp(p, &sm.full[slot], par, (p.trace && threadIdx.x == 0) ? &sm.wait_ns : nullptr);
+    if (!ab) ab = !mbar_wait_warp(p, &sm.ofull[slot], par, (p.trace && threadIdx.x == 0) ? &sm.wait_ns : nullptr);
     if (ab) continue;
     const uint8_t* tile = sm.pool[slot];
-    const int kc0 = s * kc;
-    const int kcl = min(kc, K - kc0);
-    const int nb = (kcl + 31) >> 5;
+    const uint8_t* opnd = sm.pool[slot] + kWeightBytes;
+    const int nb = 2 * ((min(kc, K - s * kc) + kBoxCols - 1) / kBoxCols);
     for (int kb = warp; kb < nb; kb += kConsumerWarps) {
-      const int kofs = kb * 32 + tq * 8;
-      const bool valid = kofs < kcl;
-      const int k = kc0 + kofs;
+      const int kgl = 8 * (kb >> 1) + 2 * tq + (kb & 1);
+      const uint8_t* chunk = tile + (size_t)(kb >> 1) * (R * 128) + ((((2 * tq + (kb & 1)) ^ g)) << 4);
+      uint4 A[2 * NMT];
       if constexpr (MT == 0) {
-        float a[8];
-        if (valid) load_act8(src, ld, 0, k, inv, gain, a);
-        else {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) a[e] = 0.f;
-        }
-#pragma unroll
-        for (int j = 0; j < kMaxBlocks; ++j) {
-          if (j < G) {
-            uint4 w = make_uint4(0, 0, 0, 0);
-            if (valid) w = *reinterpret_cast<const uint4*>(tile + (size_t)(8 * j + g) * pitch + kofs * 2);
-            float s0 = acc[j][0];
-            s0 = fmaf(bf_lo(w.x), a[0], s0); s0 = fmaf(bf_hi(w.x), a[1], s0);
-            s0 = fmaf(bf_lo(w.y), a[2], s0); s0 = fmaf(bf_hi(w.y), a[3], s0);
-            s0 = fmaf(bf_lo(w.z), a[4], s0); s0 = fmaf(bf_hi(w.z), a[5], s0);
-            s0 = fmaf(bf_lo(w.w), a[6], s0); s0 = fmaf(bf_hi(w.w), a[7], s0);
-            acc[j][0] = s0;
-          }
-        }
+        const uint4* f = reinterpret_cast<const uint4*>(opnd + (size_t)kgl * 32);
+        A[0] = f[0];
+        A[1] = f[1];
       } else {
-        uint32_t A[MT][8];
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          const int bi = mt * 8 + g;
-          float a[8];
-          if (valid && bi < p.b) load_act8(src, ld, bi, k, inv, gain, a);
-          else {
+        for (int q = 0; q < 2 * MT; ++q)
+          A[q] = *reinterpret_cast<const uint4*>(opnd + (size_t)q * opart + (size_t)kgl * 128 + ((g ^ (2 * tq)) << 4));
+      }
 #pragma unroll
-            for (int e = 0; e < 8; ++e) a[e] = 0.f;
-          }
-          float hi[8], lo[8];
+      for (int j = 0; j < G; ++j) {
+        const uint4 w = *reinterpret_cast<const uint4*>(chunk + (8 * j + g) * 128);
+        if constexpr (MT == 0) {
+          float s0 = acc[j][0][0];
+          s0 = fmaf(bf_lo(w.x), __uint_as_float(A[0].x), s0); s0 = fmaf(bf_hi(w.x), __uint_as_float(A[0].y), s0);
+          s0 = fmaf(bf_lo(w.y), __uint_as_float(A[0].z), s0); s0 = fmaf(bf_hi(w.y), __uint_as_float(A[0].w), s0);
+          s0 = fmaf(bf_lo(w.z), __uint_as_float(A[1].x), s0); s0 = fmaf(bf_hi(w.z), __uint_as_float(A[1].y), s0);
+          s0 = fmaf(bf_lo(w.w), __uint_as_float(A[1].z), s0); s0 = fmaf(bf_hi(w.w), __uint_as_float(A[1].w), s0);
+          acc[j][0][0] = s0;
+        } else {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            hi[e] = __bfloat162float(__float2bfloat16_rn(a[e]));
-            lo[e] = a[e] - hi[e];
-          }
-          // step 0: logical k (2t,2t+1) <- actual +0,+1 ; (2t+8,2t+9) <- +2,+3 ; step 1: +4..+7
-          A[mt][0] = pack_bf16(hi[0], hi[1]); A[mt][1] = pack_bf16(lo[0], lo[1]);
-          A[mt][2] = pack_bf16(hi[2], hi[3]); A[mt][3] = pack_bf16(lo[2], lo[3]);
-          A[mt][4] = pack_bf16(hi[4], hi[5]); A[mt][5] = pack_bf16(lo[4], lo[5]);
-          A[mt][6] = pack_bf16(hi[6], hi[7]); A[mt][7] = pack_bf16(lo[6], lo[7]);
-        }
-#pragma unroll
-        for (int j = 0; j < kMaxBlocks; ++j) {
-          if (j < G) {
-            uint4 w = make_uint4(0, 0, 0, 0);
-            if (valid) w = *reinterpret_cast<const uint4*>(tile + (size_t)(8 * j + g) * pitch + kofs * 2);
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
-              float(&d)[4] = *reinterpret_cast<float(*)[4]>(&acc[j][mt * 4]);
-              mma_bf16(d, A[mt][0], A[mt][1], A[mt][2], A[mt][3], w.x, w.y);
-              mma_bf16(d, A[mt][4], A[mt][5], A[mt][6], A[mt][7], w.z, w.w);
-            }
+          for (int mt = 0; mt < MT; ++mt) {
+            const uint4 H = A[2 * mt], L = A[2 * mt + 1];
+            mma_bf16(acc[j][mt], H.x, L.x, H.y, L.y, w.x, w.y);
+            mma_bf16(acc[j][mt], H.z, L.z, H.w, L.w, w.z, w.w);
           }
         }
       }
@@ -489,86 +604,95 @@ __device__ void gemv_body(const KParams& p, Smem& sm, const TaskDesc& t, uint32_
     if (lane == 0) mbar_arrive(&sm.empty[slot]);
   }
 
-  // cross-warp reduction: red[warp][block][batch][8 rows]
+  // cross-warp reduction, one 8-row batch tile at a time: red[warp][block][batch g][8 rows]
   float* red = sm.red;
-  if (!ab) {
 #pragma unroll
-    for (int j = 0; j < kMaxBlocks; ++j) {
-      if (j < G) {
+  for (int mt = 0; mt < NMT; ++mt) {
+    if (!ab) {
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
         if constexpr (MT == 0) {
-          float v = acc[j][0];
+          float v = acc[j][0][0];
           v += __shfl_xor_sync(0xffffffffu, v, 1);
           v += __shfl_xor_sync(0xffffffffu, v, 2);
-          if (tq == 0) red[((warp * kMaxBlocks + j) * kMaxBatch + 0) * 8 + g] = v;
+          if (tq == 0) red[((warp * kMaxBlocks + j) * 8 + 0) * 8 + g] = v;
         } else {
-#pragma unroll
-          for (int mt = 0; mt < MT; ++mt) {
-            const int bi = mt * 8 + g;
-            float2 y = make_float2(acc[j][mt * 4 + 0] + acc[j][mt * 4 + 2], acc[j][mt * 4 + 1] + acc[j][mt * 4 + 3]);
-            *reinterpret_cast<float2*>(&red[((warp * kMaxBlocks + j) * kMaxBatch + bi) * 8 + 2 * tq]) = y;
-          }
+          const float2 y = make_float2(acc[j][mt][0] + acc[j][mt][2], acc[j][mt][1] + acc[j][mt][3]);
+          *reinterpret_cast<float2*>(&red[((warp * kMaxBlocks + j) * 8 + g) * 8 + 2 * tq]) = y;
         }
       }
     }
-  }
-  cbar();
-  const int nb_items = G * 8 * p.b;
-  for (int idx = threadIdx.x; idx < nb_items; idx += kConsumerWarps * 32) {
-    const int bi = idx % p.b;
-    const int row = idx / p.b;  // 8*j + r
-    const int j = row >> 3, r = row & 7;
-    float s = 0.f;
+    cbar();
+    const int nb8 = min(8, p.b - mt * 8);
+    const int items = nb8 > 0 ? R * nb8 : 0;
+    for (int idx = threadIdx.x; idx < items; idx += kConsumerWarps * 32) {
+      const int bl = idx % nb8;
+      const int row = idx / nb8;  // 8*j + r
+      const int j = row >> 3, r = row & 7;
+      float sum = 0.f;
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) s += red[((w * kMaxBlocks + j) * kMaxBatch + bi) * 8 + r];
-    sm.ep[row][bi] = s;
+      for (int w = 0; w < kConsumerWarps; ++w) sum += red[((w * kMaxBlocks + j) * 8 + bl) * 8 + r];
+      sm.ep[row][mt * 8 + bl] = sum;
+    }
+    cbar();
   }
-  cbar();
+}
+
+template <int MT>
+__device__ void gemv_dispatch(const KParams& p, Smem& sm, const TaskDesc& t, uint32_t& stage, bool& ab, int G) {
+  switch (G) {
+    case 1: gemv_body<MT, 1>(p, sm, t, stage, ab); break;
+    case 2: gemv_body<MT, 2>(p, sm, t, stage, ab); break;
+    case 3: gemv_body<MT, 3>(p, sm, t, stage, ab); break;
+    case 4: gemv_body<MT, 4>(p, sm, t, stage, ab); break;
+    case 5: gemv_body<MT, 5>(p, sm, t, stage, ab); break;
+    case 6: gemv_body<MT, 6>(p, sm, t, stage, ab); break;
+    case 7: gemv_body<MT, 7>(p, sm, t, stage, ab); break;
+    default: gemv_body<MT, 8>(p, sm, t, stage, ab); break;
+  }
 }
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
+
+// Gain of the RMSNorm whose input the residual writer of (op, layer) produces.
+__device__ __forceinline__ const bf16* next_gain(const KParams& p, int op, int layer) {
+  if (op == OP_EMBED) return p.layers[0].attn_norm;
+  if (op == OP_OPROJ) return p.layers[layer].mlp_norm;
+  return layer + 1 < p.L ? p.layers[layer + 1].attn_norm : p.final_norm;
+}
 
 // ---------------------------------------------------------------------------------------
 // consumer task bodies
 
 __device__ void gemv_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_t& stage, bool& ab) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const LayerW& W = p.layers[t.layer];
-  const float* src;
-  int ld;
-  const bf16* gain = nullptr;
-  switch (t.op) {
-    case OP_QKV: src = p.x; ld = p.d; gain = W.attn_norm; break;
-    case OP_GATEUP: src = p.x; ld = p.d; gain = W.mlp_norm; break;
-    case OP_LMHEAD: src = p.x; ld = p.d; gain = p.final_norm; break;
-    case OP_OPROJ: src = p.attn; ld = p.qdim; break;
-    default: src = p.hbuf; ld = p.F; break;
-  }
-  if (gain && !ab) {
+  const bool norm = t.op == OP_QKV || t.op == OP_GATEUP || t.op == OP_LMHEAD;
+  if (norm && !ab) {
     const int inst = t.op == OP_GATEUP ? ssq_inst_oproj(t.layer)
                      : t.op == OP_QKV  ? (t.layer == 0 ? ssq_inst_embed() : ssq_inst_down(t.layer - 1))
                                        : ssq_inst_down(p.L - 1);
     compute_inv_rms(p, sm, inst, (int)t.wait_count);
   }
   cbar();
-  if (p.b == 1) gemv_body<0>(p, sm, t, stage, ab, src, ld, gain);
-  else if (p.b <= 8) gemv_body<1>(p, sm, t, stage, ab, src, ld, gain);
-  else gemv_body<2>(p, sm, t, stage, ab, src, ld, gain);
-
   const int G = t.nunits * rows_per_unit(t.op) / 8;
+  if (p.b == 1) gemv_dispatch<0>(p, sm, t, stage, ab, G);
+  else if (p.b <= 8) gemv_dispatch<1>(p, sm, t, stage, ab, G);
+  else gemv_dispatch<2>(p, sm, t, stage, ab, G);
+
   const int nthr = kConsumerWarps * 32;
+  const int n = t.nunits;
   if (t.op == OP_QKV) {
     if (!ab) {
       const int half = p.hd / 2, per_head = p.hd >> 4;
-      const int items = t.nunits * 8 * p.b;
+      const int hh = (int)t.u0 / per_head, m0 = (int)t.u0 - hh * per_head;
+      const int items = n * 8 * p.b;
       for (int idx = threadIdx.x; idx < items; idx += nthr) {
         const int bi = idx % p.b;
-        const int ur = idx / p.b;
-        const int ul = ur >> 3, r = ur & 7;
-        const int u = t.u0 + ul;
-        const int hh = u / per_head, m = u - hh * per_head;
-        const int j = 8 * m + r;
-        const float x1 = sm.ep[(2 * ul) * 8 + r][bi];
-        const float x2 = sm.ep[(2 * ul + 1) * 8 + r][bi];
+        const int row = idx / p.b;  // 0 .. 8n-1 within the first half
+        const int j = 8 * m0 + row;
+        const float r = sm.inv_rms[bi];
+        const float x1 = sm.ep[row][bi] * r;
+        const float x2 = sm.ep[8 * n + row][bi] * r;
         const int pos = p.pos[bi];
         if (hh < p.nq + p.nkv) {
           const float2 cs = p.rope[(size_t)pos * half + j];
@@ -596,20 +720,22 @@ __device__ void gemv_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_
     }
   } else if (t.op == OP_GATEUP) {
     if (!ab) {
-      const int items = t.nunits * 8 * p.b;
+      const int items = n * 8 * p.b;
       for (int idx = threadIdx.x; idx < items; idx += nthr) {
         const int bi = idx % p.b;
-        const int ur = idx / p.b;
-        const int ul = ur >> 3, r = ur & 7;
-        const float gv = sm.ep[(2 * ul) * 8 + r][bi];
-        const float uv = sm.ep[(2 * ul + 1) * 8 + r][bi];
-        p.hbuf[(size_t)bi * p.F + 8 * (t.u0 + ul) + r] = silu_f(gv) * uv;
+        const int row = idx / p.b;
+        const float r = sm.inv_rms[bi];
+        const float gv = sm.ep[row][bi] * r;
+        const float uv = sm.ep[8 * n + row][bi] * r;
+        put_operand(p.ah_t, p.ah_f, p.ld_h, bi, 8 * t.u0 + row, silu_f(gv) * uv);
       }
     }
   } else if (t.op == OP_OPROJ || t.op == OP_DOWN) {
     const int inst = t.op == OP_OPROJ ? ssq_inst_oproj(t.layer) : ssq_inst_down(t.layer);
     if (!ab) {
-      const int items = G * 8 * p.b;
+      const int rows = 8 * n;
+      const int items = rows * p.b;
+      const bf16* gain = next_gain(p, t.op, t.layer);
       float* dbg = (t.op == OP_DOWN && p.dbg) ? p.dbg + (size_t)(t.layer + 1) * p.max_b * p.d : nullptr;
       for (int idx = threadIdx.x; idx < items; idx += nthr) {
         const int bi = idx % p.b;
@@ -619,6 +745,7 @@ __device__ void gemv_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_
         const float xn = __ldcg(xp) + sm.ep[row][bi];
         *xp = xn;
         sm.ep[row][bi] = xn;
+        put_operand(p.ax_t, p.ax_f, p.ld_x, bi, grow, xn * __bfloat162float(gain[grow]));
         if (dbg) dbg[(size_t)bi * p.d + grow] = xn;
       }
     }
@@ -626,7 +753,7 @@ __device__ void gemv_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_
     if (!ab) {
       for (int bi = warp; bi < p.b; bi += kConsumerWarps) {
         float s = 0.f;
-        for (int row = lane; row < G * 8; row += 32) s += sm.ep[row][bi] * sm.ep[row][bi];
+        for (int row = lane; row < 8 * n; row += 32) s += sm.ep[row][bi] * sm.ep[row][bi];
 #pragma unroll
         for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
         if (lane == 0) p.ssq[(size_t)inst * p.ssq_stride + (size_t)t.task_idx * p.max_b + bi] = s;
@@ -634,28 +761,32 @@ __device__ void gemv_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_
     }
   } else {  // LM head
     if (!ab) {
-      const int items = G * 8 * p.b;
+      const int rows = 8 * n;
+      const int items = rows * p.b;
       for (int idx = threadIdx.x; idx < items; idx += nthr) {
         const int bi = idx % p.b;
         const int row = idx / p.b;
-        p.logits[(size_t)bi * p.V + 8 * t.u0 + row] = sm.ep[row][bi];
+        const float v = sm.ep[row][bi] * sm.inv_rms[bi];
+        sm.ep[row][bi] = v;
+        p.logits[(size_t)bi * p.V + 8 * t.u0 + row] = v;
       }
-      if (p.argmax) {
-        for (int bi = warp; bi < p.b; bi += kConsumerWarps) {
-          float best = -INFINITY;
-          int bidx = 0x7fffffff;
-          for (int row = lane; row < G * 8; row += 32) {
-            const float v = sm.ep[row][bi];
-            if (v > best) { best = v; bidx = 8 * t.u0 + row; }
-          }
-#pragma unroll
-          for (int o = 16; o; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, best, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bidx, o);
-            if (ov > best || (ov == best && oi < bidx)) { best = ov; bidx = oi; }
-          }
-          if (lane == 0) p.lmpart[(size_t)t.task_idx * p.max_b + bi] = make_float2(best, __int_as_float(bidx));
+    }
+    cbar();
+    if (!ab && p.argmax) {
+      for (int bi = warp; bi < p.b; bi += kConsumerWarps) {
+        float best = -INFINITY;
+        int bidx = 0x7fffffff;
+        for (int row = lane; row < 8 * n; row += 32) {
+          const float v = sm.ep[row][bi];
+          if (v > best) { best = v; bidx = 8 * t.u0 + row; }
         }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, best, o);
+          const int oi = __shfl_xor_sync(0xffffffffu, bidx, o);
+          if (ov > best || (ov == best && oi < bidx)) { best = ov; bidx = oi; }
+        }
+        if (lane == 0) p.lmpart[(size_t)t.task_idx * p.max_b + bi] = make_float2(best, __int_as_float(bidx));
       }
     }
   }
@@ -665,12 +796,14 @@ __device__ void embed_task(const KParams& p, Smem& sm, const TaskDesc& t, bool a
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (ab) return;
   const int c0 = 8 * t.u0, nc = 8 * t.nunits;
+  const bf16* gain = next_gain(p, OP_EMBED, 0);
   for (int bi = warp; bi < p.b; bi += kConsumerWarps) {
     const bf16* e = p.embed + (size_t)p.tok[bi] * p.d;
     float s = 0.f;
     for (int c = lane; c < nc; c += 32) {
       const float v = __bfloat162float(e[c0 + c]);
       p.x[(size_t)bi * p.d + c0 + c] = v;
+      put_operand(p.ax_t, p.ax_f, p.ld_x, bi, c0 + c, v * __bfloat162float(gain[c0 + c]));
       if (p.dbg) p.dbg[(size_t)bi * p.d + c0 + c] = v;
       s += v * v;
     }
@@ -686,7 +819,7 @@ __device__ void embed_task(const KParams& p, Smem& sm, const TaskDesc& t, bool a
 // eight warps, and - for the last chunk of (i, h) to finish - the log-sum-exp
 // combine of all chunks into the attention output.
 template <int HD>
-__device__ void attn_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_t& stage, bool& ab) {
+__device__ __noinline__ void attn_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_t& stage, bool& ab) {
   constexpr int T = HD == 64 ? 128 : 64;   // tokens per stage
   constexpr int TPW = T / kConsumerWarps;  // tokens per warp per stage: 16 or 8
   constexpr int NKB = HD / 32;             // 32-dim blocks
@@ -749,7 +882,11 @@ __device__ void attn_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_
     const int t0 = a.c0 + s * T, t1 = min(t0 + T, a.c1);
     const int ntok = t1 - t0;
     const bool has_new = newpos >= t0 && newpos < t1;
-    if (!ab) ab = !mbar_wait_warp(p, &sm.full[slot], (stage / kNumSlots) & 1);
+    if (!ab) ab = !mbar_wait_warp(p, &sm.full[slot], (stage / kNumSlots) & 1,
+                                  (p.trace && threadIdx.x == 0) ? &sm.wait_ns : nullptr);
+    // the operand cursor passes attention stages with a bare arrival; waiting on it keeps
+    // this slot's operand phases in step with the stage count
+    if (!ab) ab = !mbar_wait_warp(p, &sm.ofull[slot], (stage / kNumSlots) & 1);
     uint8_t* kreg = sm.pool[slot];
     uint8_t* vreg = sm.pool[slot] + (size_t)T * HD * 2;
     if (has_new) {
@@ -883,7 +1020,7 @@ __device__ void attn_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_
     for (int h = 0; h < 8; ++h)
       if (h < G)
 #pragma unroll
-        for (int e = 0; e < DPL; ++e) sm.red[(warp * 8 + h) * HD + lane * DPL + e] = acc[h][e];
+        for (int e = 0; e < DPL; ++e) sm.red[(warp * G + h) * HD + lane * DPL + e] = acc[h][e];
   }
   cbar();
   float* part = p.part + (size_t)t.u0 * G * (HD + 2);
@@ -897,7 +1034,7 @@ __device__ void attn_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_
 #pragma unroll
       for (int w = 0; w < kConsumerWarps; ++w) {
         const float f = sm.mw[w][h] == -INFINITY ? 0.f : exp2f(sm.mw[w][h] - M);
-        A += f * sm.red[(w * 8 + h) * HD + dd];
+        A += f * sm.red[(w * G + h) * HD + dd];
         Ls += f * sm.lw[w][h];
       }
       part[h * (HD + 2) + dd] = A;
@@ -921,20 +1058,38 @@ __device__ void attn_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_
   }
   cbar();
   if (sm.flag2) {
-    // log-sum-exp combine of the nc chunk states of (i, h)
+    // log-sum-exp combine of the nc (<= 32) chunk states of (i, h): one warp per head
+    // computes the chunk weights 2^(m_c - M) / sum_c 2^(m_c - M) l_c from all chunks at
+    // once, then every thread sums weighted partials with independent loads.
     const float* base = p.part + (size_t)(t.u0 - a.c) * G * (HD + 2);
+    float* wts = sm.red;  // [head][32]
+    const int warp = threadIdx.x >> 5;
+    for (int h = warp; h < G; h += kConsumerWarps) {
+      const float* pc = base + ((size_t)lane * G + h) * (HD + 2);
+      const float mc = lane < a.nc ? __ldcg(pc + HD) : -INFINITY;
+      const float lc = lane < a.nc ? __ldcg(pc + HD + 1) : 0.f;
+      float M = mc;
+#pragma unroll
+      for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+      const float f = lane < a.nc ? exp2f(mc - M) : 0.f;
+      float den = f * lc;
+#pragma unroll
+      for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+      wts[h * 32 + lane] = f / den;
+    }
+    cbar();
     for (int idx = threadIdx.x; idx < G * HD; idx += kConsumerWarps * 32) {
       const int h = idx / HD, dd = idx % HD;
-      float M = -INFINITY;
-      for (int c = 0; c < a.nc; ++c) M = fmaxf(M, __ldcg(base + ((size_t)c * G + h) * (HD + 2) + HD));
-      float num = 0.f, den = 0.f;
-      for (int c = 0; c < a.nc; ++c) {
-        const float* pc = base + ((size_t)c * G + h) * (HD + 2);
-        const float f = exp2f(__ldcg(pc + HD) - M);
-        num += f * __ldcg(pc + dd);
-        den += f * __ldcg(pc + HD + 1);
+      const float* pc = base + (size_t)h * (HD + 2) + dd;
+      const size_t cs = (size_t)G * (HD + 2);
+      float acc0 = 0.f, acc1 = 0.f;
+      int c = 0;
+      for (; c + 1 < a.nc; c += 2) {
+        acc0 = fmaf(wts[h * 32 + c], __ldcg(pc + c * cs), acc0);
+        acc1 = fmaf(wts[h * 32 + c + 1], __ldcg(pc + (c + 1) * cs), acc1);
       }
-      p.attn[(size_t)a.i * p.qdim + (size_t)(a.h * G + h) * HD + dd] = num / den;
+      if (c < a.nc) acc0 = fmaf(wts[h * 32 + c], __ldcg(pc + c * cs), acc0);
+      put_operand(p.aa_t, p.aa_f, p.ld_a, a.i, (a.h * G + h) * HD + dd, acc0 + acc1);
     }
   }
 }
@@ -948,10 +1103,13 @@ __device__ void consumer(const KParams& p, Smem& sm, const TaskDesc* ts, int nt)
   for (int ti = 0; ti < nt; ++ti) {
     const TaskDesc t = ts[ti];
     // dependency wait: one thread polls, the others wait at the consumer barrier
+    unsigned long long tr0 = 0, tr1 = 0;
     if (threadIdx.x == 0) {
+      if (p.trace) { tr0 = gtimer(); sm.wait_ns = 0; }
       bool ok = !ab;
       if (ok && t.wait_ctr != kNoCounter) ok = wait_counter(p, t.wait_ctr, t.wait_count);
       sm.flag = ok ? 0 : 1;
+      if (p.trace) tr1 = gtimer();
     }
     cbar();
     ab = ab || sm.flag;
@@ -967,10 +1125,19 @@ __device__ void consumer(const KParams& p, Smem& sm, const TaskDesc* ts, int nt)
     if (threadIdx.x == 0) {
       if (!ab) {
         __threadfence();
+        asm volatile("fence.proxy.async.global;" ::: "memory");  // later bulk copies read what we wrote
         const uint32_t old = atom_add_acqrel(p.ctr + t.sig_ctr, 1u);
         sm.flag = (t.op == OP_LMHEAD && p.argmax && old + 1u == (uint32_t)p.n_lm_tasks * p.epoch) ? 1 : 0;
       } else {
         sm.flag = 0;
+      }
+      if (p.trace) {
+        unsigned long long* r = p.trace + 4ull * (p.task_off[blockIdx.x] + ti);
+        r[0] = tr0;
+        r[1] = tr1;
+        r[2] = gtimer();
+        r[3] = (unsigned long long)t.op | ((unsigned long long)t.layer << 8) |
+               ((unsigned long long)blockIdx.x << 24) | (min(sm.wait_ns, 0xFFFFFFull) << 40);
       }
     }
     cbar();
@@ -1007,6 +1174,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNumSlots; ++s) {
       mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.ofull[s], 1);
       mbar_init(&sm.empty[s], kConsumerWarps);
     }
     fence_mbar_init();

@@ -22,8 +22,16 @@ struct KParams {
   const TaskDesc* tasks;
   const uint32_t* task_off;  // [num_sms + 1]
   int num_sms, n_slots, n_lm_tasks;
+  const void* tmaps;          // CUtensorMap array: weights (tmap_index) then the LM head
   // handle-owned device state
-  float *x, *q, *attn, *hbuf, *ssq, *part;
+  float *x, *q, *ssq, *part;
+  // GEMV operands, written once by the producing phase: bf16 hi/lo tiles in the layout of
+  // operand_index (all batch rows) and fp32 (batch row 0, for the batch-1 path).
+  // ax: x * gain of the next RMSNorm (input of qkv / gate-up / lm head), aa: attention output,
+  // ah: SwiGLU output; ld = K rounded up to 64, padding zero
+  __nv_bfloat16 *ax_t, *aa_t, *ah_t;
+  float *ax_f, *aa_f, *ah_f;
+  int ld_x, ld_a, ld_h;
   int ssq_stride;            // floats per ssq instance
   float2* lmpart;            // [n_lm_tasks][max_b] (value, index bits)
   uint32_t *ctr, *cmb, *ctl; // counters, split-K combine counters, {abort, status}
@@ -40,6 +48,7 @@ struct KParams {
   float* dbg;
   uint32_t epoch;
   unsigned long long timeout_ns;
+  unsigned long long* trace;  // optional [n_tasks][4] records (see mk_set_trace)
 };
 
 size_t kernel_smem_bytes();

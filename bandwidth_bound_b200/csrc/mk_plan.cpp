@@ -61,17 +61,6 @@ long long unit_weight_bytes(const Geometry& G, int op) {
   return (long long)rows_per_unit(op) * gemv_K(G, op) * 2;
 }
 
-uint16_t choose_kc(int rows, int K) {
-  if ((long long)rows * stage_pitch(K) <= kSlotBytes) return (uint16_t)K;
-  int best = 0;
-  for (int kc = 256; kc < K; kc += 256)
-    if ((long long)rows * stage_pitch(kc) <= kSlotBytes) best = kc;
-  if (best == 0)
-    for (int kc = 32; kc < K; kc += 32)
-      if ((long long)rows * stage_pitch(kc) <= kSlotBytes) best = kc;
-  return (uint16_t)best;
-}
-
 static bool set_err(std::string* err, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
 static bool set_err(std::string* err, const char* fmt, ...) {
   if (err) {
@@ -210,7 +199,9 @@ int build_plan(const mk_model_cfg& c, const mk_plan_opts* opts, mk_plan_s* P, st
       const int U = phase_units(G, op);
       const long long ub = unit_weight_bytes(G, op);
       const int rpu = op == OP_EMBED ? 8 : rows_per_unit(op);
-      const int max_units = op == OP_EMBED ? 255 : std::max(1, P->max_blocks * 8 / rpu);
+      const int max_u = op == OP_EMBED ? 255 : std::max(1, std::min(max_units(op), P->max_blocks * 8 / rpu));
+      // QKV tasks stay inside one head (their weight rows form one TMA box)
+      const int seg = op == OP_QKV ? G.hd / 16 : U;
       // units per SM: base, and +1 for the 'extra' SMs with the least bytes so far
       std::vector<int> cnt(nsm, U / nsm);
       int extra = U % nsm;
@@ -222,24 +213,34 @@ int build_plan(const mk_model_cfg& c, const mk_plan_opts* opts, mk_plan_s* P, st
       }
       int u = 0;
       for (int sm = 0; sm < nsm; ++sm) {
-        int n = cnt[sm];
+        const int n = cnt[sm];
         if (n == 0) continue;
-        int ntask = (n + max_units - 1) / max_units;
-        for (int k = 0; k < ntask; ++k) {
-          int nk = n / ntask + (k < n % ntask ? 1 : 0);
-          TaskDesc t{};
-          t.op = (uint8_t)op;
-          t.nunits = (uint8_t)nk;
-          t.layer = (uint16_t)l;
-          t.u0 = (uint32_t)u;
-          t.task_idx = (uint16_t)tidx++;
-          t.kc = op == OP_EMBED ? 0 : choose_kc(nk * rpu, gemv_K(G, op));
-          t.wait_ctr = (uint16_t)wc;
-          t.wait_count = wcount;
-          t.sig_ctr = (uint16_t)sig;
-          P->streams[sm].push_back(t);
-          u += nk;
+        // cut [u, u + n) at segment boundaries, then into near-equal tasks of <= max_u units
+        int a = u;
+        const int end = u + n;
+        while (a < end) {
+          const int b = std::min(end, (a / seg + 1) * seg);
+          const int len = b - a;
+          const int ntask = (len + max_u - 1) / max_u;
+          int v = a;
+          for (int k = 0; k < ntask; ++k) {
+            const int nk = len / ntask + (k < len % ntask ? 1 : 0);
+            TaskDesc t{};
+            t.op = (uint8_t)op;
+            t.nunits = (uint8_t)nk;
+            t.layer = (uint16_t)l;
+            t.u0 = (uint32_t)v;
+            t.task_idx = (uint16_t)tidx++;
+            t.kc = op == OP_EMBED ? 0 : (uint16_t)stage_cols(nk * rpu / 8, gemv_K(G, op), c.max_batch);
+            t.wait_ctr = (uint16_t)wc;
+            t.wait_count = wcount;
+            t.sig_ctr = (uint16_t)sig;
+            P->streams[sm].push_back(t);
+            v += nk;
+          }
+          a = b;
         }
+        u = end;
         cum[sm] += (long long)n * ub;
       }
     }
@@ -257,7 +258,9 @@ int build_plan(const mk_model_cfg& c, const mk_plan_opts* opts, mk_plan_s* P, st
 
 namespace {
 
-enum Buf { B_X, B_Q, B_ATTN, B_H, B_PART, B_LOGITS, B_LMPART, B_KVNEW, B_SSQ };
+// X: fp32 residual; AX: its normalised-gain operand for the next GEMV; AA: attention
+// output operand; AH: SwiGLU output operand.
+enum Buf { B_X, B_Q, B_ATTN, B_H, B_PART, B_LOGITS, B_LMPART, B_KVNEW, B_SSQ, B_AX };
 
 struct Access {
   int buf, inst;   // inst: layer for KVNEW, ssq instance for SSQ, 0 otherwise
@@ -266,16 +269,18 @@ struct Access {
 
 std::vector<Access> accesses(int op, int l, int L) {
   switch (op) {
-    case OP_EMBED: return {{B_X, 0, true}, {B_SSQ, ssq_inst_embed(), true}};
+    case OP_EMBED: return {{B_X, 0, true}, {B_AX, 0, true}, {B_SSQ, ssq_inst_embed(), true}};
     case OP_QKV:
-      return {{B_X, 0, false}, {B_SSQ, l == 0 ? ssq_inst_embed() : ssq_inst_down(l - 1), false},
+      return {{B_AX, 0, false}, {B_SSQ, l == 0 ? ssq_inst_embed() : ssq_inst_down(l - 1), false},
               {B_Q, 0, true}, {B_KVNEW, l, true}};
     case OP_ATTN: return {{B_Q, 0, false}, {B_KVNEW, l, false}, {B_PART, 0, true}, {B_ATTN, 0, true}};
-    case OP_OPROJ: return {{B_ATTN, 0, false}, {B_X, 0, true}, {B_SSQ, ssq_inst_oproj(l), true}};
-    case OP_GATEUP: return {{B_X, 0, false}, {B_SSQ, ssq_inst_oproj(l), false}, {B_H, 0, true}};
-    case OP_DOWN: return {{B_H, 0, false}, {B_X, 0, true}, {B_SSQ, ssq_inst_down(l), true}};
+    case OP_OPROJ:
+      return {{B_ATTN, 0, false}, {B_X, 0, true}, {B_AX, 0, true}, {B_SSQ, ssq_inst_oproj(l), true}};
+    case OP_GATEUP: return {{B_AX, 0, false}, {B_SSQ, ssq_inst_oproj(l), false}, {B_H, 0, true}};
+    case OP_DOWN:
+      return {{B_H, 0, false}, {B_X, 0, true}, {B_AX, 0, true}, {B_SSQ, ssq_inst_down(l), true}};
     case OP_LMHEAD:
-      return {{B_X, 0, false}, {B_SSQ, ssq_inst_down(L - 1), false}, {B_LOGITS, 0, true}, {B_LMPART, 0, true}};
+      return {{B_AX, 0, false}, {B_SSQ, ssq_inst_down(L - 1), false}, {B_LOGITS, 0, true}, {B_LMPART, 0, true}};
   }
   return {};
 }
@@ -321,16 +326,22 @@ int validate_plan(const mk_plan_s& p, std::string* err) {
       }
       for (uint32_t u = t.u0; u < t.u0 + t.nunits; ++u) cover[pi][u]++;
       if (t.op != OP_EMBED && t.op != OP_ATTN) {
-        int rows = t.nunits * rows_per_unit(t.op);
-        int K = gemv_K(G, t.op);
-        if (rows > kMaxBlocks * 8) {
+        const int rows = t.nunits * rows_per_unit(t.op);
+        const int K = gemv_K(G, t.op);
+        if (t.nunits > max_units(t.op)) {
           set_err(err, "sm %d task %zu: %d rows exceed %d", sm, k, rows, kMaxBlocks * 8);
           return MK_ERR_SCHEDULE_INVALID;
         }
-        if (t.kc < 8 || t.kc % 8 || (t.kc < K && t.kc % 32) || t.kc > K ||
-            (long long)rows * stage_pitch(t.kc) > kSlotBytes) {
+        const int tiles = (p.cfg.max_batch + 7) / 8;
+        if (t.kc < kBoxCols || t.kc % kBoxCols || t.kc > round_up(K, kBoxCols) ||
+            (long long)rows * t.kc * 2 > kWeightBytes || tiles * 2 * t.kc * 16 > kOperandBytes ||
+            ((t.kc / 32) % kConsumerWarps != 0 && t.kc < K)) {
           set_err(err, "sm %d task %zu: stage of %d rows x %d columns does not fit a %d-byte slot", sm, k,
                   rows, t.kc, kSlotBytes);
+          return MK_ERR_SCHEDULE_INVALID;
+        }
+        if (t.op == OP_QKV && (int)(t.u0 / (G.hd / 16)) != (int)((t.u0 + t.nunits - 1) / (G.hd / 16))) {
+          set_err(err, "sm %d task %zu: a QKV task crosses a head boundary", sm, k);
           return MK_ERR_SCHEDULE_INVALID;
         }
       }
@@ -545,7 +556,7 @@ MK_API int mk_plan_inject_fault(mk_plan_t plan, int32_t kind, int32_t arg) {
     case MK_FAULT_OVERSIZE_STAGE: {
       for (auto& s : plan->streams)
         for (auto& t : s)
-          if (t.op == mk::OP_LMHEAD) { t.kc = 0xFFE0; return MK_OK; }
+          if (t.op == mk::OP_LMHEAD) { t.kc = (uint16_t)(2 * mk::kWeightBytes / (t.nunits * 8)); return MK_OK; }
       return MK_ERR_INVALID_ARG;
     }
   }

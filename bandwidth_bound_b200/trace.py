@@ -1,0 +1,63 @@
+"""Summaries of the per-task timeline the megakernel records (mk_set_trace).
+
+Each record is {t_wait_start, t_wait_end, t_end, meta} in globaltimer ns, with
+meta = op | layer << 8 | sm << 24 | slot_wait_ns << 40.  The summary answers where
+a step's time goes: waiting on dependency counters (another SM's work not done),
+waiting on pool slots (HBM bytes not yet landed), or computing.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+OPS = {1: "embed", 2: "qkv", 3: "attn", 4: "oproj", 5: "gateup", 6: "down", 7: "lmhead"}
+
+
+def decode(records) -> dict:
+    r = np.asarray(records, dtype=np.uint64).reshape(-1, 4)
+    meta = r[:, 3]
+    return {
+        "t0": r[:, 0].astype(np.int64), "t1": r[:, 1].astype(np.int64), "t2": r[:, 2].astype(np.int64),
+        "op": (meta & np.uint64(0xFF)).astype(np.int64),
+        "layer": ((meta >> np.uint64(8)) & np.uint64(0xFFFF)).astype(np.int64),
+        "sm": ((meta >> np.uint64(24)) & np.uint64(0xFFFF)).astype(np.int64),
+        "slot_wait": (meta >> np.uint64(40)).astype(np.int64),
+    }
+
+
+def summarize(records, n_layers: int) -> str:
+    d = decode(records)
+    base = int(d["t0"].min())
+    end = int(d["t2"].max())
+    step_us = (end - base) / 1e3
+    nsm = int(d["sm"].max()) + 1
+    lines = [f"step {step_us:.1f} us over {nsm} SMs, {len(d['op'])} tasks"]
+    lines.append(f"{'op':8s} {'tasks':>6s} {'dep-wait us/SM':>15s} {'work us/SM':>11s} {'slot-wait us/SM':>16s}")
+    for op, name in OPS.items():
+        m = d["op"] == op
+        if not m.any():
+            continue
+        dep = (d["t1"][m] - d["t0"][m]).sum() / 1e3 / nsm
+        work = (d["t2"][m] - d["t1"][m]).sum() / 1e3 / nsm
+        sw = d["slot_wait"][m].sum() / 1e3 / nsm
+        lines.append(f"{name:8s} {int(m.sum()):6d} {dep:15.1f} {work:11.1f} {sw:16.1f}")
+    # per-layer phase windows (first work start -> last end), relative to the step start
+    lines.append("phase windows (us from step start: first start .. last end) for a few layers")
+    for l in sorted({0, 1, n_layers // 2, n_layers - 1}):
+        parts = []
+        for op in (2, 3, 4, 5, 6):
+            m = (d["op"] == op) & (d["layer"] == l)
+            if m.any():
+                parts.append(f"{OPS[op]} {(d['t1'][m].min() - base) / 1e3:.1f}..{(d['t2'][m].max() - base) / 1e3:.1f}")
+        lines.append(f"  layer {l}: " + ", ".join(parts))
+    m = d["op"] == 7
+    if m.any():
+        lines.append(f"  lmhead {(d['t1'][m].min() - base) / 1e3:.1f}..{(d['t2'][m].max() - base) / 1e3:.1f}")
+    busy = np.zeros(nsm)
+    dep = np.zeros(nsm)
+    for s in range(nsm):
+        m = d["sm"] == s
+        busy[s] = (d["t2"][m] - d["t1"][m]).sum() / 1e3
+        dep[s] = (d["t1"][m] - d["t0"][m]).sum() / 1e3
+    lines.append(f"per-SM work us: min {busy.min():.1f} median {np.median(busy):.1f} max {busy.max():.1f}; "
+                 f"dep-wait us: min {dep.min():.1f} median {np.median(dep):.1f} max {dep.max():.1f}")
+    return "\n".join(lines)

@@ -43,6 +43,11 @@ def parse():
     ap.add_argument("--impl", default="mk", choices=["mk", "reference"])
     ap.add_argument("--no-secondary", action="store_true", help="skip the batch-1 line of the same model")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--max-blocks", type=int, default=0, help="schedule option: 8-row blocks per GEMV task")
+    ap.add_argument("--attn-slots", type=int, default=0, help="schedule option: attention slots per SM")
+    ap.add_argument("--trace", default="", help="write a per-task timeline summary of one step to this file")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="profiling aid: run a model shortened to this many layers (not a bench line)")
     return ap.parse_args()
 
 
@@ -272,14 +277,21 @@ def run_mk(args, world, rank, local):
     import oracle
 
     w = synth.WORKLOADS[args.workload]
+    if args.layers:
+        w = synth.Workload(w.name + f"-first{args.layers}layers", synth.scaled_model(w.model, n_layers=args.layers),
+                           w.batch, w.ctx)
     m = w.model
-    lens = w.context_lengths()
+    lens = w.context_lengths() if not args.layers else synth.WORKLOADS[args.workload].context_lengths()
     b = w.batch
     max_ctx = max(lens) + 2
     wts = synth.make_weights(m, device="cuda")
     kv = synth.make_kv_cache(m, lens, device="cuda", max_ctx=max_ctx, batch_cap=max(b, 8))
     toks = synth.token_ids(m, b, tag=w.name)
-    h = mk.Megakernel(m, wts, max(b, 8), max_ctx)
+    plan = None
+    if args.max_blocks or args.attn_slots:
+        plan = mk.Plan(mk.model_cfg(m, max(b, 8), max_ctx), num_sms=torch.cuda.get_device_properties(local).multi_processor_count,
+                       attn_slots_per_sm=args.attn_slots, max_blocks=args.max_blocks)
+    h = mk.Megakernel(m, wts, max(b, 8), max_ctx, plan=plan)
     stream = torch.cuda.current_stream()
     tok_d = torch.tensor(toks, dtype=torch.int32, device="cuda")
     pos_d = torch.tensor(lens, dtype=torch.int32, device="cuda")
@@ -302,6 +314,23 @@ def run_mk(args, world, rank, local):
         step()
     torch.cuda.synchronize()
     assert h.status() == mk.MK_OK, f"device status {h.status()}"
+    if args.trace:
+        from bandwidth_bound_b200 import trace as mktrace
+
+        rec = torch.zeros((h.num_tasks(), 4), dtype=torch.int64, device="cuda")
+        h.set_trace(rec)
+        step()
+        torch.cuda.synchronize()
+        h.set_trace(None)
+        with open(args.trace, "w") as f:
+            f.write(mktrace.summarize(rec.cpu().numpy().view("uint64"), m.n_layers) + "\n")
+        if not args.no_secondary and b > 1:
+            h.set_trace(rec)
+            h.step(tok_d[:1], pos_d[:1], len_d[:1], kv, logits[:1], am[:1], stream=stream, check=False)
+            torch.cuda.synchronize()
+            h.set_trace(None)
+            with open(args.trace, "a") as f:
+                f.write("--- batch 1 ---\n" + mktrace.summarize(rec.cpu().numpy().view("uint64"), m.n_layers) + "\n")
     clocks = ClockSampler(local)
     clocks.start()
     barrier(world)

@@ -167,6 +167,16 @@ MK_API int mk_reset(mk_handle_t h);
  * batch rows.  NULL turns capture off. */
 MK_API int mk_set_debug(mk_handle_t h, float *layer_hidden);
 
+/* Per-task timeline for profiling: when records is a device uint64 buffer of
+ * [capacity][4] with capacity >= mk_num_tasks(h), each later step writes, for task
+ * k of the flattened per-SM streams, {globaltimer before its dependency wait,
+ * after the wait, at its end, meta} where meta = op | layer << 8 | sm << 24 |
+ * (ns warp 0 waited for pool slots, capped at 2^24-1) << 40.  NULL turns it off. */
+MK_API int mk_set_trace(mk_handle_t h, uint64_t *records, int64_t capacity);
+
+/* Number of task descriptors in the handle's per-SM streams (all SMs). */
+MK_API int64_t mk_num_tasks(mk_handle_t h);
+
 /* Device-side wait limit in nanoseconds (default 1e9).  A wait that runs out
  * sets MK_ERR_DEVICE_TIMEOUT, every CTA leaves after its copies in flight have
  * landed, and the launch completes. */
