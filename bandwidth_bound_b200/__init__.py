@@ -240,7 +240,7 @@ class Megakernel:
         return int(self.lib.mk_num_tasks(self.handle))
 
     def set_trace(self, records):
-        """records: device uint64 tensor [>= num_tasks()][4], or None."""
+        """records: device uint64 tensor [>= num_tasks()][8], or None."""
         n = 0 if records is None else records.shape[0]
         _check(self.lib.mk_set_trace(self.handle, _ptr(records), n), self.handle, "mk_set_trace")
 

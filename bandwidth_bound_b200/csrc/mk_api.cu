@@ -12,6 +12,7 @@
 #include "mk_plan.h"
 
 using mk::KParams;
+static_assert(sizeof(mk::TmaDesc) == sizeof(CUtensorMap), "TMA descriptor size");
 using mk::LayerW;
 
 struct mk_handle_s {
@@ -60,17 +61,22 @@ static void release(mk_handle_t h) {
 // TMA descriptors of every weight matrix (bf16, 128-byte swizzle, boxes of 64 columns x
 // 8n rows for n = 1..8).  wq/wk/wv are viewed as [heads*2 halves][head_dim/2][hidden]
 // so that one box holds rows 8m..8m+8n-1 of both halves of a head (the RoPE pairs).
-static std::string build_tensor_maps(const mk_model_cfg& c, const mk_weight_ptrs* w, std::vector<CUtensorMap>& maps) {
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   if (!encode) {
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess || !fn)
-      return "cuTensorMapEncodeTiled is not available";
-    encode = (PFN_cuTensorMapEncodeTiled_v12000)fn;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess && fn)
+      encode = (PFN_cuTensorMapEncodeTiled_v12000)fn;
   }
+  return encode;
+}
+
+static std::string build_tensor_maps(const mk_model_cfg& c, const mk_weight_ptrs* w, std::vector<CUtensorMap>& maps) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (!encode) return "cuTensorMapEncodeTiled is not available";
   const mk::Geometry G = mk::geometry(c);
-  maps.assign((size_t)(G.L + 1) * mk::kNumMats * mk::kMaxBlocks, CUtensorMap{});
+  maps.assign((size_t)mk::num_tmaps(G.L), CUtensorMap{});
   auto enc2d = [&](CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
     cuuint64_t dims[2] = {cols, rows};
     cuuint64_t strides[1] = {cols * 2};

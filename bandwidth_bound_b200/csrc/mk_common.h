@@ -86,7 +86,7 @@ MK_HD int round_up(int a, int b) { return (a + b - 1) / b * b; }
 MK_HD int stage_cols(int blocks, int K, int max_batch) {
   const int tiles = (max_batch + 7) / 8;
   int kc = blocks >= 5 ? 256 : 512;
-  while (kc > 256 && tiles * 2 * kc * 16 > kOperandBytes) kc -= 256;
+  while (kc > 256 && tiles * 2 * kc * 16 > kOperandBytes) kc -= 256;  // operand slices are whole 256-column boxes
   const int kp = round_up(K, kBoxCols);
   return kp <= kc ? kp : kc;
 }
@@ -103,6 +103,8 @@ MK_HD size_t operand_index(int mt, int part, int kg, int g, int e, int ld) {
 // Index of the TMA descriptor of weight matrix `mat` (0 wq .. 6 w_down) of a layer for
 // boxes of 8*n rows; the LM head's maps follow the layers' (mat 0 of layer L).
 MK_HD int tmap_index(int layer, int mat, int n) { return (layer * kNumMats + mat) * kMaxBlocks + (n - 1); }
+
+MK_HD int num_tmaps(int n_layers) { return (n_layers + 1) * kNumMats * kMaxBlocks; }
 
 // Tokens per attention stage: K rows then V rows of the same tokens, 32 KB total.
 MK_HD int attn_stage_tokens(int head_dim) { return head_dim == 64 ? 128 : 64; }

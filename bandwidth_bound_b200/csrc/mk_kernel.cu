@@ -23,9 +23,7 @@
 namespace mk {
 
 typedef __nv_bfloat16 bf16;
-struct alignas(64) CUtensorMapLike {  // the driver's opaque 128-byte TMA descriptor
-  unsigned long long v[16];
-};
+typedef TmaDesc CUtensorMapLike;
 
 // ---------------------------------------------------------------------------------------
 // shared memory
@@ -43,6 +41,8 @@ struct Smem {
   alignas(8) uint64_t empty[kNumSlots];                  // all consumer warps done with the stage
   int attn_ch, attn_n, bad, flag, flag2;
   unsigned long long wait_ns;  // time warp 0 spent waiting for pool slots in the current task (tracing)
+  unsigned long long tm[3];    // tracing: compute, reduce, epilogue ns of the current task (warp 0)
+  int inv_inst;                // ssq instance whose 1/rms sm.inv_rms holds (-1: none)
 };
 
 size_t kernel_smem_bytes() { return sizeof(Smem); }
@@ -71,6 +71,18 @@ __device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
   asm volatile(
       "{\n\t.reg .pred P;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, P;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Non-blocking test of an mbarrier phase (try_wait may suspend the caller for a while).
+__device__ __forceinline__ bool mbar_test(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
       "selp.b32 %0, 1, 0, P;\n\t}"
       : "=r"(ok)
       : "r"(smem_u32(b)), "r"(parity)
@@ -134,6 +146,9 @@ __device__ __forceinline__ uint32_t atom_add_acqrel(uint32_t* p, uint32_t v) {
   asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(o) : "l"(p), "r"(v) : "memory");
   return o;
 }
+__device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
 __device__ __forceinline__ void cbar() {  // the consumer warps only
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
 }
@@ -186,7 +201,7 @@ __device__ __forceinline__ bool mbar_wait_warp(const KParams& p, uint64_t* bar, 
                                                unsigned long long* wait_acc = nullptr) {
   int ok = 0;
   if ((threadIdx.x & 31) == 0) {
-    if (wait_acc && !mbar_try(bar, parity)) {
+    if (wait_acc && !mbar_test(bar, parity)) {
       const uint64_t t0 = gtimer();
       ok = mbar_wait(p, bar, parity) ? 1 : 0;
       *wait_acc += gtimer() - t0;
@@ -305,19 +320,9 @@ __device__ void attn_setup(const KParams& p, int* ch_out, int* n_out) {
 // ---------------------------------------------------------------------------------------
 // producer warp: streams weight rows and prior KV pages into the slot ring
 
-struct Operand {
-  const bf16* tiles;
-  const float* f;
-  int ld;
-};
-
-__device__ __forceinline__ Operand operand_of(const KParams& p, int op) {
-  switch (op) {
-    case OP_OPROJ: return {p.aa_t, p.aa_f, p.ld_a};
-    case OP_DOWN: return {p.ah_t, p.ah_f, p.ld_h};
-    default: return {p.ax_t, p.ax_f, p.ld_x};
-  }
-}
+// Operand kind of a GEMV op: 0 x-derived (qkv, gate/up, lm head), 1 attention output (o
+// projection), 2 SwiGLU output (down projection).
+__device__ __forceinline__ int operand_kind(int op) { return op == OP_OPROJ ? 1 : (op == OP_DOWN ? 2 : 0); }
 
 __device__ __forceinline__ int attn_stages(const AttnWork& a, int T) { return (a.c1 - a.c0 + T - 1) / T; }
 
@@ -384,10 +389,11 @@ __device__ bool issue_weights(const KParams& p, Smem& sm, const TaskDesc& t, con
 }
 
 // Operand slice of GEMV stage s of task t into the operand part of slot `slot`: one bulk
-// copy per batch tile and bf16 part (batch >= 2), or the fp32 row (batch 1).
+// copy per batch tile and bf16 part (batch >= 2), or of the fp32 row (batch 1).  (Measured on
+// B200: these L2-resident slices come faster as 1-D bulk copies than as tiled boxes.)
 __device__ void issue_operand(const KParams& p, Smem& sm, const TaskDesc& t, int s, int slot) {
   const int lane = threadIdx.x & 31;
-  const Operand op = operand_of(p, t.op);
+  const int kind = operand_kind(t.op);
   const int K = gemv_K_dev(p, t.op);
   const int kc0 = s * t.kc;
   const int cols = ((min((int)t.kc, K - kc0) + kBoxCols - 1) / kBoxCols) * kBoxCols;
@@ -395,16 +401,18 @@ __device__ void issue_operand(const KParams& p, Smem& sm, const TaskDesc& t, int
   // one lane issues: it is the lane whose acquire of the dependency counter ordered the reads
   if (lane == 0) {
     const uint64_t pol = policy_evict_last();
+    const bf16* tiles = kind == 0 ? p.ax_t : (kind == 1 ? p.aa_t : p.ah_t);
+    const float* f = kind == 0 ? p.ax_f : (kind == 1 ? p.aa_f : p.ah_f);
+    const int ld = kind == 0 ? p.ld_x : (kind == 1 ? p.ld_a : p.ld_h);
     if (p.b == 1) {
       mbar_expect_tx(&sm.ofull[slot], (uint32_t)cols * 4u);
-      bulk_g2s(dst, op.f + kc0, (uint32_t)cols * 4u, &sm.ofull[slot], pol);
+      bulk_g2s(dst, f + kc0, (uint32_t)cols * 4u, &sm.ofull[slot], pol);
     } else {
-      const int nt = (p.b + 7) >> 3;
-      mbar_expect_tx(&sm.ofull[slot], (uint32_t)(nt * 2 * cols * 16));
-      for (int q = 0; q < 2 * nt; ++q) {
-        const bf16* src = op.tiles + operand_index(q >> 1, q & 1, kc0 / 8, 0, 0, op.ld);
-        bulk_g2s(dst + (size_t)q * t.kc * 16, src, (uint32_t)cols * 16u, &sm.ofull[slot], pol);
-      }
+      const int nq = 2 * ((p.b + 7) >> 3);
+      mbar_expect_tx(&sm.ofull[slot], (uint32_t)(nq * cols * 16));
+      for (int q = 0; q < nq; ++q)
+        bulk_g2s(dst + (size_t)q * round_up(t.kc, 256) * 16, tiles + operand_index(q >> 1, q & 1, kc0 / 8, 0, 0, ld),
+                 (uint32_t)cols * 16u, &sm.ofull[slot], pol);
     }
   }
   __syncwarp();
@@ -433,7 +441,7 @@ __device__ void producer(const KParams& p, Smem& sm, const TaskDesc* ts, int nt)
       } else {
         const int slot = wk % kNumSlots;
         int ready = 0;
-        if (lane == 0) ready = mbar_try(&sm.empty[slot], ((wk / kNumSlots) & 1) ^ 1) ? 1 : 0;
+        if (lane == 0) ready = mbar_test(&sm.empty[slot], ((wk / kNumSlots) & 1) ^ 1) ? 1 : 0;
         if (__shfl_sync(0xffffffffu, ready, 0)) {
           if (!issue_weights(p, sm, t, wa, ws, slot, pol)) {
             if (lane == 0) raise_error(p, -6 /* MK_ERR_BOUNDS */);
@@ -556,7 +564,7 @@ __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDes
     for (int mt = 0; mt < NMT; ++mt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[j][mt][e] = 0.f;
-  const int opart = kc * 16;  // bytes of one (tile, part) slice in the operand area
+  const int opart = round_up(kc, 256) * 16;  // bytes of one (tile, part) slice in the operand area
 
   for (int s = 0; s < nst; ++s, ++stage) {
     const int slot = stage % kNumSlots;
@@ -564,6 +572,7 @@ __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDes
     if (!ab) ab = !mbar_wait_warp(p, &sm.full[slot], par, (p.trace && threadIdx.x == 0) ? &sm.wait_ns : nullptr);
     if (!ab) ab = !mbar_wait_warp(p, &sm.ofull[slot], par, (p.trace && threadIdx.x == 0) ? &sm.wait_ns : nullptr);
     if (ab) continue;
+    const unsigned long long tc0 = (p.trace && threadIdx.x == 0) ? gtimer() : 0ull;
     const uint8_t* tile = sm.pool[slot];
     const uint8_t* opnd = sm.pool[slot] + kWeightBytes;
     const int nb = 2 * ((min(kc, K - s * kc) + kBoxCols - 1) / kBoxCols);
@@ -602,9 +611,11 @@ __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDes
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.empty[slot]);
+    if (p.trace && threadIdx.x == 0) sm.tm[0] += gtimer() - tc0;
   }
 
   // cross-warp reduction, one 8-row batch tile at a time: red[warp][block][batch g][8 rows]
+  const unsigned long long tr0 = (p.trace && threadIdx.x == 0) ? gtimer() : 0ull;
   float* red = sm.red;
 #pragma unroll
   for (int mt = 0; mt < NMT; ++mt) {
@@ -636,6 +647,7 @@ __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDes
     }
     cbar();
   }
+  if (p.trace && threadIdx.x == 0) sm.tm[1] += gtimer() - tr0;
 }
 
 template <int MT>
@@ -667,17 +679,19 @@ __device__ __forceinline__ const bf16* next_gain(const KParams& p, int op, int l
 __device__ void gemv_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_t& stage, bool& ab) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool norm = t.op == OP_QKV || t.op == OP_GATEUP || t.op == OP_LMHEAD;
-  if (norm && !ab) {
-    const int inst = t.op == OP_GATEUP ? ssq_inst_oproj(t.layer)
-                     : t.op == OP_QKV  ? (t.layer == 0 ? ssq_inst_embed() : ssq_inst_down(t.layer - 1))
-                                       : ssq_inst_down(p.L - 1);
-    compute_inv_rms(p, sm, inst, (int)t.wait_count);
-  }
+  const int inst = t.op == OP_GATEUP ? ssq_inst_oproj(t.layer)
+                   : t.op == OP_QKV  ? (t.layer == 0 ? ssq_inst_embed() : ssq_inst_down(t.layer - 1))
+                                     : ssq_inst_down(p.L - 1);
+  // tasks of one phase share the 1/rms of their input: compute it once per phase
+  const bool fresh = norm && !ab && sm.inv_inst != inst;
+  if (fresh) compute_inv_rms(p, sm, inst, (int)t.wait_count);
   cbar();
+  if (fresh && threadIdx.x == 0) sm.inv_inst = inst;
   const int G = t.nunits * rows_per_unit(t.op) / 8;
   if (p.b == 1) gemv_dispatch<0>(p, sm, t, stage, ab, G);
   else if (p.b <= 8) gemv_dispatch<1>(p, sm, t, stage, ab, G);
   else gemv_dispatch<2>(p, sm, t, stage, ab, G);
+  const unsigned long long te0 = (p.trace && threadIdx.x == 0) ? gtimer() : 0ull;
 
   const int nthr = kConsumerWarps * 32;
   const int n = t.nunits;
@@ -790,6 +804,7 @@ __device__ void gemv_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_
       }
     }
   }
+  if (p.trace && threadIdx.x == 0) sm.tm[2] += gtimer() - te0;
 }
 
 __device__ void embed_task(const KParams& p, Smem& sm, const TaskDesc& t, bool ab) {
@@ -877,6 +892,7 @@ __device__ __noinline__ void attn_task(const KParams& p, Smem& sm, const TaskDes
     for (int e = 0; e < DPL; ++e) acc[h][e] = 0.f;
 
   const int nst = attn_stages(a, T);
+  const unsigned long long tc0 = (p.trace && threadIdx.x == 0) ? gtimer() : 0ull;
   for (int s = 0; s < nst; ++s, ++stage) {
     const int slot = stage % kNumSlots;
     const int t0 = a.c0 + s * T, t1 = min(t0 + T, a.c1);
@@ -1004,6 +1020,11 @@ __device__ __noinline__ void attn_task(const KParams& p, Smem& sm, const TaskDes
     if (!ab && lane == 0) mbar_arrive(&sm.empty[slot]);
   }
 
+  unsigned long long tr0 = 0;
+  if (p.trace && threadIdx.x == 0) {
+    tr0 = gtimer();
+    sm.tm[0] += tr0 - tc0 - sm.wait_ns;
+  }
   // merge the eight warps' (m, l, acc) states: red[warp][head][HD]
   if (!ab) {
 #pragma unroll
@@ -1045,10 +1066,11 @@ __device__ __noinline__ void attn_task(const KParams& p, Smem& sm, const TaskDes
     }
   }
   cbar();
+  const unsigned long long te0 = (p.trace && threadIdx.x == 0) ? gtimer() : 0ull;
+  if (p.trace && threadIdx.x == 0) sm.tm[1] += te0 - tr0;
   if (threadIdx.x == 0) {
     int last = 0;
     if (!ab) {
-      __threadfence();
       uint32_t* cc = p.cmb + ((size_t)t.layer * p.max_b + a.i) * p.nkv + a.h;
       const uint32_t old = atom_add_acqrel(cc, 1u);
       last = (old + 1u == (uint32_t)a.nc) ? 1 : 0;
@@ -1092,6 +1114,7 @@ __device__ __noinline__ void attn_task(const KParams& p, Smem& sm, const TaskDes
       put_operand(p.aa_t, p.aa_f, p.ld_a, a.i, (a.h * G + h) * HD + dd, acc0 + acc1);
     }
   }
+  if (p.trace && threadIdx.x == 0) sm.tm[2] += gtimer() - te0;
 }
 
 // ---------------------------------------------------------------------------------------
@@ -1100,14 +1123,23 @@ __device__ __noinline__ void attn_task(const KParams& p, Smem& sm, const TaskDes
 __device__ void consumer(const KParams& p, Smem& sm, const TaskDesc* ts, int nt) {
   uint32_t stage = 0;
   bool ab = false;
+  int met_ctr = -1;          // thread 0: the last counter/target seen satisfied (counters only grow)
+  uint32_t met_target = 0;
   for (int ti = 0; ti < nt; ++ti) {
     const TaskDesc t = ts[ti];
     // dependency wait: one thread polls, the others wait at the consumer barrier
     unsigned long long tr0 = 0, tr1 = 0;
     if (threadIdx.x == 0) {
-      if (p.trace) { tr0 = gtimer(); sm.wait_ns = 0; }
+      if (p.trace) { tr0 = gtimer(); sm.wait_ns = 0; sm.tm[0] = sm.tm[1] = sm.tm[2] = 0; }
       bool ok = !ab;
-      if (ok && t.wait_ctr != kNoCounter) ok = wait_counter(p, t.wait_ctr, t.wait_count);
+      if (ok && t.wait_ctr != kNoCounter) {
+        const uint32_t target = t.wait_count * p.epoch;
+        if (t.wait_ctr != met_ctr || target != met_target) {
+          ok = wait_counter(p, t.wait_ctr, t.wait_count);
+          met_ctr = t.wait_ctr;
+          met_target = target;
+        }
+      }
       sm.flag = ok ? 0 : 1;
       if (p.trace) tr1 = gtimer();
     }
@@ -1123,21 +1155,33 @@ __device__ void consumer(const KParams& p, Smem& sm, const TaskDesc* ts, int nt)
     }
     cbar();
     if (threadIdx.x == 0) {
+      const unsigned long long ts0 = p.trace ? gtimer() : 0ull;
       if (!ab) {
-        __threadfence();
-        asm volatile("fence.proxy.async.global;" ::: "memory");  // later bulk copies read what we wrote
-        const uint32_t old = atom_add_acqrel(p.ctr + t.sig_ctr, 1u);
-        sm.flag = (t.op == OP_LMHEAD && p.argmax && old + 1u == (uint32_t)p.n_lm_tasks * p.epoch) ? 1 : 0;
+        // release: everything the consumer warps wrote before the barrier above is visible to
+        // whoever acquires the counter; bulk copies (async proxy) may read it next
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        if (t.op == OP_LMHEAD && p.argmax) {
+          const uint32_t old = atom_add_acqrel(p.ctr + t.sig_ctr, 1u);
+          sm.flag = old + 1u == (uint32_t)p.n_lm_tasks * p.epoch ? 1 : 0;
+        } else {
+          red_release_add(p.ctr + t.sig_ctr, 1u);  // nobody here needs the old value: no round trip
+          sm.flag = 0;
+        }
       } else {
         sm.flag = 0;
       }
       if (p.trace) {
-        unsigned long long* r = p.trace + 4ull * (p.task_off[blockIdx.x] + ti);
+        unsigned long long* r = p.trace + 8ull * (p.task_off[blockIdx.x] + ti);
+        const unsigned long long te = gtimer();
         r[0] = tr0;
         r[1] = tr1;
-        r[2] = gtimer();
+        r[2] = te;
         r[3] = (unsigned long long)t.op | ((unsigned long long)t.layer << 8) |
                ((unsigned long long)blockIdx.x << 24) | (min(sm.wait_ns, 0xFFFFFFull) << 40);
+        r[4] = sm.tm[0];
+        r[5] = sm.tm[1];
+        r[6] = sm.tm[2];
+        r[7] = te - ts0;
       }
     }
     cbar();
@@ -1190,6 +1234,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
     }
     if (bad) raise_error(p, -6 /* MK_ERR_BOUNDS */);
     sm.bad = bad;
+    sm.inv_inst = -1;
     if (!bad) attn_setup(p, &sm.attn_ch, &sm.attn_n);
   }
   __syncthreads();

@@ -12,6 +12,10 @@ struct LayerW {
   const __nv_bfloat16 *attn_norm, *wq, *wk, *wv, *wo, *mlp_norm, *wg, *wu, *wd;
 };
 
+struct alignas(64) TmaDesc {  // the driver's opaque 128-byte TMA descriptor (CUtensorMap)
+  unsigned long long v[16];
+};
+
 struct KParams {
   // model shape
   int L, d, nq, nkv, hd, F, V, g, qdim, max_b, max_ctx;

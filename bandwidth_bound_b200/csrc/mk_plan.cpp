@@ -334,7 +334,7 @@ int validate_plan(const mk_plan_s& p, std::string* err) {
         }
         const int tiles = (p.cfg.max_batch + 7) / 8;
         if (t.kc < kBoxCols || t.kc % kBoxCols || t.kc > round_up(K, kBoxCols) ||
-            (long long)rows * t.kc * 2 > kWeightBytes || tiles * 2 * t.kc * 16 > kOperandBytes ||
+            (long long)rows * t.kc * 2 > kWeightBytes || tiles * 2 * round_up(t.kc, 256) * 16 > kOperandBytes ||
             ((t.kc / 32) % kConsumerWarps != 0 && t.kc < K)) {
           set_err(err, "sm %d task %zu: stage of %d rows x %d columns does not fit a %d-byte slot", sm, k,
                   rows, t.kc, kSlotBytes);

@@ -1,7 +1,7 @@
 """Summaries of the per-task timeline the megakernel records (mk_set_trace).
 
-Each record is {t_wait_start, t_wait_end, t_end, meta} in globaltimer ns, with
-meta = op | layer << 8 | sm << 24 | slot_wait_ns << 40.  The summary answers where
+Each record is {t_wait_start, t_wait_end, t_end, meta, compute, reduce, epilogue,
+signal} in globaltimer ns, with meta = op | layer << 8 | sm << 24 | slot_wait_ns << 40.  The summary answers where
 a step's time goes: waiting on dependency counters (another SM's work not done),
 waiting on pool slots (HBM bytes not yet landed), or computing.
 """
@@ -13,9 +13,11 @@ OPS = {1: "embed", 2: "qkv", 3: "attn", 4: "oproj", 5: "gateup", 6: "down", 7: "
 
 
 def decode(records) -> dict:
-    r = np.asarray(records, dtype=np.uint64).reshape(-1, 4)
+    r = np.asarray(records, dtype=np.uint64).reshape(-1, 8)
     meta = r[:, 3]
     return {
+        "compute": r[:, 4].astype(np.int64), "reduce": r[:, 5].astype(np.int64),
+        "epilogue": r[:, 6].astype(np.int64), "signal": r[:, 7].astype(np.int64),
         "t0": r[:, 0].astype(np.int64), "t1": r[:, 1].astype(np.int64), "t2": r[:, 2].astype(np.int64),
         "op": (meta & np.uint64(0xFF)).astype(np.int64),
         "layer": ((meta >> np.uint64(8)) & np.uint64(0xFFFF)).astype(np.int64),
@@ -31,7 +33,8 @@ def summarize(records, n_layers: int) -> str:
     step_us = (end - base) / 1e3
     nsm = int(d["sm"].max()) + 1
     lines = [f"step {step_us:.1f} us over {nsm} SMs, {len(d['op'])} tasks"]
-    lines.append(f"{'op':8s} {'tasks':>6s} {'dep-wait us/SM':>15s} {'work us/SM':>11s} {'slot-wait us/SM':>16s}")
+    lines.append(f"{'op':8s} {'tasks':>6s} {'dep-wait':>9s} {'work':>8s} {'slot-wait':>10s} {'compute':>8s} "
+                 f"{'reduce':>7s} {'epilog':>7s} {'signal':>7s}   (us per SM over the step)")
     for op, name in OPS.items():
         m = d["op"] == op
         if not m.any():
@@ -39,7 +42,9 @@ def summarize(records, n_layers: int) -> str:
         dep = (d["t1"][m] - d["t0"][m]).sum() / 1e3 / nsm
         work = (d["t2"][m] - d["t1"][m]).sum() / 1e3 / nsm
         sw = d["slot_wait"][m].sum() / 1e3 / nsm
-        lines.append(f"{name:8s} {int(m.sum()):6d} {dep:15.1f} {work:11.1f} {sw:16.1f}")
+        part = [d[k][m].sum() / 1e3 / nsm for k in ("compute", "reduce", "epilogue", "signal")]
+        lines.append(f"{name:8s} {int(m.sum()):6d} {dep:9.1f} {work:8.1f} {sw:10.1f} {part[0]:8.1f} {part[1]:7.1f} "
+                     f"{part[2]:7.1f} {part[3]:7.1f}")
     # per-layer phase windows (first work start -> last end), relative to the step start
     lines.append("phase windows (us from step start: first start .. last end) for a few layers")
     for l in sorted({0, 1, n_layers // 2, n_layers - 1}):

@@ -317,13 +317,17 @@ def run_mk(args, world, rank, local):
     if args.trace:
         from bandwidth_bound_b200 import trace as mktrace
 
-        rec = torch.zeros((h.num_tasks(), 4), dtype=torch.int64, device="cuda")
+        rec = torch.zeros((h.num_tasks(), 8), dtype=torch.int64, device="cuda")
         h.set_trace(rec)
         step()
         torch.cuda.synchronize()
         h.set_trace(None)
+        raw = rec.cpu().numpy().view("uint64")
         with open(args.trace, "w") as f:
-            f.write(mktrace.summarize(rec.cpu().numpy().view("uint64"), m.n_layers) + "\n")
+            f.write(mktrace.summarize(raw, m.n_layers) + "\n")
+        import numpy as np
+
+        np.save(os.path.splitext(args.trace)[0] + ".npy", raw)
         if not args.no_secondary and b > 1:
             h.set_trace(rec)
             h.step(tok_d[:1], pos_d[:1], len_d[:1], kv, logits[:1], am[:1], stream=stream, check=False)
