@@ -23,10 +23,9 @@ namespace mk {
 // ---- launch geometry -------------------------------------------------------------------
 constexpr int kConsumerWarps = 8;                       // compute warps per CTA
 constexpr int kThreads = (kConsumerWarps + 1) * 32;     // + one producer (TMA) warp
-constexpr int kWeightBytes = 32 * 1024;                 // weight (or KV) part of a pool stage
-constexpr int kOperandBytes = 16 * 1024;                // GEMV operand part of a pool stage
-constexpr int kSlotBytes = kWeightBytes + kOperandBytes; // one pool stage (1024-byte aligned)
-constexpr int kNumSlots = 4;                            // pool depth (192 KB)
+constexpr int kSlotBytes = 32 * 1024;                   // one pool stage: weights or KV pages (1024-byte aligned)
+constexpr int kNumSlots = 5;                            // pool depth (160 KB)
+constexpr int kRingBytes = 4 * 1024;                    // per consumer warp: GEMV operands of its next k blocks
 constexpr int kMaxBatch = 16;
 constexpr int kMaxBlocks = 8;                           // 8-row blocks per GEMV task (64 rows)
 constexpr int kPage = 16;                               // tokens per KV page
@@ -80,22 +79,19 @@ MK_HD int max_units(int op) { return (op == OP_QKV || op == OP_GATEUP) ? kMaxBlo
 MK_HD uint32_t ceil_div(uint32_t a, uint32_t b) { return (a + b - 1) / b; }
 MK_HD int round_up(int a, int b) { return (a + b - 1) / b * b; }
 
-// K columns per pool stage of a GEMV task with `blocks` 8-row blocks: the weights fit
-// kWeightBytes, the operand slice (2 bf16 parts x 8-row batch tiles x 16 bytes per 8
-// columns) fits kOperandBytes, and every consumer warp gets whole 32-column blocks.
+// K columns per pool stage of a GEMV task with `blocks` 8-row blocks: the weights fit a
+// slot and every consumer warp gets whole 32-column blocks (1, 2 or 4 of them).
 MK_HD int stage_cols(int blocks, int K, int max_batch) {
-  const int tiles = (max_batch + 7) / 8;
-  int kc = blocks >= 5 ? 256 : 512;
-  while (kc > 256 && tiles * 2 * kc * 16 > kOperandBytes) kc -= 256;  // operand slices are whole 256-column boxes
+  (void)max_batch;
+  const int kc = blocks >= 5 ? 256 : (blocks >= 3 ? 512 : 1024);
   const int kp = round_up(K, kBoxCols);
   return kp <= kc ? kp : kc;
 }
 
-// Operand tile layout in global memory (written by the producing epilogues, copied
-// into a pool stage with one bulk copy per tile and part): for batch tile mt (rows
-// 8mt..8mt+7) and part (0 hi, 1 lo), groups of 8 columns; group kg holds 8 rows of 16
-// bytes, row g stored in slot g ^ (2 * ((kg >> 1) & 3)) so that a quarter warp's
-// reads (two rows, four column groups) hit eight distinct bank groups.
+// Operand tile layout in global memory (written by the producing epilogues, read by the
+// consuming GEMV's lanes): for batch tile mt (rows 8mt..8mt+7) and part (0 hi, 1 lo),
+// groups of 8 columns; group kg holds 8 rows of 16 bytes (row g in slot g ^ (2 * ((kg >> 1)
+// & 3)), a permutation that keeps every 128-byte group whole for the reading warp).
 MK_HD size_t operand_index(int mt, int part, int kg, int g, int e, int ld) {
   return ((((size_t)(mt * 2 + part) * (ld / 8) + kg) * 8 + (g ^ (2 * ((kg >> 1) & 3)))) * 8 + e);
 }

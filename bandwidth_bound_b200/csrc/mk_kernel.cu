@@ -29,15 +29,15 @@ typedef TmaDesc CUtensorMapLike;
 // shared memory
 
 struct Smem {
-  alignas(1024) uint8_t pool[kNumSlots][kSlotBytes];  // per slot: weights/KV, then GEMV operands
+  alignas(1024) uint8_t pool[kNumSlots][kSlotBytes];  // per slot: weight boxes or KV pages of one stage
   alignas(16) float red[kRedBytes / 4];                 // GEMV cross-warp partials / attention merge
+  alignas(128) uint8_t ring[kConsumerWarps][kRingBytes];  // per warp: operands of its upcoming k blocks
   alignas(16) float ep[kMaxBlocks * 8][kMaxBatch];       // per-task results [row][batch]
   alignas(16) float pw[kConsumerWarps][16 * 8];          // attention probabilities [token][head]
   float mw[kConsumerWarps][8], lw[kConsumerWarps][8];    // attention merge state per warp
   float corr[kConsumerWarps][8];
   float inv_rms[kMaxBatch];
   alignas(8) uint64_t full[kNumSlots];                   // weight/KV bytes of the stage landed
-  alignas(8) uint64_t ofull[kNumSlots];                  // operand bytes of the stage landed
   alignas(8) uint64_t empty[kNumSlots];                  // all consumer warps done with the stage
   int attn_ch, attn_n, bad, flag, flag2;
   unsigned long long wait_ns;  // time warp 0 spent waiting for pool slots in the current task (tracing)
@@ -388,109 +388,26 @@ __device__ bool issue_weights(const KParams& p, Smem& sm, const TaskDesc& t, con
   return true;
 }
 
-// Operand slice of GEMV stage s of task t into the operand part of slot `slot`: one bulk
-// copy per batch tile and bf16 part (batch >= 2), or of the fp32 row (batch 1).  (Measured on
-// B200: these L2-resident slices come faster as 1-D bulk copies than as tiled boxes.)
-__device__ void issue_operand(const KParams& p, Smem& sm, const TaskDesc& t, int s, int slot) {
-  const int lane = threadIdx.x & 31;
-  const int kind = operand_kind(t.op);
-  const int K = gemv_K_dev(p, t.op);
-  const int kc0 = s * t.kc;
-  const int cols = ((min((int)t.kc, K - kc0) + kBoxCols - 1) / kBoxCols) * kBoxCols;
-  uint8_t* dst = sm.pool[slot] + kWeightBytes;
-  // one lane issues: it is the lane whose acquire of the dependency counter ordered the reads
-  if (lane == 0) {
-    const uint64_t pol = policy_evict_last();
-    const bf16* tiles = kind == 0 ? p.ax_t : (kind == 1 ? p.aa_t : p.ah_t);
-    const float* f = kind == 0 ? p.ax_f : (kind == 1 ? p.aa_f : p.ah_f);
-    const int ld = kind == 0 ? p.ld_x : (kind == 1 ? p.ld_a : p.ld_h);
-    if (p.b == 1) {
-      mbar_expect_tx(&sm.ofull[slot], (uint32_t)cols * 4u);
-      bulk_g2s(dst, f + kc0, (uint32_t)cols * 4u, &sm.ofull[slot], pol);
-    } else {
-      const int nq = 2 * ((p.b + 7) >> 3);
-      mbar_expect_tx(&sm.ofull[slot], (uint32_t)(nq * cols * 16));
-      for (int q = 0; q < nq; ++q)
-        bulk_g2s(dst + (size_t)q * round_up(t.kc, 256) * 16, tiles + operand_index(q >> 1, q & 1, kc0 / 8, 0, 0, ld),
-                 (uint32_t)cols * 16u, &sm.ofull[slot], pol);
-    }
-  }
-  __syncwarp();
-}
-
-// The producer warp: one event loop with two cursors over the CTA's stream of stages.
-// The weight cursor streams weights and prior KV pages as far ahead as free slots
-// allow - weights do not depend on this step's activations.  The operand cursor
-// follows it and fills a GEMV stage's operand part as soon as the task's dependency
-// counter is met (other stages get a bare arrival so every slot's phases stay aligned).
+// The producer warp streams the weights and prior KV pages of the CTA's whole stream of
+// stages into the slot ring, as far ahead as free slots allow: none of it depends on this
+// step's activations, so it runs ahead across dependency waits and phase boundaries.
 __device__ void producer(const KParams& p, Smem& sm, const TaskDesc* ts, int nt) {
   const int lane = threadIdx.x & 31;
   const uint64_t pol = policy_evict_first();
-  uint32_t wk = 0, ok = 0;  // stages issued by the weight / operand cursor
-  int wt = 0, ws = 0, wn = -1, ot = 0, os = 0, on = -1;
-  bool odep = false, fail = false;
-  AttnWork wa, oa;
-  uint64_t idle_since = 0;
-  while (!fail && (wt < nt || ot < nt)) {
-    bool prog = false;
-    if (wt < nt) {
-      const TaskDesc t = ts[wt];
-      if (wn < 0) wn = task_stages(p, sm, t, wa);
-      if (ws >= wn) {
-        ++wt; ws = 0; wn = -1; prog = true;
-      } else {
-        const int slot = wk % kNumSlots;
-        int ready = 0;
-        if (lane == 0) ready = mbar_test(&sm.empty[slot], ((wk / kNumSlots) & 1) ^ 1) ? 1 : 0;
-        if (__shfl_sync(0xffffffffu, ready, 0)) {
-          if (!issue_weights(p, sm, t, wa, ws, slot, pol)) {
-            if (lane == 0) raise_error(p, -6 /* MK_ERR_BOUNDS */);
-            fail = true;
-            break;
-          }
-          ++wk; ++ws; prog = true;
-        }
+  uint32_t wk = 0;  // stages issued
+  bool fail = false;
+  for (int wt = 0; wt < nt && !fail; ++wt) {
+    const TaskDesc t = ts[wt];
+    AttnWork wa;
+    const int wn = task_stages(p, sm, t, wa);
+    for (int ws = 0; ws < wn; ++ws, ++wk) {
+      const int slot = wk % kNumSlots;
+      if (!mbar_wait_warp(p, &sm.empty[slot], ((wk / kNumSlots) & 1) ^ 1)) { fail = true; break; }
+      if (!issue_weights(p, sm, t, wa, ws, slot, pol)) {
+        if (lane == 0) raise_error(p, -6 /* MK_ERR_BOUNDS */);
+        fail = true;
+        break;
       }
-    }
-    if (ot < nt) {
-      const TaskDesc t = ts[ot];
-      if (on < 0) { on = task_stages(p, sm, t, oa); odep = false; }
-      if (os >= on) {
-        ++ot; os = 0; on = -1; prog = true;
-      } else if (ok < wk) {  // a stage's operand part follows its weights into the slot
-        const int slot = ok % kNumSlots;
-        if (t.op == OP_ATTN) {
-          if (lane == 0) mbar_arrive(&sm.ofull[slot]);
-          __syncwarp();
-          ++ok; ++os; prog = true;
-        } else {
-          if (!odep) {
-            int met = 1;
-            if (lane == 0 && t.wait_ctr != kNoCounter)
-              met = (int32_t)(ld_acquire(p.ctr + t.wait_ctr) - t.wait_count * p.epoch) >= 0 ? 1 : 0;
-            odep = __shfl_sync(0xffffffffu, met, 0) != 0;
-            if (odep) asm volatile("fence.proxy.async.global;" ::: "memory");
-          }
-          if (odep) {
-            issue_operand(p, sm, t, os, slot);
-            ++ok; ++os; prog = true;
-          }
-        }
-      }
-    }
-    if (prog) {
-      idle_since = 0;
-    } else {
-      __nanosleep(32);
-      if (lane == 0) {
-        const uint64_t now = gtimer();
-        if (idle_since == 0) idle_since = now;
-        int stop = 0;
-        if (aborted(p)) stop = 1;
-        else if (now - idle_since > p.timeout_ns) { raise_error(p, -5 /* MK_ERR_DEVICE_TIMEOUT */); stop = 1; }
-        fail = stop;
-      }
-      fail = __shfl_sync(0xffffffffu, fail ? 1 : 0, 0) != 0;
     }
   }
   if (fail) {
@@ -500,12 +417,6 @@ __device__ void producer(const KParams& p, Smem& sm, const TaskDesc* ts, int nt)
       for (uint32_t s = first; s < wk; ++s) {
         const uint64_t t0 = gtimer();
         while (!mbar_try(&sm.full[s % kNumSlots], (s / kNumSlots) & 1))
-          if (gtimer() - t0 > p.timeout_ns) break;
-      }
-      const uint32_t ofirst = ok > (uint32_t)kNumSlots ? ok - kNumSlots : 0u;
-      for (uint32_t s = ofirst; s < ok; ++s) {
-        const uint64_t t0 = gtimer();
-        while (!mbar_try(&sm.ofull[s % kNumSlots], (s / kNumSlots) & 1))
           if (gtimer() - t0 > p.timeout_ns) break;
       }
     }
@@ -539,22 +450,60 @@ __device__ __forceinline__ void put_operand(bf16* tiles, float* f, int ld, int b
   if (bi == 0) f[k] = v;
 }
 
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Copy this lane's operand of column group kg (8 columns) into ring entry e of its warp:
+// MT tiles of (hi, lo) 16-byte rows (batch row 8mt + g; zeros past the batch), or the 8 fp32
+// values of batch row 0 (MT == 0).  Lane-private 16-byte pieces: entry e, piece q at
+// ((e * 2 * NMT + q) * 32 + lane) * 16.
+template <int MT>
+__device__ __forceinline__ void fetch_opnd(const KParams& p, uint8_t* ring, int e, const bf16* tiles, const float* f,
+                                           int ld, int kg, int g, int lane) {
+  constexpr int NQ = MT == 0 ? 2 : 2 * MT;
+  uint8_t* base = ring + (size_t)e * NQ * 512 + lane * 16;
+  if constexpr (MT == 0) {
+    cp_async16(base, f + 8 * kg, true);
+    cp_async16(base + 512, f + 8 * kg + 4, true);
+  } else {
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      const bool v = mt * 8 + g < p.b;
+      cp_async16(base + (2 * mt) * 512, tiles + operand_index(mt, 0, kg, g, 0, ld), v);
+      cp_async16(base + (2 * mt + 1) * 512, tiles + operand_index(mt, 1, kg, g, 0, ld), v);
+    }
+  }
+}
+
 // Stream the task's stages through the eight warps and reduce into sm.ep[row][batch].
 // Weight stage layout (per 64-column chunk): 8*G rows of 128 bytes, 16-byte chunks
 // swizzled (chunk c of row r at c ^ (r & 7)).  Warp w takes 32-column k blocks w, w+8,
-// ...; a k block is the even (h = 0) or odd (h = 1) 16-byte chunks of a 64-column
-// chunk, so lane (g, tq) reads chunk 2*tq + h of row 8j + g - conflict-free - which
-// holds columns 16*tq + 8*h .. +7.  The operand of those columns sits in the stage's
-// operand part: column group kg = 8*chunk + 2*tq + h, row g at slot g ^ 2tq.
-// MT = 0: CUDA-core FMA (batch 1, fp32 operand); MT = 1, 2: mma.sync with MT tiles of
-// 8 batch rows, rows 0-7 of the M = 16 tile the bf16 hi parts, rows 8-15 the lo parts.
+// ... of every stage; a k block is the even (h = 0) or odd (h = 1) 16-byte chunks of a
+// 64-column chunk, so lane (g, tq) reads chunk 2*tq + h of row 8j + g - conflict-free -
+// which holds columns 16*tq + 8*h .. +7, column group kg = 8*chunk + 2*tq + h.  The lane
+// loads the operand of that group itself, D blocks ahead of its use (a register ring),
+// so the L2 latency overlaps the earlier blocks' work.  MT = 0: CUDA-core FMA (batch 1);
+// MT = 1, 2: mma.sync with MT tiles of 8 batch rows, rows 0-7 of the M = 16 tile the bf16
+// hi parts, rows 8-15 the lo parts.
 template <int MT, int G>
 __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDesc t, uint32_t& stage, bool& ab) {
+  constexpr int NQ = MT == 0 ? 2 : 2 * MT;       // 16-byte pieces per lane and k block
+  constexpr int Q = kRingBytes / (NQ * 512);     // ring entries: 4 (batch <= 8) or 2 (batch > 8)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, tq = lane & 3;
   const int K = gemv_K_dev(p, t.op);
   const int kc = t.kc;
   const int nst = (K + kc - 1) / kc;
+  const int kind = operand_kind(t.op);
+  const bf16* tiles = kind == 0 ? p.ax_t : (kind == 1 ? p.aa_t : p.ah_t);
+  const float* fop = kind == 0 ? p.ax_f : (kind == 1 ? p.aa_f : p.ah_f);
+  const int ld = kind == 0 ? p.ld_x : (kind == 1 ? p.ld_a : p.ld_h);
+  uint8_t* ring = sm.ring[warp];
   constexpr int R = 8 * G;
   constexpr int NMT = MT == 0 ? 1 : MT;
   float acc[G][NMT][4];
@@ -564,31 +513,47 @@ __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDes
     for (int mt = 0; mt < NMT; ++mt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[j][mt][e] = 0.f;
-  const int opart = round_up(kc, 256) * 16;  // bytes of one (tile, part) slice in the operand area
+
+  // the warp's k blocks in order: (stage s, block kb), kb = warp + 8i < 2 * chunks(s)
+  auto nblk = [&](int s) { return 2 * ((min(kc, K - s * kc) + kBoxCols - 1) / kBoxCols); };
+  auto kgroup = [&](int s, int kb) { return s * (kc / 8) + 8 * (kb >> 1) + 2 * tq + (kb & 1); };
+  auto advance = [&](int& s, int& kb) {
+    kb += kConsumerWarps;
+    while (s < nst && kb >= nblk(s)) { ++s; kb = warp; }
+  };
+  // operand prefetch: block j's operand sits in ring entry j % Q, fetched Q - 1 blocks ahead
+  int ps = 0, pkb = warp, fetched = 0, used = 0;
+  while (ps < nst && pkb >= nblk(ps)) ++ps;
+  if (!ab) {
+#pragma unroll
+    for (int i = 0; i < Q - 1; ++i) {
+      if (ps < nst) fetch_opnd<MT>(p, ring, fetched % Q, tiles, fop, ld, kgroup(ps, pkb), g, lane);
+      cp_async_commit();
+      ++fetched;
+      advance(ps, pkb);
+    }
+  }
 
   for (int s = 0; s < nst; ++s, ++stage) {
     const int slot = stage % kNumSlots;
     const uint32_t par = (stage / kNumSlots) & 1;
     if (!ab) ab = !mbar_wait_warp(p, &sm.full[slot], par, (p.trace && threadIdx.x == 0) ? &sm.wait_ns : nullptr);
-    if (!ab) ab = !mbar_wait_warp(p, &sm.ofull[slot], par, (p.trace && threadIdx.x == 0) ? &sm.wait_ns : nullptr);
     if (ab) continue;
     const unsigned long long tc0 = (p.trace && threadIdx.x == 0) ? gtimer() : 0ull;
     const uint8_t* tile = sm.pool[slot];
-    const uint8_t* opnd = sm.pool[slot] + kWeightBytes;
-    const int nb = 2 * ((min(kc, K - s * kc) + kBoxCols - 1) / kBoxCols);
+    const int nb = nblk(s);
     for (int kb = warp; kb < nb; kb += kConsumerWarps) {
-      const int kgl = 8 * (kb >> 1) + 2 * tq + (kb & 1);
+      if (ps < nst) fetch_opnd<MT>(p, ring, fetched % Q, tiles, fop, ld, kgroup(ps, pkb), g, lane);
+      cp_async_commit();
+      ++fetched;
+      advance(ps, pkb);
+      cp_async_wait<Q - 1>();  // the group of block `used` has landed
       const uint8_t* chunk = tile + (size_t)(kb >> 1) * (R * 128) + ((((2 * tq + (kb & 1)) ^ g)) << 4);
-      uint4 A[2 * NMT];
-      if constexpr (MT == 0) {
-        const uint4* f = reinterpret_cast<const uint4*>(opnd + (size_t)kgl * 32);
-        A[0] = f[0];
-        A[1] = f[1];
-      } else {
+      const uint8_t* ab_ = ring + (size_t)(used % Q) * NQ * 512 + lane * 16;
+      ++used;
+      uint4 A[NQ];
 #pragma unroll
-        for (int q = 0; q < 2 * MT; ++q)
-          A[q] = *reinterpret_cast<const uint4*>(opnd + (size_t)q * opart + (size_t)kgl * 128 + ((g ^ (2 * tq)) << 4));
-      }
+      for (int q = 0; q < NQ; ++q) A[q] = *reinterpret_cast<const uint4*>(ab_ + q * 512);
 #pragma unroll
       for (int j = 0; j < G; ++j) {
         const uint4 w = *reinterpret_cast<const uint4*>(chunk + (8 * j + g) * 128);
@@ -614,6 +579,7 @@ __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDes
     if (p.trace && threadIdx.x == 0) sm.tm[0] += gtimer() - tc0;
   }
 
+  cp_async_wait<0>();  // no copy into the ring may be in flight past this task
   // cross-warp reduction, one 8-row batch tile at a time: red[warp][block][batch g][8 rows]
   const unsigned long long tr0 = (p.trace && threadIdx.x == 0) ? gtimer() : 0ull;
   float* red = sm.red;
@@ -900,9 +866,6 @@ __device__ __noinline__ void attn_task(const KParams& p, Smem& sm, const TaskDes
     const bool has_new = newpos >= t0 && newpos < t1;
     if (!ab) ab = !mbar_wait_warp(p, &sm.full[slot], (stage / kNumSlots) & 1,
                                   (p.trace && threadIdx.x == 0) ? &sm.wait_ns : nullptr);
-    // the operand cursor passes attention stages with a bare arrival; waiting on it keeps
-    // this slot's operand phases in step with the stage count
-    if (!ab) ab = !mbar_wait_warp(p, &sm.ofull[slot], (stage / kNumSlots) & 1);
     uint8_t* kreg = sm.pool[slot];
     uint8_t* vreg = sm.pool[slot] + (size_t)T * HD * 2;
     if (has_new) {
@@ -1218,7 +1181,6 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNumSlots; ++s) {
       mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.ofull[s], 1);
       mbar_init(&sm.empty[s], kConsumerWarps);
     }
     fence_mbar_init();

@@ -332,10 +332,8 @@ int validate_plan(const mk_plan_s& p, std::string* err) {
           set_err(err, "sm %d task %zu: %d rows exceed %d", sm, k, rows, kMaxBlocks * 8);
           return MK_ERR_SCHEDULE_INVALID;
         }
-        const int tiles = (p.cfg.max_batch + 7) / 8;
         if (t.kc < kBoxCols || t.kc % kBoxCols || t.kc > round_up(K, kBoxCols) ||
-            (long long)rows * t.kc * 2 > kWeightBytes || tiles * 2 * round_up(t.kc, 256) * 16 > kOperandBytes ||
-            ((t.kc / 32) % kConsumerWarps != 0 && t.kc < K)) {
+            (long long)rows * t.kc * 2 > kSlotBytes || ((t.kc / 32) % kConsumerWarps != 0 && t.kc < K)) {
           set_err(err, "sm %d task %zu: stage of %d rows x %d columns does not fit a %d-byte slot", sm, k,
                   rows, t.kc, kSlotBytes);
           return MK_ERR_SCHEDULE_INVALID;
@@ -556,7 +554,7 @@ MK_API int mk_plan_inject_fault(mk_plan_t plan, int32_t kind, int32_t arg) {
     case MK_FAULT_OVERSIZE_STAGE: {
       for (auto& s : plan->streams)
         for (auto& t : s)
-          if (t.op == mk::OP_LMHEAD) { t.kc = (uint16_t)(2 * mk::kWeightBytes / (t.nunits * 8)); return MK_OK; }
+          if (t.op == mk::OP_LMHEAD) { t.kc = (uint16_t)(2 * mk::kSlotBytes / (t.nunits * 8)); return MK_OK; }
       return MK_ERR_INVALID_ARG;
     }
   }
