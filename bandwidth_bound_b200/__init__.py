@@ -88,6 +88,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "mk_create_from_plan": (ctypes.c_int, [vp, ctypes.POINTER(WeightPtrs), i32, ctypes.POINTER(vp)]),
         "mk_decode_step": (ctypes.c_int, [vp, vp, vp, vp, i32, ctypes.POINTER(KvCache), vp, vp, vp]),
         "mk_decode_step_host": (ctypes.c_int, [vp, vp, vp, vp, i32, ctypes.POINTER(KvCache), vp, vp, vp]),
+        "mk_decode_step_static": (ctypes.c_int, [ctypes.POINTER(ModelCfg), ctypes.POINTER(WeightPtrs), vp, vp, vp,
+                                                 i32, ctypes.POINTER(KvCache), vp, vp, vp]),
         "mk_get_status": (ctypes.c_int, [vp]),
         "mk_reset": (ctypes.c_int, [vp]),
         "mk_set_debug": (ctypes.c_int, [vp, vp]),
@@ -264,6 +266,34 @@ class Megakernel:
             self.close()
         except Exception:
             pass
+
+
+def decode_step_static(m, weights: dict, max_batch: int, max_ctx: int, token_ids, positions, seq_lens, kv,
+                       logits, argmax=None, stream=None, check: bool = True) -> int:
+    """One decode step through mk_decode_step_static: no handle, no device allocation.
+
+    The scratch is the library's fixed 16 MiB device array; the call returns after the
+    step has finished with its device status.
+    """
+    import torch
+
+    lib = load_library()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    cfg = model_cfg(m, max_batch, max_ctx)
+    L = m.n_layers
+    arr = {name: (ctypes.c_void_p * L)(*[_ptr(weights["layers"][i][name]) for i in range(L)])
+           for name in ("attn_norm", "wq", "wk", "wv", "wo", "mlp_norm", "w_gate", "w_up", "w_down")}
+    w = WeightPtrs(_ptr(weights["embed"]), _ptr(weights["final_norm"]), _ptr(weights["lm_head"]),
+                   *[ctypes.cast(arr[n], _PP) for n in ("attn_norm", "wq", "wk", "wv", "wo", "mlp_norm",
+                                                         "w_gate", "w_up", "w_down")])
+    kvs = Megakernel.kv_struct(kv)
+    rc = lib.mk_decode_step_static(ctypes.byref(cfg), ctypes.byref(w), _ptr(token_ids), _ptr(positions),
+                                   _ptr(seq_lens), int(token_ids.numel()), ctypes.byref(kvs), _ptr(logits),
+                                   _ptr(argmax), ctypes.c_void_p(stream.cuda_stream))
+    if check:
+        _check(rc, None, "mk_decode_step_static")
+    return rc
 
 
 def header_functions(header: Optional[str] = None) -> list[str]:

@@ -412,3 +412,272 @@ MK_API int mk_destroy(mk_handle_t h) {
 MK_API const char* mk_last_error(mk_handle_t h) { return h ? h->err.c_str() : g_err.c_str(); }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------
+// The decode step on statically allocated scratch.
+//
+// For callers that may not allocate device memory: a process whose HBM belongs to another
+// allocator (a caching allocator that has reserved the free memory, where a cudaMalloc
+// beside it fails or fragments the pool), or a latency-critical serving loop in which a
+// cudaMalloc/cudaFree would synchronise the device.  The scratch the megakernel needs
+// (task streams, tensor maps, activations, partial sums, dependency counters, RoPE table,
+// status word) is carved from one file-scope __device__ array instead of a handle's
+// cudaMalloc arena; the kernel and its launch are the ones mk_decode_step uses.
+
+#include <mutex>
+
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;  // the most one device's tables may take
+constexpr int kStaticMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+struct StaticState {
+  unsigned char* base = nullptr;   // device address of g_static_scratch on this device
+  bool ready = false;              // the tables below were uploaded for cfg/weights
+  bool dirty = false;              // counters and status must be cleared before the next launch
+  mk_model_cfg cfg{};
+  std::vector<const void*> wkey;   // the weight pointers the tables were built for
+  KParams kp{};
+  int* status = nullptr;           // device word the kernel reports a failure in
+  uint32_t epoch = 0;
+};
+
+StaticState g_static[kStaticMaxDevices];
+std::mutex g_static_mu[kStaticMaxDevices];
+
+void weight_key(const mk_model_cfg& c, const mk_weight_ptrs* w, std::vector<const void*>* out) {
+  out->assign({w->embed, w->final_norm, w->lm_head});
+  const void* const* per[9] = {w->attn_norm, w->wq, w->wk, w->wv, w->wo, w->mlp_norm, w->w_gate, w->w_up, w->w_down};
+  for (const void* const* a : per)
+    for (int l = 0; l < c.n_layers; ++l) out->push_back(a ? a[l] : nullptr);
+}
+
+bool same_key(const StaticState& s, const mk_model_cfg& c, const mk_weight_ptrs* w) {
+  if (!s.ready || std::memcmp(&s.cfg, &c, sizeof(c)) != 0) return false;
+  const void* head[3] = {w->embed, w->final_norm, w->lm_head};
+  for (int i = 0; i < 3; ++i)
+    if (s.wkey[i] != head[i]) return false;
+  const void* const* per[9] = {w->attn_norm, w->wq, w->wk, w->wv, w->wo, w->mlp_norm, w->w_gate, w->w_up, w->w_down};
+  size_t k = 3;
+  for (const void* const* a : per)
+    for (int l = 0; l < c.n_layers; ++l, ++k)
+      if (!a || s.wkey[k] != a[l]) return false;
+  return true;
+}
+
+// Build the schedule and tensor maps for (cfg, weights), lay the scratch out in the static
+// array, clear it and upload the tables.  Host-synchronous on `stream`.
+int static_setup(StaticState& s, const mk_model_cfg& c, const mk_weight_ptrs* w, int dev, cudaStream_t stream) {
+  s.ready = false;
+  if (!w->embed || !w->final_norm || !w->lm_head || !w->attn_norm || !w->wq || !w->wk || !w->wv || !w->wo ||
+      !w->mlp_norm || !w->w_gate || !w->w_up || !w->w_down)
+    return fail(nullptr, MK_ERR_INVALID_ARG, "mk_decode_step_static: null weight pointer");
+  std::vector<LayerW> lw(c.n_layers > 0 ? c.n_layers : 0);
+  const void* all[3] = {w->embed, w->final_norm, w->lm_head};
+  for (const void* p : all)
+    if (!aligned16(p)) return fail(nullptr, MK_ERR_INVALID_ARG, "mk_decode_step_static: weights must be 16-byte aligned");
+  for (int l = 0; l < c.n_layers; ++l) {
+    const void* ps[9] = {w->attn_norm[l], w->wq[l], w->wk[l], w->wv[l], w->wo[l],
+                         w->mlp_norm[l], w->w_gate[l], w->w_up[l], w->w_down[l]};
+    for (const void* p : ps)
+      if (!p || !aligned16(p))
+        return fail(nullptr, MK_ERR_INVALID_ARG, "mk_decode_step_static: layer weight null or not 16-byte aligned");
+    lw[l] = LayerW{(const __nv_bfloat16*)ps[0], (const __nv_bfloat16*)ps[1], (const __nv_bfloat16*)ps[2],
+                   (const __nv_bfloat16*)ps[3], (const __nv_bfloat16*)ps[4], (const __nv_bfloat16*)ps[5],
+                   (const __nv_bfloat16*)ps[6], (const __nv_bfloat16*)ps[7], (const __nv_bfloat16*)ps[8]};
+  }
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return fail(nullptr, MK_ERR_NO_DEVICE, "no CUDA device");
+  if (prop.major != 10) return fail(nullptr, MK_ERR_NO_DEVICE, "the kernel is built for sm_100a (B200)");
+  if (!prop.cooperativeLaunch) return fail(nullptr, MK_ERR_NO_DEVICE, "device lacks cooperative launch");
+  int regs = 0, lmem = 0, maxthr = 0;
+  cudaError_t ce = mk::kernel_attributes(&regs, &lmem, &maxthr);
+  if (ce != cudaSuccess) return cuda_fail(nullptr, ce, "kernel attributes");
+  if (maxthr < mk::kThreads) return fail(nullptr, MK_ERR_CUDA, "kernel cannot run 288 threads");
+
+  mk_plan_opts o{};
+  o.num_sms = prop.multiProcessorCount;
+  mk_plan_s plan;
+  std::string e;
+  int rc = mk::build_plan(c, &o, &plan, &e);
+  if (rc) return fail(nullptr, rc, "plan: " + e);
+  rc = mk::validate_plan(plan, &e);
+  if (rc) return fail(nullptr, rc, "schedule rejected: " + e);
+
+  const mk::Geometry G = mk::geometry(c);
+  const int S = plan.num_sms * plan.attn_slots_per_sm;
+  const int mb = c.max_batch;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t at = off; off += (bytes + 255) & ~size_t(255); return at; };
+  std::vector<mk::TaskDesc> flat;
+  std::vector<uint32_t> offs(plan.num_sms + 1, 0);
+  for (int sm = 0; sm < plan.num_sms; ++sm) {
+    flat.insert(flat.end(), plan.streams[sm].begin(), plan.streams[sm].end());
+    offs[sm + 1] = (uint32_t)flat.size();
+  }
+  const size_t o_layers = take(sizeof(LayerW) * c.n_layers);
+  const size_t o_tasks = take(sizeof(mk::TaskDesc) * flat.size());
+  const size_t o_offs = take(sizeof(uint32_t) * offs.size());
+  const size_t o_maps = take(sizeof(CUtensorMap) * (size_t)mk::num_tmaps(G.L));
+  const size_t o_x = take(sizeof(float) * mb * G.d);
+  const size_t o_q = take(sizeof(float) * mb * G.qdim);
+  const int ld_x = mk::round_up(G.d, mk::kBoxCols), ld_a = mk::round_up(G.qdim, mk::kBoxCols),
+            ld_h = mk::round_up(G.F, mk::kBoxCols);
+  const int ntiles = (mb + 7) / 8;
+  auto opbytes = [&](int ld) { return (size_t)ntiles * 2 * ld * 8 * 2 + (size_t)ld * 4; };
+  const size_t o_ax = take(opbytes(ld_x)), o_aa = take(opbytes(ld_a)), o_ah = take(opbytes(ld_h));
+  const int ssq_stride = plan.max_phase_tasks * mb;
+  const size_t o_ssq = take(sizeof(float) * mk::num_ssq_inst(G.L) * ssq_stride);
+  const size_t o_part = take(sizeof(float) * (size_t)S * G.g * (G.hd + 2));
+  const size_t o_lm = take(sizeof(float2) * (size_t)plan.n_lm_tasks * mb);
+  const size_t o_ctr = take(sizeof(uint32_t) * mk::num_counters(G.L));
+  const size_t o_cmb = take(sizeof(uint32_t) * (size_t)G.L * mb * G.nkv);
+  const size_t o_ctl = take(sizeof(uint32_t) * 2);
+  const size_t o_status = take(sizeof(int));
+  const size_t o_rope = take(sizeof(float2) * (size_t)c.max_ctx * (G.hd / 2));
+  const size_t total = off;
+  if (total > kStaticScratchBytes)
+    return fail(nullptr, MK_ERR_INVALID_ARG,
+                "mk_decode_step_static: this model needs " + std::to_string(total) +
+                    " bytes of scratch; the static area holds " + std::to_string(kStaticScratchBytes) +
+                    " (lower max_batch or max_ctx, or use mk_create)");
+
+  std::vector<CUtensorMap> maps;
+  std::string merr = build_tensor_maps(c, w, maps);
+  if (!merr.empty()) return fail(nullptr, MK_ERR_CUDA, merr);
+
+  unsigned char* A = s.base;
+  ce = cudaMemsetAsync(A, 0, total, stream);
+  if (ce == cudaSuccess)
+    ce = cudaMemcpyAsync(A + o_layers, lw.data(), sizeof(LayerW) * c.n_layers, cudaMemcpyHostToDevice, stream);
+  if (ce == cudaSuccess)
+    ce = cudaMemcpyAsync(A + o_tasks, flat.data(), sizeof(mk::TaskDesc) * flat.size(), cudaMemcpyHostToDevice,
+                         stream);
+  if (ce == cudaSuccess)
+    ce = cudaMemcpyAsync(A + o_offs, offs.data(), sizeof(uint32_t) * offs.size(), cudaMemcpyHostToDevice, stream);
+  if (ce == cudaSuccess)
+    ce = cudaMemcpyAsync(A + o_maps, maps.data(), sizeof(CUtensorMap) * maps.size(), cudaMemcpyHostToDevice,
+                         stream);
+  if (ce == cudaSuccess)
+    ce = mk::launch_rope_table((float2*)(A + o_rope), c.max_ctx, G.hd, c.rope_theta, stream);
+  if (ce == cudaSuccess) ce = cudaStreamSynchronize(stream);
+  if (ce != cudaSuccess) return cuda_fail(nullptr, ce, "mk_decode_step_static: upload");
+
+  KParams k{};
+  k.L = G.L; k.d = G.d; k.nq = G.nq; k.nkv = G.nkv; k.hd = G.hd; k.F = G.F; k.V = G.V; k.g = G.g;
+  k.qdim = G.qdim; k.max_b = mb; k.max_ctx = c.max_ctx; k.eps = c.rms_eps;
+  k.layers = (const LayerW*)(A + o_layers);
+  k.embed = (const __nv_bfloat16*)w->embed;
+  k.final_norm = (const __nv_bfloat16*)w->final_norm;
+  k.lm_head = (const __nv_bfloat16*)w->lm_head;
+  k.tasks = (const mk::TaskDesc*)(A + o_tasks);
+  k.task_off = (const uint32_t*)(A + o_offs);
+  k.num_sms = plan.num_sms;
+  k.n_slots = S;
+  k.n_lm_tasks = plan.n_lm_tasks;
+  k.tmaps = A + o_maps;
+  k.x = (float*)(A + o_x); k.q = (float*)(A + o_q);
+  auto carve = [&](size_t at, int ld, __nv_bfloat16** t, float** f) {
+    *t = (__nv_bfloat16*)(A + at);
+    *f = (float*)(*t + (size_t)ntiles * 2 * ld * 8);
+  };
+  carve(o_ax, ld_x, &k.ax_t, &k.ax_f);
+  carve(o_aa, ld_a, &k.aa_t, &k.aa_f);
+  carve(o_ah, ld_h, &k.ah_t, &k.ah_f);
+  k.ld_x = ld_x; k.ld_a = ld_a; k.ld_h = ld_h;
+  k.ssq = (float*)(A + o_ssq); k.ssq_stride = ssq_stride; k.part = (float*)(A + o_part);
+  k.lmpart = (float2*)(A + o_lm);
+  k.ctr = (uint32_t*)(A + o_ctr); k.cmb = (uint32_t*)(A + o_cmb); k.ctl = (uint32_t*)(A + o_ctl);
+  k.host_status = (int*)(A + o_status);
+  k.rope = (const float2*)(A + o_rope);
+  k.timeout_ns = 1000000000ull;
+  k.dbg = nullptr;
+  k.trace = nullptr;
+  s.kp = k;
+  s.status = (int*)(A + o_status);
+  s.cfg = c;
+  weight_key(c, w, &s.wkey);
+  s.epoch = 0;
+  s.dirty = false;
+  s.ready = true;
+  return MK_OK;
+}
+
+// Zero what the kernel expects to start at zero after a failed step: the dependency and
+// combine counters, the abort flag and first error code, the status word.
+cudaError_t static_clear(StaticState& s, cudaStream_t stream) {
+  const KParams& k = s.kp;
+  cudaError_t ce = cudaMemsetAsync(k.ctr, 0, sizeof(uint32_t) * mk::num_counters(k.L), stream);
+  if (ce == cudaSuccess) ce = cudaMemsetAsync(k.cmb, 0, sizeof(uint32_t) * (size_t)k.L * k.max_b * k.nkv, stream);
+  if (ce == cudaSuccess) ce = cudaMemsetAsync(k.ctl, 0, sizeof(uint32_t) * 2, stream);
+  if (ce == cudaSuccess) ce = cudaMemsetAsync(s.status, 0, sizeof(int), stream);
+  return ce;
+}
+
+}  // namespace
+
+extern "C" MK_API int mk_decode_step_static(const mk_model_cfg* cfg, const mk_weight_ptrs* weights,
+                                            const int32_t* token_ids, const int32_t* positions,
+                                            const int32_t* seq_lens, int32_t batch, const mk_kv_cache* kv,
+                                            float* logits_out, int32_t* argmax_out, mk_stream_t stream) {
+  if (!cfg || !weights || !token_ids || !positions || !seq_lens || !kv || !logits_out)
+    return fail(nullptr, MK_ERR_INVALID_ARG, "mk_decode_step_static: null argument");
+  if (batch < 1 || batch > cfg->max_batch)
+    return fail(nullptr, MK_ERR_INVALID_ARG, "mk_decode_step_static: batch must be in [1, max_batch]");
+  if (!kv->k_pool || !kv->v_pool || !kv->page_table || kv->num_pages < 1 || kv->max_pages_per_seq < 1)
+    return fail(nullptr, MK_ERR_INVALID_ARG, "mk_decode_step_static: bad kv cache description");
+  if (!aligned16(kv->k_pool) || !aligned16(kv->v_pool))
+    return fail(nullptr, MK_ERR_INVALID_ARG, "mk_decode_step_static: kv pools must be 16-byte aligned");
+  std::string cerr;
+  int rc = mk::check_cfg(*cfg, &cerr);
+  if (rc) return fail(nullptr, rc, "mk_decode_step_static: " + cerr);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(nullptr, MK_ERR_NO_DEVICE, "no CUDA device");
+  if (dev < 0 || dev >= kStaticMaxDevices)
+    return fail(nullptr, MK_ERR_NO_DEVICE, "mk_decode_step_static: device ordinal above 63");
+  std::lock_guard<std::mutex> lock(g_static_mu[dev]);
+  StaticState& s = g_static[dev];
+  cudaStream_t st = (cudaStream_t)stream;
+  if (!s.base) {
+    // once per device, with that device current: the address of this device's copy of the array
+    void* p = nullptr;
+    cudaError_t ce = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (ce != cudaSuccess) return cuda_fail(nullptr, ce, "mk_decode_step_static: cudaGetSymbolAddress");
+    s.base = (unsigned char*)p;
+  }
+  if (!same_key(s, *cfg, weights)) {
+    rc = static_setup(s, *cfg, weights, dev, st);
+    if (rc) return rc;
+  }
+  if (s.dirty) {
+    cudaError_t ce = static_clear(s, st);
+    if (ce != cudaSuccess) return cuda_fail(nullptr, ce, "mk_decode_step_static: clear");
+    s.epoch = 0;
+    s.dirty = false;
+  }
+  KParams p = s.kp;
+  p.tok = token_ids; p.pos = positions; p.lens = seq_lens; p.b = batch;
+  p.kpool = (__nv_bfloat16*)kv->k_pool; p.vpool = (__nv_bfloat16*)kv->v_pool;
+  p.ptable = kv->page_table; p.num_pages = kv->num_pages; p.mpps = kv->max_pages_per_seq;
+  p.logits = logits_out; p.argmax = argmax_out;
+  p.epoch = ++s.epoch;
+  cudaError_t ce = mk::launch_decode(p, st);
+  if (ce != cudaSuccess) {
+    --s.epoch;
+    return cuda_fail(nullptr, ce, "mk_decode_step_static: megakernel launch");
+  }
+  int status = 0;
+  ce = cudaMemcpyAsync(&status, s.status, sizeof(int), cudaMemcpyDeviceToHost, st);
+  if (ce == cudaSuccess) ce = cudaStreamSynchronize(st);
+  if (ce != cudaSuccess) {
+    s.dirty = true;
+    return cuda_fail(nullptr, ce, "mk_decode_step_static: step");
+  }
+  if (status != 0) {
+    s.dirty = true;
+    return fail(nullptr, status, "mk_decode_step_static: the step failed on the device");
+  }
+  return MK_OK;
+}

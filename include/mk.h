@@ -153,6 +153,32 @@ MK_API int mk_decode_step_host(mk_handle_t h, const int32_t *token_ids, const in
                                const int32_t *seq_lens, int32_t batch, const mk_kv_cache *kv,
                                float *logits_host, int32_t *argmax_host, mk_stream_t stream);
 
+/* The same step without a handle and without allocating: for callers that may not
+ * allocate device memory (a process whose HBM belongs to another allocator, such as a
+ * caching allocator that has reserved the free memory, or a latency-critical loop in
+ * which cudaMalloc/cudaFree would synchronise the device).  The pages describe no such
+ * entry point; it is an interface variant of mk_decode_step, with the same kernel.
+ *   cfg, weights  as for mk_create; arguments from token_ids on as for mk_decode_step.
+ * Scratch: one file-scope __device__ array of 16 MiB per device (task streams, tensor
+ * maps, activations, counters, RoPE table).  A model whose scratch exceeds it (it
+ * grows with n_layers, max_batch and max_ctx) is rejected with MK_ERR_INVALID_ARG
+ * before anything is launched.  No call allocates device or pinned host memory.
+ * Set-up: the first call on a device (with that device current) looks the array's
+ * address up, builds and validates the schedule, encodes the tensor maps, clears the
+ * array and uploads the tables, synchronising `stream`; a later call with another cfg
+ * or other weight pointers does the same again.  Make the first call before any
+ * stream capture.
+ * Each call synchronises `stream` and returns the step's device status (MK_OK,
+ * MK_ERR_DEVICE_TIMEOUT, MK_ERR_BOUNDS); after a device error the next call first
+ * clears the counters and the status.  All calls on a device share the one array, so
+ * two of its steps that overlapped on the GPU would race on it: the entry point holds
+ * a per-device lock until its step has finished, which makes calls from several host
+ * threads run one after another.  Messages: mk_last_error(NULL). */
+MK_API int mk_decode_step_static(const mk_model_cfg *cfg, const mk_weight_ptrs *weights,
+                                 const int32_t *token_ids, const int32_t *positions,
+                                 const int32_t *seq_lens, int32_t batch, const mk_kv_cache *kv,
+                                 float *logits_out, int32_t *argmax_out, mk_stream_t stream);
+
 /* Sticky device status of the handle's last steps: MK_OK, MK_ERR_DEVICE_TIMEOUT
  * or MK_ERR_BOUNDS.  Read it after synchronising the stream of the step. */
 MK_API int mk_get_status(mk_handle_t h);
