@@ -153,9 +153,17 @@ def max_over_ranks(world, v: float) -> float:
         return v
     import torch.distributed as dist
 
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world: int, total_ms_this_rank: float, steps: int, batch: int) -> tuple[float, float]:
+    """(ms per step, tokens/s of the whole job): the slowest rank's device time over
+    `steps` steps, every rank decoding its own batch of `batch` sequences."""
+    ms = max_over_ranks(world, total_ms_this_rank) / steps
+    return ms, world * batch / (ms / 1e3)
 
 
 def traffic_from_profile(workload: str):
@@ -245,6 +253,14 @@ def run_reference(args, world, rank):
 def time_steps(fn, steps, stream, flush=None):
     """CUDA-event time of `steps` calls of fn on `stream` (ms total, per-step list)."""
     per = []
+    torch.cuda.nvtx.range_push("timed")  # lets ncu --nvtx-include "timed/" select these launches
+    try:
+        return _time_steps(fn, steps, stream, flush, per)
+    finally:
+        torch.cuda.nvtx.range_pop()
+
+
+def _time_steps(fn, steps, stream, flush, per):
     if flush is None:
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
@@ -344,8 +360,7 @@ def run_mk(args, world, rank, local):
     barrier(world)
     clk = clocks.stop()
     assert h.status() == mk.MK_OK, f"device status {h.status()}"
-    ms = max_over_ranks(world, total_ms) / args.steps
-    value = world * b / (ms / 1e3)
+    ms, value = job_throughput(world, total_ms, args.steps, b)
     peaks = measured_peaks()
     achieved = B / (ms / 1e3) / 1e9
     traffic = traffic_from_profile(w.name)
