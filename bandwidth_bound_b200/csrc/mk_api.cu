@@ -26,6 +26,8 @@ struct mk_handle_s {
   float* d_logits = nullptr;    // device logits for the host-buffer step
   int32_t* d_argmax = nullptr;
   uint32_t epoch = 0;
+  const void *kv_k = nullptr, *kv_v = nullptr;  // pools the KV tensor maps in kp were encoded for
+  int32_t kv_pages = 0;
   std::string err;
 };
 
@@ -119,6 +121,40 @@ static std::string build_tensor_maps(const mk_model_cfg& c, const mk_weight_ptrs
   return "";
 }
 
+// Tensor maps of the K and V pools, viewed as rows of head_dim values ([L][pages][nkv][16]
+// rows): boxes of one 16-token page of one head with 128-byte swizzle.  head_dim 64: a 2-D
+// box of 64 x 16; head_dim 128: a 3-D box {64 columns, 16 rows, 2 halves}, the halves
+// outermost, so that each half of a page lands as 16 rows of 128 bytes.
+static std::string encode_kv_maps(const mk_model_cfg& c, const mk_kv_cache* kv, KParams& k) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (!encode) return "cuTensorMapEncodeTiled is not available";
+  const uint64_t rows = (uint64_t)c.n_layers * (uint64_t)kv->num_pages * c.n_kv_heads * mk::kPage;
+  if (rows >= (1ull << 31)) return "KV pool too large (layers * pages * kv heads * 16 must stay below 2^31)";
+  void* pools[2] = {kv->k_pool, kv->v_pool};
+  mk::TmaDesc* maps[2] = {&k.kmap, &k.vmap};
+  for (int i = 0; i < 2; ++i) {
+    CUresult r;
+    cuuint32_t es[3] = {1, 1, 1};
+    if (c.head_dim == 64) {
+      cuuint64_t dims[2] = {64, rows};
+      cuuint64_t strides[1] = {128};
+      cuuint32_t box[2] = {64, (cuuint32_t)mk::kPage};
+      r = encode(reinterpret_cast<CUtensorMap*>(maps[i]), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pools[i], dims,
+                 strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    } else {
+      cuuint64_t dims[3] = {64, rows, 2};
+      cuuint64_t strides[2] = {256, 128};
+      cuuint32_t box[3] = {64, (cuuint32_t)mk::kPage, 2};
+      r = encode(reinterpret_cast<CUtensorMap*>(maps[i]), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, pools[i], dims,
+                 strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    }
+    if (r != CUDA_SUCCESS) return "cuTensorMapEncodeTiled failed for the KV pools (error " + std::to_string((int)r) + ")";
+  }
+  return "";
+}
+
 extern "C" {
 
 MK_API int mk_create_from_plan(mk_plan_t plan, const mk_weight_ptrs* w, int32_t flags, mk_handle_t* out) {
@@ -197,7 +233,7 @@ MK_API int mk_create_from_plan(mk_plan_t plan, const mk_weight_ptrs* w, int32_t 
   const size_t o_ax = take(opbytes(ld_x)), o_aa = take(opbytes(ld_a)), o_ah = take(opbytes(ld_h));
   const int ssq_stride = plan->max_phase_tasks * mb;
   const size_t o_ssq = take(sizeof(float) * mk::num_ssq_inst(G.L) * ssq_stride);
-  const size_t o_part = take(sizeof(float) * (size_t)S * G.g * (G.hd + 2));
+  const size_t o_part = take(sizeof(float) * (size_t)mb * G.nkv * mk::kMaxChunksPerSeq * G.g * (G.hd + 2));
   const size_t o_lm = take(sizeof(float2) * (size_t)plan->n_lm_tasks * mb);
   const size_t o_ctr = take(sizeof(uint32_t) * mk::num_counters(G.L));
   const size_t o_cmb = take(sizeof(uint32_t) * (size_t)G.L * mb * G.nkv);
@@ -304,6 +340,16 @@ static int check_step_args(mk_handle_t h, const void* tok, const void* pos, cons
 
 static int launch_step(mk_handle_t h, const int32_t* tok, const int32_t* pos, const int32_t* lens, int32_t batch,
                        const mk_kv_cache* kv, float* logits, int32_t* argmax, cudaStream_t s) {
+  if (kv->k_pool != h->kv_k || kv->v_pool != h->kv_v || kv->num_pages != h->kv_pages) {
+    const std::string e = encode_kv_maps(h->plan.cfg, kv, h->kp);
+    if (!e.empty()) {
+      h->kv_k = h->kv_v = nullptr;
+      return fail(h, MK_ERR_INVALID_ARG, "mk_decode_step: " + e);
+    }
+    h->kv_k = kv->k_pool;
+    h->kv_v = kv->v_pool;
+    h->kv_pages = kv->num_pages;
+  }
   KParams p = h->kp;
   p.tok = tok; p.pos = pos; p.lens = lens; p.b = batch;
   p.kpool = (__nv_bfloat16*)kv->k_pool; p.vpool = (__nv_bfloat16*)kv->v_pool;
@@ -442,6 +488,8 @@ struct StaticState {
   KParams kp{};
   int* status = nullptr;           // device word the kernel reports a failure in
   uint32_t epoch = 0;
+  const void *kv_k = nullptr, *kv_v = nullptr;  // pools the KV tensor maps in kp were encoded for
+  int32_t kv_pages = 0;
 };
 
 StaticState g_static[kStaticMaxDevices];
@@ -530,7 +578,7 @@ int static_setup(StaticState& s, const mk_model_cfg& c, const mk_weight_ptrs* w,
   const size_t o_ax = take(opbytes(ld_x)), o_aa = take(opbytes(ld_a)), o_ah = take(opbytes(ld_h));
   const int ssq_stride = plan.max_phase_tasks * mb;
   const size_t o_ssq = take(sizeof(float) * mk::num_ssq_inst(G.L) * ssq_stride);
-  const size_t o_part = take(sizeof(float) * (size_t)S * G.g * (G.hd + 2));
+  const size_t o_part = take(sizeof(float) * (size_t)mb * G.nkv * mk::kMaxChunksPerSeq * G.g * (G.hd + 2));
   const size_t o_lm = take(sizeof(float2) * (size_t)plan.n_lm_tasks * mb);
   const size_t o_ctr = take(sizeof(uint32_t) * mk::num_counters(G.L));
   const size_t o_cmb = take(sizeof(uint32_t) * (size_t)G.L * mb * G.nkv);
@@ -596,6 +644,7 @@ int static_setup(StaticState& s, const mk_model_cfg& c, const mk_weight_ptrs* w,
   k.dbg = nullptr;
   k.trace = nullptr;
   s.kp = k;
+  s.kv_k = s.kv_v = nullptr;
   s.status = (int*)(A + o_status);
   s.cfg = c;
   weight_key(c, w, &s.wkey);
@@ -656,6 +705,16 @@ extern "C" MK_API int mk_decode_step_static(const mk_model_cfg* cfg, const mk_we
     if (ce != cudaSuccess) return cuda_fail(nullptr, ce, "mk_decode_step_static: clear");
     s.epoch = 0;
     s.dirty = false;
+  }
+  if (kv->k_pool != s.kv_k || kv->v_pool != s.kv_v || kv->num_pages != s.kv_pages) {
+    const std::string e = encode_kv_maps(*cfg, kv, s.kp);
+    if (!e.empty()) {
+      s.kv_k = s.kv_v = nullptr;
+      return fail(nullptr, MK_ERR_INVALID_ARG, "mk_decode_step_static: " + e);
+    }
+    s.kv_k = kv->k_pool;
+    s.kv_v = kv->v_pool;
+    s.kv_pages = kv->num_pages;
   }
   KParams p = s.kp;
   p.tok = token_ids; p.pos = positions; p.lens = seq_lens; p.b = batch;

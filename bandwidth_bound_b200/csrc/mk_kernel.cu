@@ -33,13 +33,11 @@ struct Smem {
   alignas(16) float red[kRedBytes / 4];                 // GEMV cross-warp partials / attention merge
   alignas(128) uint8_t ring[kConsumerWarps][kRingBytes];  // per warp: operands of its upcoming k blocks
   alignas(16) float ep[kMaxBlocks * 8][kMaxBatch];       // per-task results [row][batch]
-  alignas(16) float pw[kConsumerWarps][16 * 8];          // attention probabilities [token][head]
   float mw[kConsumerWarps][8], lw[kConsumerWarps][8];    // attention merge state per warp
-  float corr[kConsumerWarps][8];
   float inv_rms[kMaxBatch];
   alignas(8) uint64_t full[kNumSlots];                   // weight/KV bytes of the stage landed
   alignas(8) uint64_t empty[kNumSlots];                  // all consumer warps done with the stage
-  int attn_ch, attn_n, bad, flag, flag2;
+  int attn_R, bad, flag, flag2;  // attn_R: tokens per attention range (this step)
   unsigned long long wait_ns;  // time warp 0 spent waiting for pool slots in the current task (tracing)
   unsigned long long tm[3];    // tracing: compute, reduce, epilogue ns of the current task (warp 0)
   int inv_inst;                // ssq instance whose 1/rms sm.inv_rms holds (-1: none)
@@ -264,57 +262,68 @@ __device__ __forceinline__ void issue_gemv_chunk(const KParams& p, const TaskDes
   }
 }
 
-// Split-K attention: slot w -> (sequence, kv head, chunk), or false for an empty slot.
-struct AttnWork {
-  int i, h, c, nc, n, c0, c1;
+// Split-K attention work.  The (sequence i, kv head h) pairs are laid end to end, pair
+// (i, h) taking ceil16(len_i) token places; attention range u covers places [u R, u R + R)
+// of that line.  Its pieces are the parts of the pairs it overlaps, cut at 16-token
+// (page) boundaries, so every range holds the same number of KV bytes whatever the
+// lengths, and a piece is the unit of split-K state (one log-sum-exp partial).
+struct AttnPiece {
+  int i, h;    // sequence, kv head
+  int c, nc;   // piece index within the pair, pieces of the pair
+  int n;       // keys of the sequence (position + 1)
+  int t0, t1;  // tokens [t0, t1) of the pair, t0 a multiple of 16
 };
 
-__device__ bool attn_work(const KParams& p, int ch, int w, AttnWork& a) {
+// Piece j (in order) of range u, or false past the last one.
+__device__ bool attn_piece(const KParams& p, int R, int u, int j, AttnPiece& a) {
+  const long long lo = (long long)u * R, hi = lo + R;
+  long long off = 0;
   for (int i = 0; i < p.b; ++i) {
     const int n = p.lens[i];
-    const int nc = (n + ch - 1) / ch;
-    const int cnt = p.nkv * nc;
-    if (w < cnt) {
-      a.i = i;
-      a.h = w / nc;
-      a.c = w - a.h * nc;
-      a.nc = nc;
-      a.n = n;
-      a.c0 = a.c * ch;
-      a.c1 = min(a.c0 + ch, n);
-      return true;
+    const int Lp = (n + kPage - 1) / kPage * kPage;
+    const long long blk = (long long)p.nkv * Lp;
+    if (off + blk > lo) {
+      if (off >= hi) return false;
+      const int h0 = lo > off ? (int)((lo - off) / Lp) : 0;
+      const int h1 = (int)min((long long)p.nkv - 1, (hi - 1 - off) / Lp);
+      for (int h = h0; h <= h1; ++h) {
+        const long long st = off + (long long)h * Lp;
+        const long long ts = (lo > st ? lo : st) - st, te = (hi < st + n ? hi : st + n) - st;
+        if (ts >= te) continue;
+        if (j-- > 0) continue;
+        a.i = i;
+        a.h = h;
+        a.n = n;
+        a.t0 = (int)ts;
+        a.t1 = (int)te;
+        a.c = u - (int)(st / R);
+        a.nc = (int)((st + n - 1) / R - st / R) + 1;
+        return true;
+      }
     }
-    w -= cnt;
+    off += blk;
   }
   return false;
 }
 
-// Chunk length: the smallest multiple of 16 such that all chunks fit the slots and
-// no (sequence, kv head) has more than kMaxChunksPerSeq chunks.
-__device__ void attn_setup(const KParams& p, int* ch_out, int* n_out) {
-  long long sum = 0;
-  int mx = 1;
+// Range length R (tokens, a multiple of 16): the padded pair lengths spread evenly over the
+// n_slots ranges, at least one full stage, and short enough that no pair is cut into more
+// than kMaxChunksPerSeq pieces.
+__device__ int attn_setup(const KParams& p) {
+  long long tot = 0;
+  int mx = kPage;
   for (int i = 0; i < p.b; ++i) {
-    sum += p.lens[i];
-    mx = max(mx, p.lens[i]);
+    const int Lp = (p.lens[i] + kPage - 1) / kPage * kPage;
+    tot += (long long)p.nkv * Lp;
+    mx = max(mx, Lp);
   }
-  int ch = ((mx + 16 * kMaxChunksPerSeq - 1) / (16 * kMaxChunksPerSeq)) * 16;
-  ch = max(ch, 16);
-  const long long room = (long long)p.n_slots - (long long)p.nkv * p.b;
-  if (room > 0) {
-    long long lb = ((long long)p.nkv * sum + room - 1) / room;
-    lb = ((lb + 15) / 16) * 16;
-    if (lb > ch) { const long long cap = (long long)((mx + 15) / 16) * 16; ch = (int)(lb < cap ? lb : cap); }
-  }
-  for (;; ch += 16) {
-    long long tot = 0;
-    for (int i = 0; i < p.b; ++i) tot += (long long)p.nkv * ((p.lens[i] + ch - 1) / ch);
-    if (tot <= p.n_slots || ch >= mx) {
-      *ch_out = ch;
-      *n_out = (int)tot;
-      return;
-    }
-  }
+  long long R = (tot + p.n_slots - 1) / p.n_slots;
+  R = (R + kPage - 1) / kPage * kPage;
+  const long long rmin = attn_stage_tokens(p.hd);
+  const long long rcap = ((mx + kMaxChunksPerSeq - 3) / (kMaxChunksPerSeq - 2) + kPage - 1) / kPage * kPage;
+  if (R < rmin) R = rmin;
+  if (R < rcap) R = rcap;
+  return (int)R;
 }
 
 // ---------------------------------------------------------------------------------------
@@ -324,59 +333,16 @@ __device__ void attn_setup(const KParams& p, int* ch_out, int* n_out) {
 // projection), 2 SwiGLU output (down projection).
 __device__ __forceinline__ int operand_kind(int op) { return op == OP_OPROJ ? 1 : (op == OP_DOWN ? 2 : 0); }
 
-__device__ __forceinline__ int attn_stages(const AttnWork& a, int T) { return (a.c1 - a.c0 + T - 1) / T; }
-
-// Stages (pool slots) a task occupies: K / kc for a GEMV, its pages for an attention slot.
-__device__ __forceinline__ int task_stages(const KParams& p, const Smem& sm, const TaskDesc& t, AttnWork& a) {
+// Pool stages of a GEMV task: K / kc.
+__device__ __forceinline__ int gemv_stages(const KParams& p, const TaskDesc& t) {
   if (t.op == OP_EMBED) return 0;
-  if (t.op == OP_ATTN) {
-    if ((int)t.u0 >= sm.attn_n || !attn_work(p, sm.attn_ch, (int)t.u0, a)) return 0;
-    return attn_stages(a, attn_stage_tokens(p.hd));
-  }
   const int K = gemv_K_dev(p, t.op);
   return (K + t.kc - 1) / t.kc;
 }
 
-// Weights (or KV pages) of stage s of task t into slot `slot`.  Returns false on a bad page id.
-__device__ bool issue_weights(const KParams& p, Smem& sm, const TaskDesc& t, const AttnWork& a, int s, int slot,
-                              uint64_t pol) {
+// Weights of stage s of GEMV task t into slot `slot`: one tiled box per 64 columns.
+__device__ void issue_weights(const KParams& p, Smem& sm, const TaskDesc& t, int s, int slot, uint64_t pol) {
   const int lane = threadIdx.x & 31;
-  if (t.op == OP_ATTN) {
-    const int T = attn_stage_tokens(p.hd);
-    const int newpos = a.n - 1;
-    const int t0 = a.c0 + s * T, t1 = min(t0 + T, a.c1);
-    const int tp = min(t1, newpos);  // prior entries only; the new one is read after the wait
-    bool bad = false;
-    for (int pg = t0 / kPage; pg * kPage < tp; ++pg) {
-      const int id = p.ptable[a.i * p.mpps + pg];
-      if (id < 0 || id >= p.num_pages) bad = true;
-    }
-    if (bad) return false;
-    const uint32_t bytes = tp > t0 ? (uint32_t)(tp - t0) * p.hd * 2u * 2u : 0u;
-    if (lane == 0) {
-      if (bytes) mbar_expect_tx(&sm.full[slot], bytes);
-      else mbar_arrive(&sm.full[slot]);
-    }
-    __syncwarp();
-    if (bytes) {
-      const size_t head_stride = (size_t)kPage * p.hd;
-      uint8_t* kdst = sm.pool[slot];
-      uint8_t* vdst = sm.pool[slot] + (size_t)T * p.hd * 2;
-      const int pg0 = t0 / kPage;
-      const int npg = (tp - 1) / kPage - pg0 + 1;
-      for (int k = lane; k < 2 * npg; k += 32) {
-        const int pg = pg0 + (k >> 1);
-        const int r0 = max(pg * kPage, t0), r1 = min(pg * kPage + kPage, tp);
-        const int id = p.ptable[a.i * p.mpps + pg];
-        const size_t off = (((size_t)t.layer * p.num_pages + id) * p.nkv + a.h) * head_stride +
-                           (size_t)(r0 - pg * kPage) * p.hd;
-        const uint32_t nb = (uint32_t)(r1 - r0) * p.hd * 2u;
-        if (k & 1) bulk_g2s(vdst + (size_t)(r0 - t0) * p.hd * 2, p.vpool + off, nb, &sm.full[slot], pol);
-        else bulk_g2s(kdst + (size_t)(r0 - t0) * p.hd * 2, p.kpool + off, nb, &sm.full[slot], pol);
-      }
-    }
-    return true;
-  }
   const int K = gemv_K_dev(p, t.op);
   const int R = t.nunits * rows_per_unit(t.op);
   const int kc0 = s * t.kc;
@@ -385,6 +351,35 @@ __device__ bool issue_weights(const KParams& p, Smem& sm, const TaskDesc& t, con
   __syncwarp();
   for (int c = lane; c < nch; c += 32)
     issue_gemv_chunk(p, t, kc0 + c * kBoxCols, sm.pool[slot] + (size_t)c * R * 128, &sm.full[slot], pol);
+}
+
+// K and V pages of stage k of attention piece a into slot `slot`: whole 16-token pages as
+// tiled boxes (128-byte swizzle; head_dim 128 as [2 halves][16 rows][64]), K pages at the
+// slot's start and V pages at half the slot.  Returns false on a page id out of range.
+__device__ bool issue_kv(const KParams& p, Smem& sm, const TaskDesc& t, const AttnPiece& a, int k, int slot,
+                         uint64_t pol) {
+  const int lane = threadIdx.x & 31;
+  const int T = attn_stage_tokens(p.hd);
+  const int s0 = a.t0 + k * T, s1 = min(s0 + T, a.t1);
+  const int pg0 = s0 / kPage, npg = (s1 - 1) / kPage - pg0 + 1;
+  bool bad = false;
+  for (int q = lane; q < npg; q += 32) {
+    const int id = p.ptable[a.i * p.mpps + pg0 + q];
+    if (id < 0 || id >= p.num_pages) bad = true;
+  }
+  if (__any_sync(0xffffffffu, bad)) return false;
+  const uint32_t page_bytes = (uint32_t)kPage * p.hd * 2u;
+  if (lane == 0) mbar_expect_tx(&sm.full[slot], 2u * npg * page_bytes);
+  __syncwarp();
+  for (int e = lane; e < 2 * npg; e += 32) {
+    const int q = e >> 1;
+    const int id = p.ptable[a.i * p.mpps + pg0 + q];
+    const int row = ((t.layer * p.num_pages + id) * p.nkv + a.h) * kPage;
+    uint8_t* dst = sm.pool[slot] + (size_t)(e & 1) * T * p.hd * 2 + (size_t)q * page_bytes;
+    const void* map = (e & 1) ? (const void*)&p.vmap : (const void*)&p.kmap;
+    if (p.hd == 64) tma_2d(dst, map, 0, row, &sm.full[slot], pol);
+    else tma_3d(dst, map, 0, row, 0, &sm.full[slot], pol);
+  }
   return true;
 }
 
@@ -394,20 +389,32 @@ __device__ bool issue_weights(const KParams& p, Smem& sm, const TaskDesc& t, con
 __device__ void producer(const KParams& p, Smem& sm, const TaskDesc* ts, int nt) {
   const int lane = threadIdx.x & 31;
   const uint64_t pol = policy_evict_first();
+  const int T = attn_stage_tokens(p.hd);
   uint32_t wk = 0;  // stages issued
   bool fail = false;
   for (int wt = 0; wt < nt && !fail; ++wt) {
     const TaskDesc t = ts[wt];
-    AttnWork wa;
-    const int wn = task_stages(p, sm, t, wa);
+    if (t.op == OP_ATTN) {
+      AttnPiece a;
+      for (int j = 0; !fail && attn_piece(p, sm.attn_R, (int)t.u0, j, a); ++j) {
+        const int ns = (a.t1 - a.t0 + T - 1) / T;
+        for (int k = 0; k < ns; ++k, ++wk) {
+          const int slot = wk % kNumSlots;
+          if (!mbar_wait_warp(p, &sm.empty[slot], ((wk / kNumSlots) & 1) ^ 1)) { fail = true; break; }
+          if (!issue_kv(p, sm, t, a, k, slot, pol)) {
+            if (lane == 0) raise_error(p, -6 /* MK_ERR_BOUNDS */);
+            fail = true;
+            break;
+          }
+        }
+      }
+      continue;
+    }
+    const int wn = gemv_stages(p, t);
     for (int ws = 0; ws < wn; ++ws, ++wk) {
       const int slot = wk % kNumSlots;
       if (!mbar_wait_warp(p, &sm.empty[slot], ((wk / kNumSlots) & 1) ^ 1)) { fail = true; break; }
-      if (!issue_weights(p, sm, t, wa, ws, slot, pol)) {
-        if (lane == 0) raise_error(p, -6 /* MK_ERR_BOUNDS */);
-        fail = true;
-        break;
-      }
+      issue_weights(p, sm, t, ws, slot, pol);
     }
   }
   if (fail) {
@@ -794,290 +801,254 @@ __device__ void embed_task(const KParams& p, Smem& sm, const TaskDesc& t, bool a
   }
 }
 
-// One split-K chunk of GQA decode attention for (sequence i, kv head h): QK^T on
-// tensor cores (A = keys from the slot, B = the g query heads as bf16 hi/lo pairs),
-// an online softmax per warp in the log2 domain, PV on CUDA cores, a merge of the
-// eight warps, and - for the last chunk of (i, h) to finish - the log-sum-exp
-// combine of all chunks into the attention output.
+// Byte offset of 16-byte chunk ch (dims 8ch..8ch+7) of token row r (0..15) inside one page
+// block of the pool slot: the box layout [head_dim / 64 halves][16 rows][128 bytes] with the
+// 128-byte swizzle (chunk position ^= row & 7).
+__device__ __forceinline__ uint32_t kv_off(int r, int ch) {
+  return (uint32_t)((((ch >> 3) << 4) + r) << 7) + (uint32_t)(((ch & 7) ^ (r & 7)) << 4);
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr)
+               : "memory");
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr)
+               : "memory");
+}
+__device__ __forceinline__ uint32_t split_pair(float x, float y, bool lo) {
+  const float hx = __bfloat162float(__float2bfloat16_rn(x)), hy = __bfloat162float(__float2bfloat16_rn(y));
+  return lo ? pack_bf16(x - hx, y - hy) : pack_bf16(hx, hy);
+}
+
+// One attention range (its pieces in turn) of GQA decode attention, flash-decode style, all
+// products on tensor cores.  Per piece = (sequence i, kv head h, tokens [t0, t1)):
+//   * each warp owns 16-token groups of the stages it takes (head_dim 64: all warps every
+//     stage; head_dim 128: warps 0-3 even stages, 4-7 odd ones);
+//   * S = Q K^T with A = the g query heads (rows 0-7 bf16 hi parts, rows 8-15 the lo
+//     remainders, so q keeps ~16 mantissa bits) and B = K rows by ldmatrix;
+//   * online softmax in the log2 domain, the row max shared by the 4 lanes of a row;
+//   * O += P V with A = P split the same way into hi/lo rows and B = V by ldmatrix.trans;
+//   * the 8 warps' (m, l, O) merge in shared memory into one log-sum-exp partial; the last
+//     piece of (i, h) to finish combines all its pieces into the O-projection operand.
 template <int HD>
 __device__ __noinline__ void attn_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_t& stage, bool& ab) {
-  constexpr int T = HD == 64 ? 128 : 64;   // tokens per stage
-  constexpr int TPW = T / kConsumerWarps;  // tokens per warp per stage: 16 or 8
-  constexpr int NKB = HD / 32;             // 32-dim blocks
-  constexpr int DPL = HD / 32;             // dims per lane in PV
-  constexpr int NT = HD == 64 ? 2 : 1;     // n-tiles of 4 heads
+  constexpr int T = HD == 64 ? 128 : 64;      // tokens per stage (K then V: 32 KB)
+  constexpr int WPS = T / 16;                 // warps per stage, one 16-token group each
+  constexpr int NG = kConsumerWarps / WPS;    // stages in flight across warp groups
+  constexpr int NK = HD / 16;                 // k steps of Q K^T
+  constexpr int NN = HD / 8;                  // n tiles of P V
+  constexpr int PAGE = kPage * HD * 2;        // bytes of one page block
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g_ = lane >> 2, tq = lane & 3;
-  AttnWork a;
-  const bool has = (int)t.u0 < sm.attn_n && attn_work(p, sm.attn_ch, (int)t.u0, a);
-  if (!has) return;  // empty slot: no stages, nothing to merge
+  const int grp = warp % WPS, wsel = warp / WPS;
   const int G = p.g;
-  const int newpos = a.n - 1;
   const float sc = 1.4426950408889634f / sqrtf((float)HD);
+  const bool tr = p.trace && threadIdx.x == 0;
+  uint32_t ks = 0;  // stage count within the task: picks the warp group
+  AttnPiece a;
+  for (int j = 0; attn_piece(p, sm.attn_R, (int)t.u0, j, a); ++j) {
+    const unsigned long long tc0 = tr ? gtimer() : 0ull;
+    const unsigned long long wait0 = tr ? sm.wait_ns : 0ull;
+    // Q fragments of head g_ of this kv group
+    uint32_t qa[NK][4];
+    {
+      const bool hv = g_ < G && !ab;
+      const float* qs = p.q + (size_t)a.i * p.qdim + (size_t)(a.h * G + (hv ? g_ : 0)) * HD + 2 * tq;
+#pragma unroll
+      for (int kk = 0; kk < NK; ++kk) {
+        float2 v0 = make_float2(0.f, 0.f), v1 = make_float2(0.f, 0.f);
+        if (hv) {
+          v0 = __ldcg(reinterpret_cast<const float2*>(qs + 16 * kk));
+          v1 = __ldcg(reinterpret_cast<const float2*>(qs + 16 * kk + 8));
+        }
+        qa[kk][0] = split_pair(v0.x, v0.y, false);
+        qa[kk][1] = split_pair(v0.x, v0.y, true);
+        qa[kk][2] = split_pair(v1.x, v1.y, false);
+        qa[kk][3] = split_pair(v1.x, v1.y, true);
+      }
+    }
+    float m_run = -INFINITY, l_run = 0.f;
+    float o[NN][4];
+#pragma unroll
+    for (int n = 0; n < NN; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    const int newpos = a.n - 1;
+    const int ns = (a.t1 - a.t0 + T - 1) / T;
+    for (int k = 0; k < ns; ++k, ++stage, ++ks) {
+      const int slot = stage % kNumSlots;
+      if (!ab) ab = !mbar_wait_warp(p, &sm.full[slot], (stage / kNumSlots) & 1, tr ? &sm.wait_ns : nullptr);
+      const int g0 = a.t0 + k * T + 16 * grp;  // first token of this warp's group
+      const int nv = min(16, a.t1 - g0);        // valid tokens in the group (<= 0: none)
+      if (!ab && (int)(ks % NG) == wsel && nv > 0) {
+        uint8_t* kpg = sm.pool[slot] + grp * PAGE;
+        uint8_t* vpg = sm.pool[slot] + T * HD * 2 + grp * PAGE;
+        bool wrote = false;
+        if (newpos >= g0 && newpos < g0 + 16) {
+          // the new token's K/V, written by this layer's QKV tasks after the page was fetched
+          const int r = newpos - g0;
+          const int page = p.ptable[a.i * p.mpps + newpos / kPage];
+          const size_t off = ((((size_t)t.layer * p.num_pages + page) * p.nkv + a.h) * kPage + r) * HD;
+          constexpr int CH = HD / 8;
+          if (lane < 2 * CH) {
+            const int ch = lane % CH;
+            const uint4 v = __ldcg(reinterpret_cast<const uint4*>((lane < CH ? p.kpool : p.vpool) + off + ch * 8));
+            *reinterpret_cast<uint4*>((lane < CH ? kpg : vpg) + kv_off(r, ch)) = v;
+          }
+          wrote = true;
+        }
+        if (nv < 16) {
+          // rows past the sequence's end hold whatever the page held: zero their V (P is 0 there)
+          for (int e = lane; e < (16 - nv) * (HD / 8); e += 32)
+            *reinterpret_cast<uint4*>(vpg + kv_off(nv + e / (HD / 8), e % (HD / 8))) = make_uint4(0, 0, 0, 0);
+          wrote = true;
+        }
+        if (wrote) {
+          fence_proxy_async_smem();  // the slot is refilled by the async proxy later
+          __syncwarp();
+        }
+        // S = Q K^T: n tile 0 = tokens 0..7, n tile 1 = tokens 8..15 of the group
+        float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+        const uint32_t kb = smem_u32(kpg), vb = smem_u32(vpg);
+        const int mi = lane >> 3, rr = lane & 7;
+#pragma unroll
+        for (int kk = 0; kk < NK; ++kk) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(kb + kv_off(((mi >> 1) << 3) + rr, 2 * kk + (mi & 1)), b0, b1, b2, b3);
+          mma_bf16(s0, qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b0, b1);
+          mma_bf16(s1, qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b2, b3);
+        }
+        // this lane's scores of head g_: tokens 2tq, 2tq+1, 8+2tq, 9+2tq (hi row + lo row)
+        float sv[4] = {(s0[0] + s0[2]) * sc, (s0[1] + s0[3]) * sc, (s1[0] + s1[2]) * sc, (s1[1] + s1[3]) * sc};
+        if (2 * tq >= nv) sv[0] = -INFINITY;
+        if (2 * tq + 1 >= nv) sv[1] = -INFINITY;
+        if (8 + 2 * tq >= nv) sv[2] = -INFINITY;
+        if (9 + 2 * tq >= nv) sv[3] = -INFINITY;
+        float mx = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        const float mn = fmaxf(m_run, mx);  // finite: token 0 of the group is valid
+        const float corr = exp2f(m_run - mn);
+        float pr[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) pr[e] = exp2f(sv[e] - mn);
+        l_run = l_run * corr + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
+        m_run = mn;
+#pragma unroll
+        for (int n = 0; n < NN; ++n) {
+          o[n][0] *= corr;
+          o[n][1] *= corr;
+          o[n][2] *= corr;
+          o[n][3] *= corr;
+        }
+        const uint32_t pa0 = split_pair(pr[0], pr[1], false), pa1 = split_pair(pr[0], pr[1], true);
+        const uint32_t pa2 = split_pair(pr[2], pr[3], false), pa3 = split_pair(pr[2], pr[3], true);
+        // O += P V: B = V rows (k = the 16 tokens) transposed by ldmatrix
+#pragma unroll
+        for (int nn = 0; nn < NN / 2; ++nn) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(vb + kv_off(((mi & 1) << 3) + rr, 2 * nn + (mi >> 1)), b0, b1, b2, b3);
+          mma_bf16(o[2 * nn], pa0, pa1, pa2, pa3, b0, b1);
+          mma_bf16(o[2 * nn + 1], pa0, pa1, pa2, pa3, b2, b3);
+        }
+      }
+      __syncwarp();
+      if (!ab && lane == 0) mbar_arrive(&sm.empty[slot]);
+    }
 
-  // q fragments (B operand): column g_ = head (g_ & 3) of the n-tile, part g_ >> 2 (hi, lo)
-  uint32_t qf[NT][NKB][4];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    const int hq = nt * 4 + (g_ & 3);
-    const bool lo = g_ >= 4;
-#pragma unroll
-    for (int kb = 0; kb < NKB; ++kb) {
-      float v[8];
-      if (hq < G && !ab) {
-        const float* qs = p.q + (size_t)a.i * p.qdim + (size_t)(a.h * G + hq) * HD + kb * 32 + tq * 8;
-        const float4 v0 = __ldcg(reinterpret_cast<const float4*>(qs));
-        const float4 v1 = __ldcg(reinterpret_cast<const float4*>(qs + 4));
-        v[0] = v0.x; v[1] = v0.y; v[2] = v0.z; v[3] = v0.w; v[4] = v1.x; v[5] = v1.y; v[6] = v1.z; v[7] = v1.w;
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] = 0.f;
-      }
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float hi = __bfloat162float(__float2bfloat16_rn(v[e]));
-        v[e] = lo ? v[e] - hi : hi;
-      }
-      qf[nt][kb][0] = pack_bf16(v[0], v[1]);
-      qf[nt][kb][1] = pack_bf16(v[2], v[3]);
-      qf[nt][kb][2] = pack_bf16(v[4], v[5]);
-      qf[nt][kb][3] = pack_bf16(v[6], v[7]);
+    unsigned long long tr0 = 0;
+    if (tr) {
+      tr0 = gtimer();
+      sm.tm[0] += tr0 - tc0 - (sm.wait_ns - wait0);
     }
-  }
-
-  float m_st[NT][2], l_st[NT][2];
+    // this warp's state of head g_: l summed over the row's 4 lanes, O = hi row + lo row
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+    if (!ab && g_ < G) {
+      float* rw = sm.red + (warp * G + g_) * HD + 2 * tq;
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    m_st[nt][0] = m_st[nt][1] = -INFINITY;
-    l_st[nt][0] = l_st[nt][1] = 0.f;
-  }
-  float acc[8][DPL];
-#pragma unroll
-  for (int h = 0; h < 8; ++h)
-#pragma unroll
-    for (int e = 0; e < DPL; ++e) acc[h][e] = 0.f;
-
-  const int nst = attn_stages(a, T);
-  const unsigned long long tc0 = (p.trace && threadIdx.x == 0) ? gtimer() : 0ull;
-  for (int s = 0; s < nst; ++s, ++stage) {
-    const int slot = stage % kNumSlots;
-    const int t0 = a.c0 + s * T, t1 = min(t0 + T, a.c1);
-    const int ntok = t1 - t0;
-    const bool has_new = newpos >= t0 && newpos < t1;
-    if (!ab) ab = !mbar_wait_warp(p, &sm.full[slot], (stage / kNumSlots) & 1,
-                                  (p.trace && threadIdx.x == 0) ? &sm.wait_ns : nullptr);
-    uint8_t* kreg = sm.pool[slot];
-    uint8_t* vreg = sm.pool[slot] + (size_t)T * HD * 2;
-    if (has_new) {
-      // the new token's K/V were written by this layer's QKV tasks: read them now
-      if (warp == 0 && !ab) {
-        const int page = p.ptable[a.i * p.mpps + newpos / kPage];
-        const size_t off = ((((size_t)t.layer * p.num_pages + page) * p.nkv + a.h) * kPage + newpos % kPage) * HD;
-        constexpr int CH = HD * 2 / 16;  // 16-byte chunks per row
-        if (lane < 2 * CH) {
-          const int c = lane % CH;
-          const bf16* srcp = (lane < CH ? p.kpool : p.vpool) + off + c * 8;
-          const uint4 v = __ldcg(reinterpret_cast<const uint4*>(srcp));
-          uint8_t* dst = (lane < CH ? kreg : vreg) + (size_t)(newpos - t0) * HD * 2 + c * 16;
-          *reinterpret_cast<uint4*>(dst) = v;
-        }
-        fence_proxy_async_smem();
+      for (int n = 0; n < NN; ++n)
+        *reinterpret_cast<float2*>(rw + 8 * n) = make_float2(o[n][0] + o[n][2], o[n][1] + o[n][3]);
+      if (tq == 0) {
+        sm.mw[warp][g_] = m_run;
+        sm.lw[warp][g_] = l_run;
       }
-      cbar();
-    }
-    if (!ab) {
-      const int tokA = warp * TPW + g_;
-      const int tokB = warp * TPW + 8 + g_;
-      const bool vA = tokA < ntok;
-      const bool vB = TPW == 16 && tokB < ntok;
-      const int nw = max(0, min(TPW, ntok - warp * TPW));  // this warp's tokens
-      if (nw > 0) {
-        float sacc[NT][4];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
-#pragma unroll
-        for (int kb = 0; kb < NKB; ++kb) {
-          uint4 ka = make_uint4(0, 0, 0, 0), kbv = make_uint4(0, 0, 0, 0);
-          if (vA) ka = *reinterpret_cast<const uint4*>(kreg + (size_t)tokA * HD * 2 + kb * 64 + tq * 16);
-          if (vB) kbv = *reinterpret_cast<const uint4*>(kreg + (size_t)tokB * HD * 2 + kb * 64 + tq * 16);
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            mma_bf16(sacc[nt], ka.x, kbv.x, ka.y, kbv.y, qf[nt][kb][0], qf[nt][kb][1]);
-            mma_bf16(sacc[nt], ka.z, kbv.z, ka.w, kbv.w, qf[nt][kb][2], qf[nt][kb][3]);
-          }
-        }
-        // scores: lanes tq<2 hold hi columns, tq>=2 the lo columns of the same heads
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          float sv[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) sv[e] = sacc[nt][e] + __shfl_xor_sync(0xffffffffu, sacc[nt][e], 2);
-#pragma unroll
-          for (int hs = 0; hs < 2; ++hs) {
-            const int hq = nt * 4 + 2 * (tq & 1) + hs;
-            const bool hv = hq < G;
-            float sA = (vA && hv) ? sv[hs] * sc : -INFINITY;
-            float sB = (vB && hv) ? sv[2 + hs] * sc : -INFINITY;
-            float mx = fmaxf(sA, sB);
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-            const float mo = m_st[nt][hs];
-            const float mn = fmaxf(mo, mx);
-            float corr = 1.f, pA = 0.f, pB = 0.f;
-            if (mn != -INFINITY) {
-              corr = exp2f(mo - mn);
-              pA = exp2f(sA - mn);
-              pB = exp2f(sB - mn);
-            }
-            float ls = pA + pB;
-            ls += __shfl_xor_sync(0xffffffffu, ls, 4);
-            ls += __shfl_xor_sync(0xffffffffu, ls, 8);
-            ls += __shfl_xor_sync(0xffffffffu, ls, 16);
-            m_st[nt][hs] = mn;
-            l_st[nt][hs] = l_st[nt][hs] * corr + ls;
-            if (tq < 2 && hq < 8) {
-              sm.pw[warp][g_ * 8 + hq] = pA;
-              if (TPW == 16) sm.pw[warp][(8 + g_) * 8 + hq] = pB;
-              if (g_ == 0) sm.corr[warp][hq] = corr;
-            }
-          }
-        }
-        __syncwarp();
-        // PV: lane owns dims lane*DPL .. +DPL-1
-#pragma unroll
-        for (int h = 0; h < 8; ++h) {
-          if (h < G) {
-            const float c = sm.corr[warp][h];
-#pragma unroll
-            for (int e = 0; e < DPL; ++e) acc[h][e] *= c;
-          }
-        }
-        for (int tk = 0; tk < nw; ++tk) {
-          const uint8_t* vr = vreg + (size_t)(warp * TPW + tk) * HD * 2 + lane * DPL * 2;
-          float vv[DPL];
-          if constexpr (DPL == 4) {
-            const uint2 u = *reinterpret_cast<const uint2*>(vr);
-            vv[0] = bf_lo(u.x); vv[1] = bf_hi(u.x); vv[2] = bf_lo(u.y); vv[3] = bf_hi(u.y);
-          } else {
-            const uint32_t u = *reinterpret_cast<const uint32_t*>(vr);
-            vv[0] = bf_lo(u); vv[1] = bf_hi(u);
-          }
-          const float4 p0 = *reinterpret_cast<const float4*>(&sm.pw[warp][tk * 8]);
-          const float4 p1 = *reinterpret_cast<const float4*>(&sm.pw[warp][tk * 8 + 4]);
-          const float pr[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-#pragma unroll
-          for (int h = 0; h < 8; ++h) {
-            if (h < G) {
-#pragma unroll
-              for (int e = 0; e < DPL; ++e) acc[h][e] = fmaf(pr[h], vv[e], acc[h][e]);
-            }
-          }
-        }
-        __syncwarp();
-      }
-    }
-    __syncwarp();
-    if (!ab && lane == 0) mbar_arrive(&sm.empty[slot]);
-  }
-
-  unsigned long long tr0 = 0;
-  if (p.trace && threadIdx.x == 0) {
-    tr0 = gtimer();
-    sm.tm[0] += tr0 - tc0 - sm.wait_ns;
-  }
-  // merge the eight warps' (m, l, acc) states: red[warp][head][HD]
-  if (!ab) {
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int hs = 0; hs < 2; ++hs) {
-        const int hq = nt * 4 + 2 * (tq & 1) + hs;
-        if (g_ == 0 && tq < 2 && hq < 8) {
-          sm.mw[warp][hq] = m_st[nt][hs];
-          sm.lw[warp][hq] = l_st[nt][hs];
-        }
-      }
-#pragma unroll
-    for (int h = 0; h < 8; ++h)
-      if (h < G)
-#pragma unroll
-        for (int e = 0; e < DPL; ++e) sm.red[(warp * G + h) * HD + lane * DPL + e] = acc[h][e];
-  }
-  cbar();
-  float* part = p.part + (size_t)t.u0 * G * (HD + 2);
-  if (!ab) {
-    for (int idx = threadIdx.x; idx < G * HD; idx += kConsumerWarps * 32) {
-      const int h = idx / HD, dd = idx % HD;
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm.mw[w][h]);
-      float A = 0.f, Ls = 0.f;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) {
-        const float f = sm.mw[w][h] == -INFINITY ? 0.f : exp2f(sm.mw[w][h] - M);
-        A += f * sm.red[(w * G + h) * HD + dd];
-        Ls += f * sm.lw[w][h];
-      }
-      part[h * (HD + 2) + dd] = A;
-      if (dd == 0) {
-        part[h * (HD + 2) + HD] = M;
-        part[h * (HD + 2) + HD + 1] = Ls;
-      }
-    }
-  }
-  cbar();
-  const unsigned long long te0 = (p.trace && threadIdx.x == 0) ? gtimer() : 0ull;
-  if (p.trace && threadIdx.x == 0) sm.tm[1] += te0 - tr0;
-  if (threadIdx.x == 0) {
-    int last = 0;
-    if (!ab) {
-      uint32_t* cc = p.cmb + ((size_t)t.layer * p.max_b + a.i) * p.nkv + a.h;
-      const uint32_t old = atom_add_acqrel(cc, 1u);
-      last = (old + 1u == (uint32_t)a.nc) ? 1 : 0;
-      if (last) *cc = 0u;  // ready for the next step (every chunk of (i, h) has arrived)
-    }
-    sm.flag2 = last;
-  }
-  cbar();
-  if (sm.flag2) {
-    // log-sum-exp combine of the nc (<= 32) chunk states of (i, h): one warp per head
-    // computes the chunk weights 2^(m_c - M) / sum_c 2^(m_c - M) l_c from all chunks at
-    // once, then every thread sums weighted partials with independent loads.
-    const float* base = p.part + (size_t)(t.u0 - a.c) * G * (HD + 2);
-    float* wts = sm.red;  // [head][32]
-    const int warp = threadIdx.x >> 5;
-    for (int h = warp; h < G; h += kConsumerWarps) {
-      const float* pc = base + ((size_t)lane * G + h) * (HD + 2);
-      const float mc = lane < a.nc ? __ldcg(pc + HD) : -INFINITY;
-      const float lc = lane < a.nc ? __ldcg(pc + HD + 1) : 0.f;
-      float M = mc;
-#pragma unroll
-      for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-      const float f = lane < a.nc ? exp2f(mc - M) : 0.f;
-      float den = f * lc;
-#pragma unroll
-      for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-      wts[h * 32 + lane] = f / den;
     }
     cbar();
-    for (int idx = threadIdx.x; idx < G * HD; idx += kConsumerWarps * 32) {
-      const int h = idx / HD, dd = idx % HD;
-      const float* pc = base + (size_t)h * (HD + 2) + dd;
-      const size_t cs = (size_t)G * (HD + 2);
-      float acc0 = 0.f, acc1 = 0.f;
-      int c = 0;
-      for (; c + 1 < a.nc; c += 2) {
-        acc0 = fmaf(wts[h * 32 + c], __ldcg(pc + c * cs), acc0);
-        acc1 = fmaf(wts[h * 32 + c + 1], __ldcg(pc + (c + 1) * cs), acc1);
+    const size_t pst = (size_t)G * (HD + 2);  // floats per piece partial
+    float* pbase = p.part + ((size_t)a.i * p.nkv + a.h) * kMaxChunksPerSeq * pst;
+    if (!ab) {
+      float* part = pbase + (size_t)a.c * pst;
+      for (int idx = threadIdx.x; idx < G * HD; idx += kConsumerWarps * 32) {
+        const int h = idx / HD, dd = idx % HD;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm.mw[w][h]);
+        float A = 0.f, Ls = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          const float f = sm.mw[w][h] == -INFINITY ? 0.f : exp2f(sm.mw[w][h] - M);
+          A += f * sm.red[(w * G + h) * HD + dd];
+          Ls += f * sm.lw[w][h];
+        }
+        part[h * (HD + 2) + dd] = A;
+        if (dd == 0) {
+          part[h * (HD + 2) + HD] = M;
+          part[h * (HD + 2) + HD + 1] = Ls;
+        }
       }
-      if (c < a.nc) acc0 = fmaf(wts[h * 32 + c], __ldcg(pc + c * cs), acc0);
-      put_operand(p.aa_t, p.aa_f, p.ld_a, a.i, (a.h * G + h) * HD + dd, acc0 + acc1);
     }
+    cbar();
+    const unsigned long long te0 = tr ? gtimer() : 0ull;
+    if (tr) sm.tm[1] += te0 - tr0;
+    if (threadIdx.x == 0) {
+      int last = 0;
+      if (!ab) {
+        uint32_t* cc = p.cmb + ((size_t)t.layer * p.max_b + a.i) * p.nkv + a.h;
+        const uint32_t old = atom_add_acqrel(cc, 1u);
+        last = (old + 1u == (uint32_t)a.nc) ? 1 : 0;
+        if (last) *cc = 0u;  // ready for the next step (every piece of (i, h) has arrived)
+      }
+      sm.flag2 = last;
+    }
+    cbar();
+    if (sm.flag2) {
+      // log-sum-exp combine of the nc (<= 32) piece states of (i, h): one warp per head
+      // computes the weights 2^(m_c - M) / sum_c 2^(m_c - M) l_c of all pieces at once,
+      // then every thread sums weighted partials with independent loads.
+      float* wts = sm.red;  // [head][32]
+      for (int h = warp; h < G; h += kConsumerWarps) {
+        const float* pc = pbase + ((size_t)lane * G + h) * (HD + 2);
+        const float mc = lane < a.nc ? __ldcg(pc + HD) : -INFINITY;
+        const float lc = lane < a.nc ? __ldcg(pc + HD + 1) : 0.f;
+        float M = mc;
+#pragma unroll
+        for (int o2 = 16; o2; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o2));
+        const float f = lane < a.nc ? exp2f(mc - M) : 0.f;
+        float den = f * lc;
+#pragma unroll
+        for (int o2 = 16; o2; o2 >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o2);
+        wts[h * 32 + lane] = f / den;
+      }
+      cbar();
+      for (int idx = threadIdx.x; idx < G * HD; idx += kConsumerWarps * 32) {
+        const int h = idx / HD, dd = idx % HD;
+        const float* pc = pbase + (size_t)h * (HD + 2) + dd;
+        float acc0 = 0.f, acc1 = 0.f;
+        int c = 0;
+        for (; c + 1 < a.nc; c += 2) {
+          acc0 = fmaf(wts[h * 32 + c], __ldcg(pc + c * pst), acc0);
+          acc1 = fmaf(wts[h * 32 + c + 1], __ldcg(pc + (c + 1) * pst), acc1);
+        }
+        if (c < a.nc) acc0 = fmaf(wts[h * 32 + c], __ldcg(pc + c * pst), acc0);
+        put_operand(p.aa_t, p.aa_f, p.ld_a, a.i, (a.h * G + h) * HD + dd, acc0 + acc1);
+      }
+    }
+    cbar();  // sm.red is reused by the next piece
+    if (tr) sm.tm[2] += gtimer() - te0;
   }
-  if (p.trace && threadIdx.x == 0) sm.tm[2] += gtimer() - te0;
 }
 
 // ---------------------------------------------------------------------------------------
@@ -1197,7 +1168,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
     if (bad) raise_error(p, -6 /* MK_ERR_BOUNDS */);
     sm.bad = bad;
     sm.inv_inst = -1;
-    if (!bad) attn_setup(p, &sm.attn_ch, &sm.attn_n);
+    if (!bad) sm.attn_R = attn_setup(p);
   }
   __syncthreads();
   if (sm.bad) return;

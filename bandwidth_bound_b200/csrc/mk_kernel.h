@@ -17,6 +17,9 @@ struct alignas(64) TmaDesc {  // the driver's opaque 128-byte TMA descriptor (CU
 };
 
 struct KParams {
+  // this step's KV pools as tiled maps (16-token page boxes, 128-byte swizzle), encoded by
+  // the host when the pools change
+  TmaDesc kmap, vmap;
   // model shape
   int L, d, nq, nkv, hd, F, V, g, qdim, max_b, max_ctx;
   float eps;
@@ -28,7 +31,8 @@ struct KParams {
   int num_sms, n_slots, n_lm_tasks;
   const void* tmaps;          // CUtensorMap array: weights (tmap_index) then the LM head
   // handle-owned device state
-  float *x, *q, *ssq, *part;
+  float *x, *q, *ssq;
+  float* part;               // split-K partials [max_b * nkv][kMaxChunksPerSeq][g][hd + 2]
   // GEMV operands, written once by the producing phase: bf16 hi/lo tiles in the layout of
   // operand_index (all batch rows) and fp32 (batch row 0, for the batch-1 path).
   // ax: x * gain of the next RMSNorm (input of qkv / gate-up / lm head), aa: attention output,

@@ -152,15 +152,12 @@ int build_plan(const mk_model_cfg& c, const mk_plan_opts* opts, mk_plan_s* P, st
   const Geometry G = geometry(c);
   P->cfg = c;
   P->num_sms = (opts && opts->num_sms > 0) ? opts->num_sms : 148;
-  P->attn_slots_per_sm = (opts && opts->attn_slots_per_sm > 0) ? opts->attn_slots_per_sm : 4;
+  P->attn_slots_per_sm = (opts && opts->attn_slots_per_sm > 0) ? opts->attn_slots_per_sm : 1;
   P->max_blocks = (opts && opts->max_blocks > 0) ? opts->max_blocks : kMaxBlocks;
   if (P->num_sms > 4096 || P->attn_slots_per_sm > 64 || P->max_blocks > kMaxBlocks) {
     set_err(err, "plan options out of range");
     return MK_ERR_INVALID_ARG;
   }
-  // every (sequence, kv head) needs at least one split-K slot
-  const int need = (c.max_batch * G.nkv + P->num_sms - 1) / P->num_sms;
-  if (P->attn_slots_per_sm < need) P->attn_slots_per_sm = need;
   const int S = P->num_sms * P->attn_slots_per_sm;
   if (S > 65535) { set_err(err, "too many attention slots"); return MK_ERR_INVALID_ARG; }
   const int nsm = P->num_sms;

@@ -96,7 +96,7 @@ typedef struct mk_plan_s *mk_plan_t;
 /* Options of the per-SM task schedule (zero fields take the defaults). */
 typedef struct mk_plan_opts {
   int32_t num_sms;           /* CTAs = SMs of the device (default: queried; host-only plans: 148) */
-  int32_t attn_slots_per_sm; /* split-K attention slots per SM and layer (default 4) */
+  int32_t attn_slots_per_sm; /* attention ranges (split-K work items) per SM and layer (default 1) */
   int32_t max_blocks;        /* 8-row blocks per GEMV task, 1..8 (default 8) */
 } mk_plan_opts;
 
