@@ -38,8 +38,8 @@ struct Smem {
   alignas(8) uint64_t full[kNumSlots];                   // weight/KV bytes of the stage landed
   alignas(8) uint64_t empty[kNumSlots];                  // all consumer warps done with the stage
   int attn_R, bad, flag, flag2;  // attn_R: tokens per attention range (this step)
-  unsigned long long wait_ns;  // time warp 0 spent waiting for pool slots in the current task (tracing)
-  unsigned long long tm[3];    // tracing: compute, reduce, epilogue ns of the current task (warp 0)
+  unsigned long long wait_cyc;  // tracing: SM cycles warp 0 spent waiting for pool slots in the current task
+  unsigned long long tm[3];     // tracing: compute, reduce, epilogue SM cycles of the current task (warp 0)
   int inv_inst;                // ssq instance whose 1/rms sm.inv_rms holds (-1: none)
 };
 
@@ -200,9 +200,9 @@ __device__ __forceinline__ bool mbar_wait_warp(const KParams& p, uint64_t* bar, 
   int ok = 0;
   if ((threadIdx.x & 31) == 0) {
     if (wait_acc && !mbar_test(bar, parity)) {
-      const uint64_t t0 = gtimer();
+      const long long c0 = clock64();
       ok = mbar_wait(p, bar, parity) ? 1 : 0;
-      *wait_acc += gtimer() - t0;
+      *wait_acc += (unsigned long long)(clock64() - c0);
     } else {
       ok = mbar_wait(p, bar, parity) ? 1 : 0;
     }
@@ -465,19 +465,19 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// Copy this lane's operand of column group kg (8 columns) into ring entry e of its warp:
-// MT tiles of (hi, lo) 16-byte rows (batch row 8mt + g; zeros past the batch), or the 8 fp32
-// values of batch row 0 (MT == 0).  Lane-private 16-byte pieces: entry e, piece q at
-// ((e * 2 * NMT + q) * 32 + lane) * 16.
+// Copy the operand of column group kg (8 columns) of this lane into ring entry e of its
+// warp.  MT >= 1: MT tiles of (hi, lo) 16-byte rows (batch row 8mt + g; zeros past the
+// batch), lane-private pieces: entry e, piece q at ((e * 2 * MT + q) * 32 + lane) * 16.
+// MT == 0: the 8 fp32 values of batch row 0, shared by the 8 lanes (g = 0..7) of one tq:
+// lanes g = 0, 1 copy one half each to entry e at (e * 4 + tq) * 32 + g * 16, so that
+// every column group is read from L2 once per warp.
 template <int MT>
 __device__ __forceinline__ void fetch_opnd(const KParams& p, uint8_t* ring, int e, const bf16* tiles, const float* f,
                                            int ld, int kg, int g, int lane) {
-  constexpr int NQ = MT == 0 ? 2 : 2 * MT;
-  uint8_t* base = ring + (size_t)e * NQ * 512 + lane * 16;
   if constexpr (MT == 0) {
-    cp_async16(base, f + 8 * kg, true);
-    cp_async16(base + 512, f + 8 * kg + 4, true);
+    if (g < 2) cp_async16(ring + ((size_t)e * 4 + (lane & 3)) * 32 + g * 16, f + 8 * kg + 4 * g, true);
   } else {
+    uint8_t* base = ring + (size_t)e * 2 * MT * 512 + lane * 16;
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
       const bool v = mt * 8 + g < p.b;
@@ -492,15 +492,17 @@ __device__ __forceinline__ void fetch_opnd(const KParams& p, uint8_t* ring, int 
 // swizzled (chunk c of row r at c ^ (r & 7)).  Warp w takes 32-column k blocks w, w+8,
 // ... of every stage; a k block is the even (h = 0) or odd (h = 1) 16-byte chunks of a
 // 64-column chunk, so lane (g, tq) reads chunk 2*tq + h of row 8j + g - conflict-free -
-// which holds columns 16*tq + 8*h .. +7, column group kg = 8*chunk + 2*tq + h.  The lane
-// loads the operand of that group itself, D blocks ahead of its use (a register ring),
-// so the L2 latency overlaps the earlier blocks' work.  MT = 0: CUDA-core FMA (batch 1);
+// which holds columns 16*tq + 8*h .. +7, column group kg = 8*chunk + 2*tq + h.  The
+// operand of that group is copied (cp.async) into the warp's shared-memory ring Q - 1
+// blocks ahead of its use, so the L2 latency overlaps the earlier blocks' work.  MT = 0:
+// CUDA-core FMA (batch 1);
 // MT = 1, 2: mma.sync with MT tiles of 8 batch rows, rows 0-7 of the M = 16 tile the bf16
 // hi parts, rows 8-15 the lo parts.
 template <int MT, int G>
 __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDesc t, uint32_t& stage, bool& ab) {
   constexpr int NQ = MT == 0 ? 2 : 2 * MT;       // 16-byte pieces per lane and k block
-  constexpr int Q = kRingBytes / (NQ * 512);     // ring entries: 4 (batch <= 8) or 2 (batch > 8)
+  // ring entries: 16 of 128 bytes (batch 1), 4 of 1 KB (batch <= 8) or 2 of 2 KB (batch > 8)
+  constexpr int Q = MT == 0 ? 16 : kRingBytes / (NQ * 512);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, tq = lane & 3;
   const int K = gemv_K_dev(p, t.op);
@@ -544,23 +546,31 @@ __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDes
   for (int s = 0; s < nst; ++s, ++stage) {
     const int slot = stage % kNumSlots;
     const uint32_t par = (stage / kNumSlots) & 1;
-    if (!ab) ab = !mbar_wait_warp(p, &sm.full[slot], par, (p.trace && threadIdx.x == 0) ? &sm.wait_ns : nullptr);
+    if (!ab) ab = !mbar_wait_warp(p, &sm.full[slot], par, (p.trace && threadIdx.x == 0) ? &sm.wait_cyc : nullptr);
     if (ab) continue;
-    const unsigned long long tc0 = (p.trace && threadIdx.x == 0) ? gtimer() : 0ull;
+    const long long tc0 = (p.trace && threadIdx.x == 0) ? clock64() : 0ll;
     const uint8_t* tile = sm.pool[slot];
     const int nb = nblk(s);
     for (int kb = warp; kb < nb; kb += kConsumerWarps) {
+      if constexpr (MT == 0) __syncwarp();  // every lane has read the entry the next copy overwrites
       if (ps < nst) fetch_opnd<MT>(p, ring, fetched % Q, tiles, fop, ld, kgroup(ps, pkb), g, lane);
       cp_async_commit();
       ++fetched;
       advance(ps, pkb);
       cp_async_wait<Q - 1>();  // the group of block `used` has landed
       const uint8_t* chunk = tile + (size_t)(kb >> 1) * (R * 128) + ((((2 * tq + (kb & 1)) ^ g)) << 4);
-      const uint8_t* ab_ = ring + (size_t)(used % Q) * NQ * 512 + lane * 16;
-      ++used;
       uint4 A[NQ];
+      if constexpr (MT == 0) {
+        __syncwarp();  // lanes g = 0, 1 copied what all 8 lanes of their tq read
+        const uint8_t* ab_ = ring + ((size_t)(used % Q) * 4 + tq) * 32;
+        A[0] = *reinterpret_cast<const uint4*>(ab_);
+        A[1] = *reinterpret_cast<const uint4*>(ab_ + 16);
+      } else {
+        const uint8_t* ab_ = ring + (size_t)(used % Q) * NQ * 512 + lane * 16;
 #pragma unroll
-      for (int q = 0; q < NQ; ++q) A[q] = *reinterpret_cast<const uint4*>(ab_ + q * 512);
+        for (int q = 0; q < NQ; ++q) A[q] = *reinterpret_cast<const uint4*>(ab_ + q * 512);
+      }
+      ++used;
 #pragma unroll
       for (int j = 0; j < G; ++j) {
         const uint4 w = *reinterpret_cast<const uint4*>(chunk + (8 * j + g) * 128);
@@ -583,12 +593,12 @@ __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDes
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.empty[slot]);
-    if (p.trace && threadIdx.x == 0) sm.tm[0] += gtimer() - tc0;
+    if (p.trace && threadIdx.x == 0) sm.tm[0] += (unsigned long long)(clock64() - tc0);
   }
 
   cp_async_wait<0>();  // no copy into the ring may be in flight past this task
   // cross-warp reduction, one 8-row batch tile at a time: red[warp][block][batch g][8 rows]
-  const unsigned long long tr0 = (p.trace && threadIdx.x == 0) ? gtimer() : 0ull;
+  const long long tr0 = (p.trace && threadIdx.x == 0) ? clock64() : 0ll;
   float* red = sm.red;
 #pragma unroll
   for (int mt = 0; mt < NMT; ++mt) {
@@ -620,7 +630,7 @@ __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDes
     }
     cbar();
   }
-  if (p.trace && threadIdx.x == 0) sm.tm[1] += gtimer() - tr0;
+  if (p.trace && threadIdx.x == 0) sm.tm[1] += (unsigned long long)(clock64() - tr0);
 }
 
 template <int MT>
@@ -664,7 +674,7 @@ __device__ void gemv_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_
   if (p.b == 1) gemv_dispatch<0>(p, sm, t, stage, ab, G);
   else if (p.b <= 8) gemv_dispatch<1>(p, sm, t, stage, ab, G);
   else gemv_dispatch<2>(p, sm, t, stage, ab, G);
-  const unsigned long long te0 = (p.trace && threadIdx.x == 0) ? gtimer() : 0ull;
+  const long long te0 = (p.trace && threadIdx.x == 0) ? clock64() : 0ll;
 
   const int nthr = kConsumerWarps * 32;
   const int n = t.nunits;
@@ -777,7 +787,7 @@ __device__ void gemv_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_
       }
     }
   }
-  if (p.trace && threadIdx.x == 0) sm.tm[2] += gtimer() - te0;
+  if (p.trace && threadIdx.x == 0) sm.tm[2] += (unsigned long long)(clock64() - te0);
 }
 
 __device__ void embed_task(const KParams& p, Smem& sm, const TaskDesc& t, bool ab) {
@@ -851,8 +861,8 @@ __device__ __noinline__ void attn_task(const KParams& p, Smem& sm, const TaskDes
   uint32_t ks = 0;  // stage count within the task: picks the warp group
   AttnPiece a;
   for (int j = 0; attn_piece(p, sm.attn_R, (int)t.u0, j, a); ++j) {
-    const unsigned long long tc0 = tr ? gtimer() : 0ull;
-    const unsigned long long wait0 = tr ? sm.wait_ns : 0ull;
+    const long long tc0 = tr ? clock64() : 0ll;
+    const unsigned long long wait0 = tr ? sm.wait_cyc : 0ull;
     // Q fragments of head g_ of this kv group
     uint32_t qa[NK][4];
     {
@@ -879,7 +889,7 @@ __device__ __noinline__ void attn_task(const KParams& p, Smem& sm, const TaskDes
     const int ns = (a.t1 - a.t0 + T - 1) / T;
     for (int k = 0; k < ns; ++k, ++stage, ++ks) {
       const int slot = stage % kNumSlots;
-      if (!ab) ab = !mbar_wait_warp(p, &sm.full[slot], (stage / kNumSlots) & 1, tr ? &sm.wait_ns : nullptr);
+      if (!ab) ab = !mbar_wait_warp(p, &sm.full[slot], (stage / kNumSlots) & 1, tr ? &sm.wait_cyc : nullptr);
       const int g0 = a.t0 + k * T + 16 * grp;  // first token of this warp's group
       const int nv = min(16, a.t1 - g0);        // valid tokens in the group (<= 0: none)
       if (!ab && (int)(ks % NG) == wsel && nv > 0) {
@@ -958,10 +968,10 @@ __device__ __noinline__ void attn_task(const KParams& p, Smem& sm, const TaskDes
       if (!ab && lane == 0) mbar_arrive(&sm.empty[slot]);
     }
 
-    unsigned long long tr0 = 0;
+    long long tr0 = 0;
     if (tr) {
-      tr0 = gtimer();
-      sm.tm[0] += tr0 - tc0 - (sm.wait_ns - wait0);
+      tr0 = clock64();
+      sm.tm[0] += (unsigned long long)(tr0 - tc0) - (sm.wait_cyc - wait0);
     }
     // this warp's state of head g_: l summed over the row's 4 lanes, O = hi row + lo row
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
@@ -1001,8 +1011,8 @@ __device__ __noinline__ void attn_task(const KParams& p, Smem& sm, const TaskDes
       }
     }
     cbar();
-    const unsigned long long te0 = tr ? gtimer() : 0ull;
-    if (tr) sm.tm[1] += te0 - tr0;
+    const long long te0 = tr ? clock64() : 0ll;
+    if (tr) sm.tm[1] += (unsigned long long)(te0 - tr0);
     if (threadIdx.x == 0) {
       int last = 0;
       if (!ab) {
@@ -1047,7 +1057,7 @@ __device__ __noinline__ void attn_task(const KParams& p, Smem& sm, const TaskDes
       }
     }
     cbar();  // sm.red is reused by the next piece
-    if (tr) sm.tm[2] += gtimer() - te0;
+    if (tr) sm.tm[2] += (unsigned long long)(clock64() - te0);
   }
 }
 
@@ -1064,7 +1074,7 @@ __device__ void consumer(const KParams& p, Smem& sm, const TaskDesc* ts, int nt)
     // dependency wait: one thread polls, the others wait at the consumer barrier
     unsigned long long tr0 = 0, tr1 = 0;
     if (threadIdx.x == 0) {
-      if (p.trace) { tr0 = gtimer(); sm.wait_ns = 0; sm.tm[0] = sm.tm[1] = sm.tm[2] = 0; }
+      if (p.trace) { tr0 = gtimer(); sm.wait_cyc = 0; sm.tm[0] = sm.tm[1] = sm.tm[2] = 0; }
       bool ok = !ab;
       if (ok && t.wait_ctr != kNoCounter) {
         const uint32_t target = t.wait_count * p.epoch;
@@ -1089,7 +1099,7 @@ __device__ void consumer(const KParams& p, Smem& sm, const TaskDesc* ts, int nt)
     }
     cbar();
     if (threadIdx.x == 0) {
-      const unsigned long long ts0 = p.trace ? gtimer() : 0ull;
+      const long long ts0 = p.trace ? clock64() : 0ll;
       if (!ab) {
         // release: everything the consumer warps wrote before the barrier above is visible to
         // whoever acquires the counter; bulk copies (async proxy) may read it next
@@ -1106,16 +1116,17 @@ __device__ void consumer(const KParams& p, Smem& sm, const TaskDesc* ts, int nt)
       }
       if (p.trace) {
         unsigned long long* r = p.trace + 8ull * (p.task_off[blockIdx.x] + ti);
+        const long long ce = clock64();
         const unsigned long long te = gtimer();
         r[0] = tr0;
         r[1] = tr1;
         r[2] = te;
         r[3] = (unsigned long long)t.op | ((unsigned long long)t.layer << 8) |
-               ((unsigned long long)blockIdx.x << 24) | (min(sm.wait_ns, 0xFFFFFFull) << 40);
+               ((unsigned long long)blockIdx.x << 24) | (min(sm.wait_cyc, 0xFFFFFFull) << 40);
         r[4] = sm.tm[0];
         r[5] = sm.tm[1];
         r[6] = sm.tm[2];
-        r[7] = te - ts0;
+        r[7] = (unsigned long long)(ce - ts0);
       }
     }
     cbar();

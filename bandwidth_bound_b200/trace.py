@@ -1,9 +1,12 @@
 """Summaries of the per-task timeline the megakernel records (mk_set_trace).
 
 Each record is {t_wait_start, t_wait_end, t_end, meta, compute, reduce, epilogue,
-signal} in globaltimer ns, with meta = op | layer << 8 | sm << 24 | slot_wait_ns << 40.  The summary answers where
-a step's time goes: waiting on dependency counters (another SM's work not done),
-waiting on pool slots (HBM bytes not yet landed), or computing.
+signal}: the three timestamps in globaltimer ns (comparable across SMs), meta = op |
+layer << 8 | sm << 24 | slot_wait << 40, and the durations in SM clock cycles (the
+globaltimer is too coarse for sub-microsecond intervals), converted here with the SM
+clock.  The summary answers where a step's time goes: waiting on dependency counters
+(another SM's work not done), waiting on pool slots (HBM bytes not yet landed), or
+computing.
 """
 from __future__ import annotations
 
@@ -12,22 +15,25 @@ import numpy as np
 OPS = {1: "embed", 2: "qkv", 3: "attn", 4: "oproj", 5: "gateup", 6: "down", 7: "lmhead"}
 
 
-def decode(records) -> dict:
+def decode(records, sm_mhz: float = 1965.0) -> dict:
+    """Fields of the records; durations converted from SM cycles to ns at sm_mhz."""
     r = np.asarray(records, dtype=np.uint64).reshape(-1, 8)
     meta = r[:, 3]
+    ns = 1e3 / sm_mhz
+    cyc = lambda a: (a.astype(np.float64) * ns).astype(np.int64)  # noqa: E731
     return {
-        "compute": r[:, 4].astype(np.int64), "reduce": r[:, 5].astype(np.int64),
-        "epilogue": r[:, 6].astype(np.int64), "signal": r[:, 7].astype(np.int64),
+        "compute": cyc(r[:, 4]), "reduce": cyc(r[:, 5]),
+        "epilogue": cyc(r[:, 6]), "signal": cyc(r[:, 7]),
         "t0": r[:, 0].astype(np.int64), "t1": r[:, 1].astype(np.int64), "t2": r[:, 2].astype(np.int64),
         "op": (meta & np.uint64(0xFF)).astype(np.int64),
         "layer": ((meta >> np.uint64(8)) & np.uint64(0xFFFF)).astype(np.int64),
         "sm": ((meta >> np.uint64(24)) & np.uint64(0xFFFF)).astype(np.int64),
-        "slot_wait": (meta >> np.uint64(40)).astype(np.int64),
+        "slot_wait": cyc(meta >> np.uint64(40)),
     }
 
 
-def summarize(records, n_layers: int) -> str:
-    d = decode(records)
+def summarize(records, n_layers: int, sm_mhz: float = 1965.0) -> str:
+    d = decode(records, sm_mhz)
     base = int(d["t0"].min())
     end = int(d["t2"].max())
     step_us = (end - base) / 1e3

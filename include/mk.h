@@ -195,13 +195,13 @@ MK_API int mk_set_debug(mk_handle_t h, float *layer_hidden);
 
 /* Per-task timeline for profiling: when records is a device uint64 buffer of
  * [capacity][8] with capacity >= mk_num_tasks(h), each later step writes, for task
- * k of the flattened per-SM streams, {globaltimer before its dependency wait,
- * after the wait, at its end, meta, compute ns, reduce ns, epilogue ns, signal ns}
- * where meta = op | layer << 8 | sm << 24 | (ns warp 0 waited for pool slots,
- * capped at 2^24-1) << 40 and the four durations are measured by warp 0 (compute:
- * stage processing after the slot waits; reduce: cross-warp reduction or attention
- * merge; epilogue: the task's writes, attention combine; signal: the counter
- * release).  NULL turns it off. */
+ * k of the flattened per-SM streams, {globaltimer ns before its dependency wait,
+ * after the wait, at its end, meta, compute, reduce, epilogue, signal} where
+ * meta = op | layer << 8 | sm << 24 | (SM cycles warp 0 waited for pool slots,
+ * capped at 2^24-1) << 40 and the four durations are SM clock cycles measured by
+ * warp 0 (compute: stage processing after the slot waits; reduce: cross-warp
+ * reduction or attention merge; epilogue: the task's writes, attention combine;
+ * signal: the counter release).  NULL turns it off. */
 MK_API int mk_set_trace(mk_handle_t h, uint64_t *records, int64_t capacity);
 
 /* Number of task descriptors in the handle's per-SM streams (all SMs). */
