@@ -121,6 +121,39 @@ static std::string build_tensor_maps(const mk_model_cfg& c, const mk_weight_ptrs
   return "";
 }
 
+// Tensor maps of the GEMV operand buffers (appended after the weight maps): per operand kind,
+// bf16 tile parts q = 2 * mt + part as rows of 64 values (boxes of 8 rows = 64 columns of one
+// tile part), then the fp32 batch row 0 as rows of 32 values (boxes of 2 rows = 64 columns).
+static std::string encode_operand_maps(std::vector<CUtensorMap>& maps, int L, int ntiles,
+                                       const __nv_bfloat16* const tiles[3], const float* const rows[3],
+                                       const int lds[3]) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (!encode) return "cuTensorMapEncodeTiled is not available";
+  maps.resize((size_t)mk::num_all_tmaps(L), CUtensorMap{});
+  cuuint32_t es[2] = {1, 1};
+  for (int kind = 0; kind < 3; ++kind) {
+    const int ld = lds[kind];
+    for (int q = 0; q < 2 * ntiles; ++q) {
+      cuuint64_t dims[2] = {64, (cuuint64_t)ld / 8};
+      cuuint64_t strides[1] = {128};
+      cuuint32_t box[2] = {64, 8};
+      CUresult r = encode(&maps[mk::opmap_index(L, kind, q)], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                          const_cast<__nv_bfloat16*>(tiles[kind]) + (size_t)q * ld * 8, dims, strides, box, es,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      if (r != CUDA_SUCCESS) return "cuTensorMapEncodeTiled failed for an operand buffer";
+    }
+    cuuint64_t dims[2] = {32, (cuuint64_t)ld / 32};
+    cuuint64_t strides[1] = {128};
+    cuuint32_t box[2] = {32, 2};
+    CUresult r = encode(&maps[mk::opmap_index(L, kind, mk::kOpMapsPerKind - 1)], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+                        const_cast<float*>(rows[kind]), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return "cuTensorMapEncodeTiled failed for an operand row";
+  }
+  return "";
+}
+
 // Tensor maps of the K and V pools, viewed as rows of head_dim values ([L][pages][nkv][16]
 // rows): boxes of one 16-token page of one head with 128-byte swizzle.  head_dim 64: a 2-D
 // box of 64 x 16; head_dim 128: a 3-D box {64 columns, 16 rows, 2 halves}, the halves
@@ -201,7 +234,7 @@ MK_API int mk_create_from_plan(mk_plan_t plan, const mk_weight_ptrs* w, int32_t 
   int regs = 0, lmem = 0, maxthr = 0;
   cudaError_t ce = mk::kernel_attributes(&regs, &lmem, &maxthr);
   if (ce != cudaSuccess) { release(h); return cuda_fail(nullptr, ce, "kernel attributes"); }
-  if (maxthr < mk::kThreads) { release(h); return fail(nullptr, MK_ERR_CUDA, "kernel cannot run 288 threads"); }
+  if (maxthr < mk::kThreads) { release(h); return fail(nullptr, MK_ERR_CUDA, "kernel cannot run its 320 threads"); }
 
   const mk::Geometry G = mk::geometry(c);
   const int S = plan->num_sms * plan->attn_slots_per_sm;
@@ -221,7 +254,7 @@ MK_API int mk_create_from_plan(mk_plan_t plan, const mk_weight_ptrs* w, int32_t 
   std::vector<CUtensorMap> maps;
   std::string merr = build_tensor_maps(c, w, maps);
   if (!merr.empty()) { release(h); return fail(nullptr, MK_ERR_CUDA, merr); }
-  const size_t o_maps = take(sizeof(CUtensorMap) * maps.size());
+  const size_t o_maps = take(sizeof(CUtensorMap) * (size_t)mk::num_all_tmaps(G.L));
   const size_t o_x = take(sizeof(float) * mb * G.d);
   const size_t o_q = take(sizeof(float) * mb * G.qdim);
   const int ld_x = mk::round_up(G.d, mk::kBoxCols), ld_a = mk::round_up(G.qdim, mk::kBoxCols),
@@ -256,6 +289,15 @@ MK_API int mk_create_from_plan(mk_plan_t plan, const mk_weight_ptrs* w, int32_t 
   if (ce != cudaSuccess) { release(h); return cuda_fail(nullptr, ce, "cudaHostGetDevicePointer"); }
 
   char* A = (char*)h->arena;
+  {
+    auto tl = [&](size_t o) { return (const __nv_bfloat16*)(A + o); };
+    auto rw = [&](size_t o, int ld) { return (const float*)(A + o + (size_t)ntiles * 2 * ld * 8 * 2); };
+    const __nv_bfloat16* tiles[3] = {tl(o_ax), tl(o_aa), tl(o_ah)};
+    const float* rows[3] = {rw(o_ax, ld_x), rw(o_aa, ld_a), rw(o_ah, ld_h)};
+    const int lds[3] = {ld_x, ld_a, ld_h};
+    merr = encode_operand_maps(maps, G.L, ntiles, tiles, rows, lds);
+    if (!merr.empty()) { release(h); return fail(nullptr, MK_ERR_CUDA, merr); }
+  }
   ce = cudaMemcpy(A + o_layers, lw.data(), sizeof(LayerW) * c.n_layers, cudaMemcpyHostToDevice);
   if (ce == cudaSuccess)
     ce = cudaMemcpy(A + o_tasks, flat.data(), sizeof(mk::TaskDesc) * flat.size(), cudaMemcpyHostToDevice);
@@ -543,7 +585,7 @@ int static_setup(StaticState& s, const mk_model_cfg& c, const mk_weight_ptrs* w,
   int regs = 0, lmem = 0, maxthr = 0;
   cudaError_t ce = mk::kernel_attributes(&regs, &lmem, &maxthr);
   if (ce != cudaSuccess) return cuda_fail(nullptr, ce, "kernel attributes");
-  if (maxthr < mk::kThreads) return fail(nullptr, MK_ERR_CUDA, "kernel cannot run 288 threads");
+  if (maxthr < mk::kThreads) return fail(nullptr, MK_ERR_CUDA, "kernel cannot run its 320 threads");
 
   mk_plan_opts o{};
   o.num_sms = prop.multiProcessorCount;
@@ -568,7 +610,7 @@ int static_setup(StaticState& s, const mk_model_cfg& c, const mk_weight_ptrs* w,
   const size_t o_layers = take(sizeof(LayerW) * c.n_layers);
   const size_t o_tasks = take(sizeof(mk::TaskDesc) * flat.size());
   const size_t o_offs = take(sizeof(uint32_t) * offs.size());
-  const size_t o_maps = take(sizeof(CUtensorMap) * (size_t)mk::num_tmaps(G.L));
+  const size_t o_maps = take(sizeof(CUtensorMap) * (size_t)mk::num_all_tmaps(G.L));
   const size_t o_x = take(sizeof(float) * mb * G.d);
   const size_t o_q = take(sizeof(float) * mb * G.qdim);
   const int ld_x = mk::round_up(G.d, mk::kBoxCols), ld_a = mk::round_up(G.qdim, mk::kBoxCols),
@@ -597,6 +639,15 @@ int static_setup(StaticState& s, const mk_model_cfg& c, const mk_weight_ptrs* w,
   if (!merr.empty()) return fail(nullptr, MK_ERR_CUDA, merr);
 
   unsigned char* A = s.base;
+  {
+    auto tl = [&](size_t o) { return (const __nv_bfloat16*)(A + o); };
+    auto rw = [&](size_t o, int ld) { return (const float*)(A + o + (size_t)ntiles * 2 * ld * 8 * 2); };
+    const __nv_bfloat16* tiles[3] = {tl(o_ax), tl(o_aa), tl(o_ah)};
+    const float* rows[3] = {rw(o_ax, ld_x), rw(o_aa, ld_a), rw(o_ah, ld_h)};
+    const int lds[3] = {ld_x, ld_a, ld_h};
+    merr = encode_operand_maps(maps, G.L, ntiles, tiles, rows, lds);
+    if (!merr.empty()) return fail(nullptr, MK_ERR_CUDA, merr);
+  }
   ce = cudaMemsetAsync(A, 0, total, stream);
   if (ce == cudaSuccess)
     ce = cudaMemcpyAsync(A + o_layers, lw.data(), sizeof(LayerW) * c.n_layers, cudaMemcpyHostToDevice, stream);

@@ -22,10 +22,9 @@ namespace mk {
 
 // ---- launch geometry -------------------------------------------------------------------
 constexpr int kConsumerWarps = 8;                       // compute warps per CTA
-constexpr int kThreads = (kConsumerWarps + 1) * 32;     // + one producer (TMA) warp
-constexpr int kSlotBytes = 32 * 1024;                   // one pool stage: weights or KV pages (1024-byte aligned)
-constexpr int kNumSlots = 5;                            // pool depth (160 KB)
-constexpr int kRingBytes = 4 * 1024;                    // per consumer warp: GEMV operands of its next k blocks
+constexpr int kThreads = (kConsumerWarps + 2) * 32;     // + the weight/KV producer warp + the operand warp
+constexpr int kSlotBytes = 40 * 1024;                   // one pool stage: weights + their operands, or KV pages
+constexpr int kNumSlots = 5;                            // pool depth (200 KB)
 constexpr int kMaxBatch = 16;
 constexpr int kMaxBlocks = 8;                           // 8-row blocks per GEMV task (64 rows)
 constexpr int kPage = 16;                               // tokens per KV page
@@ -79,28 +78,47 @@ MK_HD int max_units(int op) { return (op == OP_QKV || op == OP_GATEUP) ? kMaxBlo
 MK_HD uint32_t ceil_div(uint32_t a, uint32_t b) { return (a + b - 1) / b; }
 MK_HD int round_up(int a, int b) { return (a + b - 1) / b * b; }
 
-// K columns per pool stage of a GEMV task with `blocks` 8-row blocks: the weights fit a
-// slot and every consumer warp gets whole 32-column blocks (1, 2 or 4 of them).
+// Operand bytes per K column of one stage for a batch of up to max_batch rows: bf16 hi and
+// lo parts of every 8-row batch tile (16 bytes each per column).  The batch-1 path uses the
+// first 4 bytes (fp32) of the same room.
+MK_HD int operand_col_bytes(int max_batch) { return 32 * ((max_batch + 7) / 8); }
+
+// K columns per pool stage of a GEMV task with `blocks` 8-row blocks: the largest multiple of
+// 64 whose weights (blocks * 8 rows) and operands fit one slot, at most K rounded up to 64.
 MK_HD int stage_cols(int blocks, int K, int max_batch) {
-  (void)max_batch;
-  const int kc = blocks >= 5 ? 256 : (blocks >= 3 ? 512 : 1024);
+  const int per_col = blocks * 8 * 2 + operand_col_bytes(max_batch);
+  int kc = (kSlotBytes / per_col) / kBoxCols * kBoxCols;
+  if (kc < kBoxCols) kc = kBoxCols;
   const int kp = round_up(K, kBoxCols);
   return kp <= kc ? kp : kc;
 }
 
-// Operand tile layout in global memory (written by the producing epilogues, read by the
-// consuming GEMV's lanes): for batch tile mt (rows 8mt..8mt+7) and part (0 hi, 1 lo),
-// groups of 8 columns; group kg holds 8 rows of 16 bytes (row g in slot g ^ (2 * ((kg >> 1)
-// & 3)), a permutation that keeps every 128-byte group whole for the reading warp).
-MK_HD size_t operand_index(int mt, int part, int kg, int g, int e, int ld) {
-  return ((((size_t)(mt * 2 + part) * (ld / 8) + kg) * 8 + (g ^ (2 * ((kg >> 1) & 3)))) * 8 + e);
+// Operand layouts in global memory, written by the producing epilogues and copied per stage
+// by tiled TMA boxes into the slot, where the consuming lanes read them.  A 64-column chunk c
+// holds two 32-column k blocks kb = 2c + h: block h takes the 16-byte column groups 2tq + h
+// (tq = 0..3) of the chunk, the groups lane (g, tq) reads from its weight rows.
+//   bf16 tiles: per batch tile mt (rows 8mt..8mt+7) and part (0 hi, 1 lo), block kb is 512
+//   contiguous bytes: 32 pieces of 16 bytes, piece 4 * row + tq = the 8 columns of group
+//   2tq + h of batch row `row` - lane (g, tq) reads piece `lane`;
+//   fp32 batch row 0: block kb is 128 bytes, piece tq = the 8 values of group 2tq + h.
+MK_HD int opnd_block(int k) { return ((k >> 6) << 1) | ((k >> 3) & 1); }
+MK_HD size_t opnd_tile_index(int mt, int part, int k, int row, int ld) {
+  return ((((size_t)(mt * 2 + part) * (ld / 32) + opnd_block(k)) * 32 + row * 4 + ((k >> 4) & 3)) * 8 + (k & 7));
 }
+MK_HD size_t opnd_row0_index(int k) { return ((size_t)opnd_block(k) * 4 + ((k >> 4) & 3)) * 8 + (k & 7); }
 
 // Index of the TMA descriptor of weight matrix `mat` (0 wq .. 6 w_down) of a layer for
 // boxes of 8*n rows; the LM head's maps follow the layers' (mat 0 of layer L).
 MK_HD int tmap_index(int layer, int mat, int n) { return (layer * kNumMats + mat) * kMaxBlocks + (n - 1); }
 
 MK_HD int num_tmaps(int n_layers) { return (n_layers + 1) * kNumMats * kMaxBlocks; }
+
+// Operand tensor maps, after the weight maps: per operand kind (0 normed x, 1 attention
+// output, 2 SwiGLU output), 2 * tiles bf16 maps (tile mt, part) then the fp32 row-0 map.
+constexpr int kMaxTiles = (kMaxBatch + 7) / 8;
+constexpr int kOpMapsPerKind = 2 * kMaxTiles + 1;
+MK_HD int opmap_index(int n_layers, int kind, int q) { return num_tmaps(n_layers) + kind * kOpMapsPerKind + q; }
+MK_HD int num_all_tmaps(int n_layers) { return num_tmaps(n_layers) + 3 * kOpMapsPerKind; }
 
 // Tokens per attention stage: K rows then V rows of the same tokens, 32 KB total.
 MK_HD int attn_stage_tokens(int head_dim) { return head_dim == 64 ? 128 : 64; }

@@ -29,13 +29,13 @@ typedef TmaDesc CUtensorMapLike;
 // shared memory
 
 struct Smem {
-  alignas(1024) uint8_t pool[kNumSlots][kSlotBytes];  // per slot: weight boxes or KV pages of one stage
+  alignas(1024) uint8_t pool[kNumSlots][kSlotBytes];  // per slot: weight boxes + operands, or KV pages, of one stage
   alignas(16) float red[kRedBytes / 4];                 // GEMV cross-warp partials / attention merge
-  alignas(128) uint8_t ring[kConsumerWarps][kRingBytes];  // per warp: operands of its upcoming k blocks
   alignas(16) float ep[kMaxBlocks * 8][kMaxBatch];       // per-task results [row][batch]
   float mw[kConsumerWarps][8], lw[kConsumerWarps][8];    // attention merge state per warp
   float inv_rms[kMaxBatch];
-  alignas(8) uint64_t full[kNumSlots];                   // weight/KV bytes of the stage landed
+  alignas(8) uint64_t wfull[kNumSlots];                  // weight/KV bytes of the stage landed
+  alignas(8) uint64_t ofull[kNumSlots];                  // the stage's operand bytes landed (operand warp)
   alignas(8) uint64_t empty[kNumSlots];                  // all consumer warps done with the stage
   int attn_R, bad, flag, flag2;  // attn_R: tokens per attention range (this step)
   unsigned long long wait_cyc;  // tracing: SM cycles warp 0 spent waiting for pool slots in the current task
@@ -347,10 +347,10 @@ __device__ void issue_weights(const KParams& p, Smem& sm, const TaskDesc& t, int
   const int R = t.nunits * rows_per_unit(t.op);
   const int kc0 = s * t.kc;
   const int nch = (min((int)t.kc, K - kc0) + kBoxCols - 1) / kBoxCols;
-  if (lane == 0) mbar_expect_tx(&sm.full[slot], (uint32_t)(nch * R * 128));
+  if (lane == 0) mbar_expect_tx(&sm.wfull[slot], (uint32_t)(nch * R * 128));
   __syncwarp();
   for (int c = lane; c < nch; c += 32)
-    issue_gemv_chunk(p, t, kc0 + c * kBoxCols, sm.pool[slot] + (size_t)c * R * 128, &sm.full[slot], pol);
+    issue_gemv_chunk(p, t, kc0 + c * kBoxCols, sm.pool[slot] + (size_t)c * R * 128, &sm.wfull[slot], pol);
 }
 
 // K and V pages of stage k of attention piece a into slot `slot`: whole 16-token pages as
@@ -369,7 +369,7 @@ __device__ bool issue_kv(const KParams& p, Smem& sm, const TaskDesc& t, const At
   }
   if (__any_sync(0xffffffffu, bad)) return false;
   const uint32_t page_bytes = (uint32_t)kPage * p.hd * 2u;
-  if (lane == 0) mbar_expect_tx(&sm.full[slot], 2u * npg * page_bytes);
+  if (lane == 0) mbar_expect_tx(&sm.wfull[slot], 2u * npg * page_bytes);
   __syncwarp();
   for (int e = lane; e < 2 * npg; e += 32) {
     const int q = e >> 1;
@@ -377,8 +377,8 @@ __device__ bool issue_kv(const KParams& p, Smem& sm, const TaskDesc& t, const At
     const int row = ((t.layer * p.num_pages + id) * p.nkv + a.h) * kPage;
     uint8_t* dst = sm.pool[slot] + (size_t)(e & 1) * T * p.hd * 2 + (size_t)q * page_bytes;
     const void* map = (e & 1) ? (const void*)&p.vmap : (const void*)&p.kmap;
-    if (p.hd == 64) tma_2d(dst, map, 0, row, &sm.full[slot], pol);
-    else tma_3d(dst, map, 0, row, 0, &sm.full[slot], pol);
+    if (p.hd == 64) tma_2d(dst, map, 0, row, &sm.wfull[slot], pol);
+    else tma_3d(dst, map, 0, row, 0, &sm.wfull[slot], pol);
   }
   return true;
 }
@@ -423,7 +423,96 @@ __device__ void producer(const KParams& p, Smem& sm, const TaskDesc* ts, int nt)
       const uint32_t first = wk > (uint32_t)kNumSlots ? wk - kNumSlots : 0u;
       for (uint32_t s = first; s < wk; ++s) {
         const uint64_t t0 = gtimer();
-        while (!mbar_try(&sm.full[s % kNumSlots], (s / kNumSlots) & 1))
+        while (!mbar_try(&sm.wfull[s % kNumSlots], (s / kNumSlots) & 1))
+          if (gtimer() - t0 > p.timeout_ns) break;
+      }
+    }
+    __syncwarp();
+  }
+}
+
+// The operand warp: for each GEMV task of the CTA's stream, in order, it waits for the
+// dependency counter that guards the task's activations and then copies every stage's
+// operand slice into the stage's slot behind the weights - per 64-column chunk one tiled box
+// per bf16 (tile, part), or one box of the fp32 row for batch 1 - completing on the slot's
+// ofull barrier.  Attention stages get a plain arrival, so that ofull completes one phase
+// per use of the slot like wfull.  It never waits on the consumers' work beyond the slot
+// being free, so the operands of a stage are requested as soon as both allow.
+__device__ void operand_loader(const KParams& p, Smem& sm, const TaskDesc* ts, int nt) {
+  const int lane = threadIdx.x & 31;
+  const uint64_t pol = policy_evict_last();  // every SM reads the same operands
+  const CUtensorMapLike* maps = reinterpret_cast<const CUtensorMapLike*>(p.tmaps);
+  const int T = attn_stage_tokens(p.hd);
+  const int ntile = (p.b + 7) >> 3;
+  uint32_t wk = 0;  // stages handled
+  bool fail = false;
+  int met_ctr = -1;
+  uint32_t met_target = 0;
+  for (int wt = 0; wt < nt && !fail; ++wt) {
+    const TaskDesc t = ts[wt];
+    if (t.op == OP_EMBED) continue;
+    if (t.op == OP_ATTN) {
+      AttnPiece a;
+      for (int j = 0; !fail && attn_piece(p, sm.attn_R, (int)t.u0, j, a); ++j) {
+        const int ns = (a.t1 - a.t0 + T - 1) / T;
+        for (int k = 0; k < ns; ++k, ++wk) {
+          const int slot = wk % kNumSlots;
+          if (!mbar_wait_warp(p, &sm.empty[slot], ((wk / kNumSlots) & 1) ^ 1)) { fail = true; break; }
+          if (lane == 0) mbar_arrive(&sm.ofull[slot]);
+          __syncwarp();
+        }
+      }
+      continue;
+    }
+    // the task's activations are complete once its dependency counter is met
+    if (t.wait_ctr != kNoCounter) {
+      const uint32_t target = t.wait_count * p.epoch;
+      if (t.wait_ctr != met_ctr || target != met_target) {
+        int ok = 1;
+        if (lane == 0) ok = wait_counter(p, t.wait_ctr, t.wait_count) ? 1 : 0;
+        if (!__shfl_sync(0xffffffffu, ok, 0)) { fail = true; break; }
+        met_ctr = t.wait_ctr;
+        met_target = target;
+        if (lane == 0) asm volatile("fence.proxy.async.global;" ::: "memory");  // the copies below read it
+        __syncwarp();
+      }
+    }
+    const int kind = operand_kind(t.op);
+    const int K = gemv_K_dev(p, t.op);
+    const int R = t.nunits * rows_per_unit(t.op);
+    const int nst = gemv_stages(p, t);
+    for (int ws = 0; ws < nst; ++ws, ++wk) {
+      const int slot = wk % kNumSlots;
+      if (!mbar_wait_warp(p, &sm.empty[slot], ((wk / kNumSlots) & 1) ^ 1)) { fail = true; break; }
+      uint8_t* dst = sm.pool[slot] + (size_t)R * t.kc * 2;
+      const int k0 = ws * t.kc;
+      const int nch = (min((int)t.kc, K - k0) + kBoxCols - 1) / kBoxCols;
+      if (p.b == 1) {
+        if (lane == 0) mbar_expect_tx(&sm.ofull[slot], (uint32_t)nch * 256u);
+        __syncwarp();
+        for (int c = lane; c < nch; c += 32)
+          tma_2d(dst + (size_t)c * 256, maps + opmap_index(p.L, kind, kOpMapsPerKind - 1), 0, k0 / 32 + 2 * c,
+                 &sm.ofull[slot], pol);
+      } else {
+        const int nbox = 2 * ntile * nch;
+        if (lane == 0) mbar_expect_tx(&sm.ofull[slot], (uint32_t)nbox * 1024u);
+        __syncwarp();
+        for (int e = lane; e < nbox; e += 32) {
+          const int q = e / nch, c = e - q * nch;
+          tma_2d(dst + (size_t)q * t.kc * 16 + (size_t)c * 1024, maps + opmap_index(p.L, kind, q), 0, k0 / 8 + 8 * c,
+                 &sm.ofull[slot], pol);
+        }
+      }
+      __syncwarp();
+    }
+  }
+  if (fail) {
+    // Drain: let every copy already issued land before the CTA may exit.
+    if (lane == 0) {
+      const uint32_t first = wk > (uint32_t)kNumSlots ? wk - kNumSlots : 0u;
+      for (uint32_t s = first; s < wk; ++s) {
+        const uint64_t t0 = gtimer();
+        while (!mbar_try(&sm.ofull[s % kNumSlots], (s / kNumSlots) & 1))
           if (gtimer() - t0 > p.timeout_ns) break;
       }
     }
@@ -451,68 +540,29 @@ __device__ void compute_inv_rms(const KParams& p, Smem& sm, int inst, int nparts
 // (the remainder) into the tile layout, and fp32 for batch row 0.
 __device__ __forceinline__ void put_operand(bf16* tiles, float* f, int ld, int bi, int k, float v) {
   const bf16 h = __float2bfloat16_rn(v);
-  const int mt = bi >> 3, g = bi & 7, kg = k >> 3, e = k & 7;
-  tiles[operand_index(mt, 0, kg, g, e, ld)] = h;
-  tiles[operand_index(mt, 1, kg, g, e, ld)] = __float2bfloat16_rn(v - __bfloat162float(h));
-  if (bi == 0) f[k] = v;
-}
-
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(valid ? 16 : 0)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-// Copy the operand of column group kg (8 columns) of this lane into ring entry e of its
-// warp.  MT >= 1: MT tiles of (hi, lo) 16-byte rows (batch row 8mt + g; zeros past the
-// batch), lane-private pieces: entry e, piece q at ((e * 2 * MT + q) * 32 + lane) * 16.
-// MT == 0: the 8 fp32 values of batch row 0, shared by the 8 lanes (g = 0..7) of one tq:
-// lanes g = 0, 1 copy one half each to entry e at (e * 4 + tq) * 32 + g * 16, so that
-// every column group is read from L2 once per warp.
-template <int MT>
-__device__ __forceinline__ void fetch_opnd(const KParams& p, uint8_t* ring, int e, const bf16* tiles, const float* f,
-                                           int ld, int kg, int g, int lane) {
-  if constexpr (MT == 0) {
-    if (g < 2) cp_async16(ring + ((size_t)e * 4 + (lane & 3)) * 32 + g * 16, f + 8 * kg + 4 * g, true);
-  } else {
-    uint8_t* base = ring + (size_t)e * 2 * MT * 512 + lane * 16;
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-      const bool v = mt * 8 + g < p.b;
-      cp_async16(base + (2 * mt) * 512, tiles + operand_index(mt, 0, kg, g, 0, ld), v);
-      cp_async16(base + (2 * mt + 1) * 512, tiles + operand_index(mt, 1, kg, g, 0, ld), v);
-    }
-  }
+  const int mt = bi >> 3, row = bi & 7;
+  tiles[opnd_tile_index(mt, 0, k, row, ld)] = h;
+  tiles[opnd_tile_index(mt, 1, k, row, ld)] = __float2bfloat16_rn(v - __bfloat162float(h));
+  if (bi == 0) f[opnd_row0_index(k)] = v;
 }
 
 // Stream the task's stages through the eight warps and reduce into sm.ep[row][batch].
-// Weight stage layout (per 64-column chunk): 8*G rows of 128 bytes, 16-byte chunks
-// swizzled (chunk c of row r at c ^ (r & 7)).  Warp w takes 32-column k blocks w, w+8,
-// ... of every stage; a k block is the even (h = 0) or odd (h = 1) 16-byte chunks of a
-// 64-column chunk, so lane (g, tq) reads chunk 2*tq + h of row 8j + g - conflict-free -
-// which holds columns 16*tq + 8*h .. +7, column group kg = 8*chunk + 2*tq + h.  The
-// operand of that group is copied (cp.async) into the warp's shared-memory ring Q - 1
-// blocks ahead of its use, so the L2 latency overlaps the earlier blocks' work.  MT = 0:
-// CUDA-core FMA (batch 1);
-// MT = 1, 2: mma.sync with MT tiles of 8 batch rows, rows 0-7 of the M = 16 tile the bf16
-// hi parts, rows 8-15 the lo parts.
+// Slot layout of a stage: the weights (per 64-column chunk: 8*G rows of 128 bytes, 16-byte
+// pieces swizzled, piece c of row r at c ^ (r & 7)), then the stage's operands (opnd_*
+// layouts: per bf16 (tile, part) kc * 16 bytes, or kc * 4 bytes of fp32 row 0).  Warp w takes
+// 32-column k blocks w, w+8, ... of every stage; block kb is the even (h = 0) or odd (h = 1)
+// 16-byte pieces of chunk kb / 2, so lane (g, tq) reads piece 2*tq + h of row 8j + g -
+// conflict-free - which holds columns 16*tq + 8*h .. +7, and the operand piece of the same
+// columns at `lane` (bf16) or `tq` (fp32, shared by the 8 lanes of one tq).
+// MT = 0: CUDA-core FMA (batch 1); MT = 1, 2: mma.sync with MT tiles of 8 batch rows, rows
+// 0-7 of the M = 16 tile the bf16 hi parts, rows 8-15 the lo parts.
 template <int MT, int G>
 __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDesc t, uint32_t& stage, bool& ab) {
-  constexpr int NQ = MT == 0 ? 2 : 2 * MT;       // 16-byte pieces per lane and k block
-  // ring entries: 16 of 128 bytes (batch 1), 4 of 1 KB (batch <= 8) or 2 of 2 KB (batch > 8)
-  constexpr int Q = MT == 0 ? 16 : kRingBytes / (NQ * 512);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, tq = lane & 3;
   const int K = gemv_K_dev(p, t.op);
   const int kc = t.kc;
   const int nst = (K + kc - 1) / kc;
-  const int kind = operand_kind(t.op);
-  const bf16* tiles = kind == 0 ? p.ax_t : (kind == 1 ? p.aa_t : p.ah_t);
-  const float* fop = kind == 0 ? p.ax_f : (kind == 1 ? p.aa_f : p.ah_f);
-  const int ld = kind == 0 ? p.ld_x : (kind == 1 ? p.ld_a : p.ld_h);
-  uint8_t* ring = sm.ring[warp];
   constexpr int R = 8 * G;
   constexpr int NMT = MT == 0 ? 1 : MT;
   float acc[G][NMT][4];
@@ -523,54 +573,29 @@ __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDes
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[j][mt][e] = 0.f;
 
-  // the warp's k blocks in order: (stage s, block kb), kb = warp + 8i < 2 * chunks(s)
-  auto nblk = [&](int s) { return 2 * ((min(kc, K - s * kc) + kBoxCols - 1) / kBoxCols); };
-  auto kgroup = [&](int s, int kb) { return s * (kc / 8) + 8 * (kb >> 1) + 2 * tq + (kb & 1); };
-  auto advance = [&](int& s, int& kb) {
-    kb += kConsumerWarps;
-    while (s < nst && kb >= nblk(s)) { ++s; kb = warp; }
-  };
-  // operand prefetch: block j's operand sits in ring entry j % Q, fetched Q - 1 blocks ahead
-  int ps = 0, pkb = warp, fetched = 0, used = 0;
-  while (ps < nst && pkb >= nblk(ps)) ++ps;
-  if (!ab) {
-#pragma unroll
-    for (int i = 0; i < Q - 1; ++i) {
-      if (ps < nst) fetch_opnd<MT>(p, ring, fetched % Q, tiles, fop, ld, kgroup(ps, pkb), g, lane);
-      cp_async_commit();
-      ++fetched;
-      advance(ps, pkb);
-    }
-  }
-
   for (int s = 0; s < nst; ++s, ++stage) {
     const int slot = stage % kNumSlots;
     const uint32_t par = (stage / kNumSlots) & 1;
-    if (!ab) ab = !mbar_wait_warp(p, &sm.full[slot], par, (p.trace && threadIdx.x == 0) ? &sm.wait_cyc : nullptr);
+    unsigned long long* wacc = (p.trace && threadIdx.x == 0) ? &sm.wait_cyc : nullptr;
+    if (!ab) ab = !mbar_wait_warp(p, &sm.wfull[slot], par, wacc);
+    if (!ab) ab = !mbar_wait_warp(p, &sm.ofull[slot], par, wacc);
     if (ab) continue;
     const long long tc0 = (p.trace && threadIdx.x == 0) ? clock64() : 0ll;
     const uint8_t* tile = sm.pool[slot];
-    const int nb = nblk(s);
+    const uint8_t* opnd = tile + (size_t)R * kc * 2;
+    const int nb = 2 * ((min(kc, K - s * kc) + kBoxCols - 1) / kBoxCols);
     for (int kb = warp; kb < nb; kb += kConsumerWarps) {
-      if constexpr (MT == 0) __syncwarp();  // every lane has read the entry the next copy overwrites
-      if (ps < nst) fetch_opnd<MT>(p, ring, fetched % Q, tiles, fop, ld, kgroup(ps, pkb), g, lane);
-      cp_async_commit();
-      ++fetched;
-      advance(ps, pkb);
-      cp_async_wait<Q - 1>();  // the group of block `used` has landed
       const uint8_t* chunk = tile + (size_t)(kb >> 1) * (R * 128) + ((((2 * tq + (kb & 1)) ^ g)) << 4);
-      uint4 A[NQ];
+      uint4 A[2 * NMT];
       if constexpr (MT == 0) {
-        __syncwarp();  // lanes g = 0, 1 copied what all 8 lanes of their tq read
-        const uint8_t* ab_ = ring + ((size_t)(used % Q) * 4 + tq) * 32;
-        A[0] = *reinterpret_cast<const uint4*>(ab_);
-        A[1] = *reinterpret_cast<const uint4*>(ab_ + 16);
+        const uint8_t* ap = opnd + (size_t)kb * 128 + tq * 32;
+        A[0] = *reinterpret_cast<const uint4*>(ap);
+        A[1] = *reinterpret_cast<const uint4*>(ap + 16);
       } else {
-        const uint8_t* ab_ = ring + (size_t)(used % Q) * NQ * 512 + lane * 16;
 #pragma unroll
-        for (int q = 0; q < NQ; ++q) A[q] = *reinterpret_cast<const uint4*>(ab_ + q * 512);
+        for (int q = 0; q < 2 * MT; ++q)
+          A[q] = *reinterpret_cast<const uint4*>(opnd + (size_t)q * kc * 16 + (size_t)kb * 512 + lane * 16);
       }
-      ++used;
 #pragma unroll
       for (int j = 0; j < G; ++j) {
         const uint4 w = *reinterpret_cast<const uint4*>(chunk + (8 * j + g) * 128);
@@ -596,7 +621,6 @@ __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDes
     if (p.trace && threadIdx.x == 0) sm.tm[0] += (unsigned long long)(clock64() - tc0);
   }
 
-  cp_async_wait<0>();  // no copy into the ring may be in flight past this task
   // cross-warp reduction, one 8-row batch tile at a time: red[warp][block][batch g][8 rows]
   const long long tr0 = (p.trace && threadIdx.x == 0) ? clock64() : 0ll;
   float* red = sm.red;
@@ -889,7 +913,7 @@ __device__ __noinline__ void attn_task(const KParams& p, Smem& sm, const TaskDes
     const int ns = (a.t1 - a.t0 + T - 1) / T;
     for (int k = 0; k < ns; ++k, ++stage, ++ks) {
       const int slot = stage % kNumSlots;
-      if (!ab) ab = !mbar_wait_warp(p, &sm.full[slot], (stage / kNumSlots) & 1, tr ? &sm.wait_cyc : nullptr);
+      if (!ab) ab = !mbar_wait_warp(p, &sm.wfull[slot], (stage / kNumSlots) & 1, tr ? &sm.wait_cyc : nullptr);
       const int g0 = a.t0 + k * T + 16 * grp;  // first token of this warp's group
       const int nv = min(16, a.t1 - g0);        // valid tokens in the group (<= 0: none)
       if (!ab && (int)(ks % NG) == wsel && nv > 0) {
@@ -1162,7 +1186,8 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNumSlots; ++s) {
-      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.wfull[s], 1);
+      mbar_init(&sm.ofull[s], 1);
       mbar_init(&sm.empty[s], kConsumerWarps);
     }
     fence_mbar_init();
@@ -1184,7 +1209,9 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
   __syncthreads();
   if (sm.bad) return;
   const uint32_t o0 = p.task_off[blockIdx.x], o1 = p.task_off[blockIdx.x + 1];
-  if ((threadIdx.x >> 5) == kConsumerWarps) producer(p, sm, p.tasks + o0, (int)(o1 - o0));
+  const int warp = threadIdx.x >> 5;
+  if (warp == kConsumerWarps) producer(p, sm, p.tasks + o0, (int)(o1 - o0));
+  else if (warp == kConsumerWarps + 1) operand_loader(p, sm, p.tasks + o0, (int)(o1 - o0));
   else consumer(p, sm, p.tasks + o0, (int)(o1 - o0));
 }
 

@@ -330,7 +330,7 @@ int validate_plan(const mk_plan_s& p, std::string* err) {
           return MK_ERR_SCHEDULE_INVALID;
         }
         if (t.kc < kBoxCols || t.kc % kBoxCols || t.kc > round_up(K, kBoxCols) ||
-            (long long)rows * t.kc * 2 > kSlotBytes || ((t.kc / 32) % kConsumerWarps != 0 && t.kc < K)) {
+            (long long)t.kc * (rows * 2 + operand_col_bytes(p.cfg.max_batch)) > kSlotBytes) {
           set_err(err, "sm %d task %zu: stage of %d rows x %d columns does not fit a %d-byte slot", sm, k,
                   rows, t.kc, kSlotBytes);
           return MK_ERR_SCHEDULE_INVALID;
