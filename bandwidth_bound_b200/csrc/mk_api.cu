@@ -268,6 +268,9 @@ MK_API int mk_create_from_plan(mk_plan_t plan, const mk_weight_ptrs* w, int32_t 
   const size_t o_ssq = take(sizeof(float) * mk::num_ssq_inst(G.L) * ssq_stride);
   const size_t o_part = take(sizeof(float) * (size_t)mb * G.nkv * mk::kMaxChunksPerSeq * G.g * (G.hd + 2));
   const size_t o_lm = take(sizeof(float2) * (size_t)plan->n_lm_tasks * mb);
+  const int nsplit = plan->max_split_ids > 0 ? plan->max_split_ids : 1;
+  const size_t o_spart = take(sizeof(float) * (size_t)nsplit * mk::kMaxPieces * mk::kMaxBlocks * 8 * mb);
+  const size_t o_scnt = take(sizeof(uint32_t) * (size_t)nsplit);
   const size_t o_ctr = take(sizeof(uint32_t) * mk::num_counters(G.L));
   const size_t o_cmb = take(sizeof(uint32_t) * (size_t)G.L * mb * G.nkv);
   const size_t o_ctl = take(sizeof(uint32_t) * 2);
@@ -333,6 +336,9 @@ MK_API int mk_create_from_plan(mk_plan_t plan, const mk_weight_ptrs* w, int32_t 
   k.ld_x = ld_x; k.ld_a = ld_a; k.ld_h = ld_h;
   k.ssq = (float*)(A + o_ssq); k.ssq_stride = ssq_stride; k.part = (float*)(A + o_part);
   k.lmpart = (float2*)(A + o_lm);
+  k.spart = (float*)(A + o_spart);
+  k.scnt = (uint32_t*)(A + o_scnt);
+  k.n_split = nsplit;
   k.ctr = (uint32_t*)(A + o_ctr); k.cmb = (uint32_t*)(A + o_cmb); k.ctl = (uint32_t*)(A + o_ctl);
   k.host_status = dev_status;
   k.rope = (const float2*)(A + o_rope);
@@ -454,6 +460,7 @@ MK_API int mk_reset(mk_handle_t h) {
   MK_CUDA(h, cudaMemset(k.ctr, 0, sizeof(uint32_t) * mk::num_counters(k.L)));
   MK_CUDA(h, cudaMemset(k.cmb, 0, sizeof(uint32_t) * (size_t)k.L * k.max_b * k.nkv));
   MK_CUDA(h, cudaMemset(k.ctl, 0, sizeof(uint32_t) * 2));
+  MK_CUDA(h, cudaMemset(k.scnt, 0, sizeof(uint32_t) * k.n_split));
   MK_CUDA(h, cudaDeviceSynchronize());
   *(volatile int*)h->host_status = 0;
   h->epoch = 0;
@@ -622,6 +629,9 @@ int static_setup(StaticState& s, const mk_model_cfg& c, const mk_weight_ptrs* w,
   const size_t o_ssq = take(sizeof(float) * mk::num_ssq_inst(G.L) * ssq_stride);
   const size_t o_part = take(sizeof(float) * (size_t)mb * G.nkv * mk::kMaxChunksPerSeq * G.g * (G.hd + 2));
   const size_t o_lm = take(sizeof(float2) * (size_t)plan.n_lm_tasks * mb);
+  const int nsplit = plan.max_split_ids > 0 ? plan.max_split_ids : 1;
+  const size_t o_spart = take(sizeof(float) * (size_t)nsplit * mk::kMaxPieces * mk::kMaxBlocks * 8 * mb);
+  const size_t o_scnt = take(sizeof(uint32_t) * (size_t)nsplit);
   const size_t o_ctr = take(sizeof(uint32_t) * mk::num_counters(G.L));
   const size_t o_cmb = take(sizeof(uint32_t) * (size_t)G.L * mb * G.nkv);
   const size_t o_ctl = take(sizeof(uint32_t) * 2);
@@ -688,6 +698,9 @@ int static_setup(StaticState& s, const mk_model_cfg& c, const mk_weight_ptrs* w,
   k.ld_x = ld_x; k.ld_a = ld_a; k.ld_h = ld_h;
   k.ssq = (float*)(A + o_ssq); k.ssq_stride = ssq_stride; k.part = (float*)(A + o_part);
   k.lmpart = (float2*)(A + o_lm);
+  k.spart = (float*)(A + o_spart);
+  k.scnt = (uint32_t*)(A + o_scnt);
+  k.n_split = nsplit;
   k.ctr = (uint32_t*)(A + o_ctr); k.cmb = (uint32_t*)(A + o_cmb); k.ctl = (uint32_t*)(A + o_ctl);
   k.host_status = (int*)(A + o_status);
   k.rope = (const float2*)(A + o_rope);
@@ -712,6 +725,7 @@ cudaError_t static_clear(StaticState& s, cudaStream_t stream) {
   cudaError_t ce = cudaMemsetAsync(k.ctr, 0, sizeof(uint32_t) * mk::num_counters(k.L), stream);
   if (ce == cudaSuccess) ce = cudaMemsetAsync(k.cmb, 0, sizeof(uint32_t) * (size_t)k.L * k.max_b * k.nkv, stream);
   if (ce == cudaSuccess) ce = cudaMemsetAsync(k.ctl, 0, sizeof(uint32_t) * 2, stream);
+  if (ce == cudaSuccess) ce = cudaMemsetAsync(k.scnt, 0, sizeof(uint32_t) * k.n_split, stream);
   if (ce == cudaSuccess) ce = cudaMemsetAsync(s.status, 0, sizeof(int), stream);
   return ce;
 }

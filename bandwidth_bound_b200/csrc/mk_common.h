@@ -45,7 +45,16 @@ enum Op : uint8_t {
   OP_LMHEAD = 7,  // logits = Wlm xn; unit: 8 rows of the LM head
 };
 
-struct TaskDesc {          // 24 bytes, read by every thread of the CTA
+// A GEMV task group may be cut along K into up to kMaxPieces pieces; split tag = id << 4 |
+// piece << 2 | (pieces - 1), id = the group's K-piece partial slot.
+constexpr uint16_t kNoSplit = 0xFFFF;
+constexpr int kMaxPieces = 4;
+MK_HD uint16_t split_tag(int id, int piece, int pieces) { return (uint16_t)((id << 4) | (piece << 2) | (pieces - 1)); }
+MK_HD int split_id(uint16_t s) { return s >> 4; }
+MK_HD int split_piece(uint16_t s) { return (s >> 2) & 3; }
+MK_HD int split_pieces(uint16_t s) { return (s & 3) + 1; }
+
+struct TaskDesc {          // 32 bytes, read by every thread of the CTA
   uint8_t op;
   uint8_t nunits;          // work units covered: [u0, u0 + nunits)
   uint16_t layer;
@@ -55,6 +64,9 @@ struct TaskDesc {          // 24 bytes, read by every thread of the CTA
   uint16_t wait_ctr;       // counter to wait on before reading activations (kNoCounter: none)
   uint16_t sig_ctr;        // counter this task adds one to when it is done
   uint32_t wait_count;     // signals per step the wait needs: target = wait_count * epoch
+  uint16_t k0, k1;         // GEMV: the 64-column chunks [k0, k1) of K the task covers
+  uint16_t split;          // kNoSplit, or split_tag(id, piece, pieces) for a K piece of a task group
+  uint16_t slot0;          // per-task partial slot the task group's result goes to (piece 0's task_idx)
 };
 
 // ---- counters ---------------------------------------------------------------------------

@@ -333,20 +333,28 @@ __device__ int attn_setup(const KParams& p) {
 // projection), 2 SwiGLU output (down projection).
 __device__ __forceinline__ int operand_kind(int op) { return op == OP_OPROJ ? 1 : (op == OP_DOWN ? 2 : 0); }
 
-// Pool stages of a GEMV task: K / kc.
+// The K columns [kbeg, kend) a GEMV task covers: all of K, or one K piece of a unit.
+__device__ __forceinline__ void gemv_krange(const KParams& p, const TaskDesc& t, int& kbeg, int& kend) {
+  kbeg = (int)t.k0 * kBoxCols;
+  kend = min((int)t.k1 * kBoxCols, gemv_K_dev(p, t.op));
+}
+
+// Pool stages of a GEMV task: its columns / kc.
 __device__ __forceinline__ int gemv_stages(const KParams& p, const TaskDesc& t) {
   if (t.op == OP_EMBED) return 0;
-  const int K = gemv_K_dev(p, t.op);
-  return (K + t.kc - 1) / t.kc;
+  int kbeg, kend;
+  gemv_krange(p, t, kbeg, kend);
+  return (kend - kbeg + t.kc - 1) / t.kc;
 }
 
 // Weights of stage s of GEMV task t into slot `slot`: one tiled box per 64 columns.
 __device__ void issue_weights(const KParams& p, Smem& sm, const TaskDesc& t, int s, int slot, uint64_t pol) {
   const int lane = threadIdx.x & 31;
-  const int K = gemv_K_dev(p, t.op);
+  int kbeg, kend;
+  gemv_krange(p, t, kbeg, kend);
   const int R = t.nunits * rows_per_unit(t.op);
-  const int kc0 = s * t.kc;
-  const int nch = (min((int)t.kc, K - kc0) + kBoxCols - 1) / kBoxCols;
+  const int kc0 = kbeg + s * t.kc;
+  const int nch = (min((int)t.kc, kend - kc0) + kBoxCols - 1) / kBoxCols;
   if (lane == 0) mbar_expect_tx(&sm.wfull[slot], (uint32_t)(nch * R * 128));
   __syncwarp();
   for (int c = lane; c < nch; c += 32)
@@ -478,15 +486,16 @@ __device__ void operand_loader(const KParams& p, Smem& sm, const TaskDesc* ts, i
       }
     }
     const int kind = operand_kind(t.op);
-    const int K = gemv_K_dev(p, t.op);
+    int kbeg, kend;
+    gemv_krange(p, t, kbeg, kend);
     const int R = t.nunits * rows_per_unit(t.op);
     const int nst = gemv_stages(p, t);
     for (int ws = 0; ws < nst; ++ws, ++wk) {
       const int slot = wk % kNumSlots;
       if (!mbar_wait_warp(p, &sm.empty[slot], ((wk / kNumSlots) & 1) ^ 1)) { fail = true; break; }
       uint8_t* dst = sm.pool[slot] + (size_t)R * t.kc * 2;
-      const int k0 = ws * t.kc;
-      const int nch = (min((int)t.kc, K - k0) + kBoxCols - 1) / kBoxCols;
+      const int k0 = kbeg + ws * t.kc;
+      const int nch = (min((int)t.kc, kend - k0) + kBoxCols - 1) / kBoxCols;
       if (p.b == 1) {
         if (lane == 0) mbar_expect_tx(&sm.ofull[slot], (uint32_t)nch * 256u);
         __syncwarp();
@@ -560,9 +569,10 @@ template <int MT, int G>
 __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDesc t, uint32_t& stage, bool& ab) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, tq = lane & 3;
-  const int K = gemv_K_dev(p, t.op);
+  int kbeg, kend;
+  gemv_krange(p, t, kbeg, kend);
   const int kc = t.kc;
-  const int nst = (K + kc - 1) / kc;
+  const int nst = (kend - kbeg + kc - 1) / kc;
   constexpr int R = 8 * G;
   constexpr int NMT = MT == 0 ? 1 : MT;
   float acc[G][NMT][4];
@@ -583,7 +593,7 @@ __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDes
     const long long tc0 = (p.trace && threadIdx.x == 0) ? clock64() : 0ll;
     const uint8_t* tile = sm.pool[slot];
     const uint8_t* opnd = tile + (size_t)R * kc * 2;
-    const int nb = 2 * ((min(kc, K - s * kc) + kBoxCols - 1) / kBoxCols);
+    const int nb = 2 * ((min(kc, kend - kbeg - s * kc) + kBoxCols - 1) / kBoxCols);
     for (int kb = warp; kb < nb; kb += kConsumerWarps) {
       const uint8_t* chunk = tile + (size_t)(kb >> 1) * (R * 128) + ((((2 * tq + (kb & 1)) ^ g)) << 4);
       uint4 A[2 * NMT];
@@ -702,6 +712,53 @@ __device__ void gemv_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_
 
   const int nthr = kConsumerWarps * 32;
   const int n = t.nunits;
+  if (t.split != kNoSplit) {
+    // one of the K pieces of a task group: publish this piece's sums; the last piece to
+    // arrive adds all pieces' sums in piece order (the same order whoever arrives last) and
+    // runs the epilogue, the others only clear their per-task partial slots
+    const int rows = 8 * G;
+    const int id = split_id(t.split), np = split_pieces(t.split);
+    const size_t stride = (size_t)kMaxBlocks * 8 * p.max_b;  // floats per piece
+    float* base = p.spart + (size_t)id * kMaxPieces * stride;
+    if (!ab)
+      for (int idx = threadIdx.x; idx < rows * p.b; idx += nthr) {
+        const int bi = idx % p.b, row = idx / p.b;
+        __stcg(base + split_piece(t.split) * stride + (size_t)row * p.max_b + bi, sm.ep[row][bi]);
+      }
+    cbar();
+    if (threadIdx.x == 0) {
+      int last = 0;
+      if (!ab) {
+        __threadfence();
+        const uint32_t old = atom_add_acqrel(p.scnt + id, 1u);
+        last = old + 1u == (uint32_t)np ? 1 : 0;
+        if (last) p.scnt[id] = 0u;  // ready for the next phase
+      }
+      sm.flag2 = last;
+    }
+    cbar();
+    if (!sm.flag2) {
+      if (!ab && (t.op == OP_OPROJ || t.op == OP_DOWN)) {
+        const int inst = t.op == OP_OPROJ ? ssq_inst_oproj(t.layer) : ssq_inst_down(t.layer);
+        for (int bi = threadIdx.x; bi < p.b; bi += nthr)
+          p.ssq[(size_t)inst * p.ssq_stride + (size_t)t.task_idx * p.max_b + bi] = 0.f;
+      }
+      if (!ab && t.op == OP_LMHEAD && p.argmax)
+        for (int bi = threadIdx.x; bi < p.b; bi += nthr)
+          p.lmpart[(size_t)t.task_idx * p.max_b + bi] = make_float2(-INFINITY, __int_as_float(0x7fffffff));
+      if (p.trace && threadIdx.x == 0) sm.tm[2] += (unsigned long long)(clock64() - te0);
+      return;
+    }
+    if (!ab)
+      for (int idx = threadIdx.x; idx < rows * p.b; idx += nthr) {
+        const int bi = idx % p.b, row = idx / p.b;
+        const float* src = base + (size_t)row * p.max_b + bi;
+        float v = __ldcg(src);
+        for (int q = 1; q < np; ++q) v += __ldcg(src + q * stride);
+        sm.ep[row][bi] = v;
+      }
+    cbar();
+  }
   if (t.op == OP_QKV) {
     if (!ab) {
       const int half = p.hd / 2, per_head = p.hd >> 4;
@@ -777,7 +834,9 @@ __device__ void gemv_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_
         for (int row = lane; row < 8 * n; row += 32) s += sm.ep[row][bi] * sm.ep[row][bi];
 #pragma unroll
         for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (lane == 0) p.ssq[(size_t)inst * p.ssq_stride + (size_t)t.task_idx * p.max_b + bi] = s;
+        // a K-split group's sum always goes to piece 0's slot: the 1/rms reduction then adds
+        // the same values in the same order whichever piece finished last
+        if (lane == 0) p.ssq[(size_t)inst * p.ssq_stride + (size_t)t.slot0 * p.max_b + bi] = s;
       }
     }
   } else {  // LM head

@@ -42,6 +42,9 @@ struct KParams {
   int ld_x, ld_a, ld_h;
   int ssq_stride;            // floats per ssq instance
   float2* lmpart;            // [n_lm_tasks][max_b] (value, index bits)
+  float* spart;              // K-piece partial sums [split id][kMaxPieces][64 rows][max_b]
+  uint32_t* scnt;            // K-piece arrival counters [split id]
+  int n_split;               // split ids (entries of scnt)
   uint32_t *ctr, *cmb, *ctl; // counters, split-K combine counters, {abort, status}
   int* host_status;          // mapped host word
   const float2* rope;        // [max_ctx][hd/2] (cos, sin)

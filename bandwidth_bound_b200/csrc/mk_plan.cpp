@@ -5,10 +5,11 @@
 // a static validator proves the schedule deadlock-free and race-free before it
 // runs; "Inside the megakernel serving engine": idle SMs take ready work instead
 // of waiting on a wave) is realised here as plain host code:
-//  * every phase (embed, per layer qkv / attn / oproj / gateup / down, lm head)
-//    is cut into fixed work units; each SM gets a contiguous range of units, and
-//    the SMs that carry the extra unit of a phase are the ones with the least
-//    cumulative weight bytes so far, so that bytes stay balanced over the step;
+//  * every GEMV phase (per layer qkv / oproj / gateup / down, lm head) is cut into
+//    equal ranges of (unit, 64-column chunk) work, one per SM, because each phase
+//    ends at a counter that every SM waits on: its slowest SM sets the pace.  A unit
+//    that a range boundary cuts becomes two K pieces whose partial sums the second
+//    to finish adds; the attention phase is cut into equal token ranges at run time;
 //  * each task waits on exactly one counter (all tasks of the phase it reads)
 //    and adds one to its own phase's counter.
 #include "mk_plan.h"
@@ -20,6 +21,9 @@
 #include <numeric>
 
 namespace mk {
+
+// GEMV phases with less than this many weight bytes per SM keep whole units per task.
+constexpr long long kSplitMinBytes = 512 * 1024;
 
 Geometry geometry(const mk_model_cfg& c) {
   Geometry G;
@@ -192,53 +196,159 @@ int build_plan(const mk_model_cfg& c, const mk_plan_opts* opts, mk_plan_s* P, st
           t.sig_ctr = (uint16_t)sig;
           P->streams[sm].push_back(t);
         }
-    } else {
+    } else if (op == OP_EMBED) {
       const int U = phase_units(G, op);
-      const long long ub = unit_weight_bytes(G, op);
-      const int rpu = op == OP_EMBED ? 8 : rows_per_unit(op);
-      const int max_u = op == OP_EMBED ? 255 : std::max(1, std::min(max_units(op), P->max_blocks * 8 / rpu));
-      // QKV tasks stay inside one head (their weight rows form one TMA box)
-      const int seg = op == OP_QKV ? G.hd / 16 : U;
-      // units per SM: base, and +1 for the 'extra' SMs with the least bytes so far
-      std::vector<int> cnt(nsm, U / nsm);
-      int extra = U % nsm;
-      if (extra) {
-        std::vector<int> idx(nsm);
-        std::iota(idx.begin(), idx.end(), 0);
-        std::stable_sort(idx.begin(), idx.end(), [&](int a, int b) { return cum[a] < cum[b]; });
-        for (int k = 0; k < extra; ++k) cnt[idx[k]]++;
-      }
-      int u = 0;
-      for (int sm = 0; sm < nsm; ++sm) {
-        const int n = cnt[sm];
+      for (int sm = 0, u = 0; sm < nsm; ++sm) {
+        const int n = U / nsm + (sm < U % nsm ? 1 : 0);
         if (n == 0) continue;
-        // cut [u, u + n) at segment boundaries, then into near-equal tasks of <= max_u units
-        int a = u;
-        const int end = u + n;
-        while (a < end) {
-          const int b = std::min(end, (a / seg + 1) * seg);
-          const int len = b - a;
-          const int ntask = (len + max_u - 1) / max_u;
-          int v = a;
-          for (int k = 0; k < ntask; ++k) {
-            const int nk = len / ntask + (k < len % ntask ? 1 : 0);
-            TaskDesc t{};
-            t.op = (uint8_t)op;
-            t.nunits = (uint8_t)nk;
-            t.layer = (uint16_t)l;
-            t.u0 = (uint32_t)v;
-            t.task_idx = (uint16_t)tidx++;
-            t.kc = op == OP_EMBED ? 0 : (uint16_t)stage_cols(nk * rpu / 8, gemv_K(G, op), c.max_batch);
-            t.wait_ctr = (uint16_t)wc;
-            t.wait_count = wcount;
-            t.sig_ctr = (uint16_t)sig;
-            P->streams[sm].push_back(t);
-            v += nk;
-          }
-          a = b;
+        TaskDesc t{};
+        t.op = (uint8_t)op;
+        t.nunits = (uint8_t)n;
+        t.u0 = (uint32_t)u;
+        t.task_idx = (uint16_t)tidx++;
+        t.wait_ctr = (uint16_t)wc;
+        t.sig_ctr = (uint16_t)sig;
+        t.split = kNoSplit;
+        t.slot0 = t.task_idx;
+        P->streams[sm].push_back(t);
+        u += n;
+      }
+    } else {
+      // GEMV phase: units are grouped into tasks of <= max_u units (QKV groups inside one
+      // head); the work is the line of (group, 64-column chunk) pairs weighted by the group's
+      // units, cut into equal ranges, one per SM.  A group that a cut falls into becomes K
+      // pieces (<= kMaxPieces), each with all of the group's rows; the last piece to finish
+      // adds the partial sums.
+      const int U = phase_units(G, op);
+      const int K = gemv_K(G, op);
+      const int nkb = (K + kBoxCols - 1) / kBoxCols;
+      const int rpu = rows_per_unit(op);
+      // groups small enough that every SM gets work and no group needs more than kMaxPieces
+      const int max_u = std::max(1, std::min({max_units(op), P->max_blocks * 8 / rpu, (kMaxPieces - 1) * U / nsm}));
+      const int seg = op == OP_QKV ? G.hd / 16 : U;
+      std::vector<std::pair<int, int>> groups;  // (u0, n)
+      for (int x = 0; x < U;) {
+        const int y = std::min(U, (x / seg + 1) * seg);
+        const int len = y - x, ng = (len + max_u - 1) / max_u;
+        for (int k = 0, v = x; k < ng; ++k) {
+          const int nk = len / ng + (k < len % ng ? 1 : 0);
+          groups.push_back({v, nk});
+          v += nk;
         }
-        u = end;
-        cum[sm] += (long long)n * ub;
+        x = y;
+      }
+      const long long W = (long long)U * nkb;
+      if ((long long)U * unit_weight_bytes(G, op) / nsm < kSplitMinBytes) {
+        // a small phase: whole units only (split pieces would add more fixed cost per task than
+        // they save), each SM a contiguous range of U / nsm or U / nsm + 1 units cut into
+        // tasks of <= max_units units inside head segments
+        const int mu = std::max(1, std::min(max_units(op), P->max_blocks * 8 / rpu));
+        // the extra units of the phase go to the SMs with the fewest bytes so far
+        std::vector<int> cnt(nsm, U / nsm), idx(nsm);
+        std::iota(idx.begin(), idx.end(), 0);
+        std::stable_sort(idx.begin(), idx.end(), [&](int a2, int b2) { return cum[a2] < cum[b2]; });
+        for (int k = 0; k < U % nsm; ++k) cnt[idx[k]]++;
+        for (int sm = 0, u = 0; sm < nsm; ++sm) {
+          const int n = cnt[sm];
+          for (int a = u, end = u + n; a < end;) {
+            const int b = std::min(end, (a / seg + 1) * seg);
+            const int len = b - a, ntask = (len + mu - 1) / mu;
+            for (int k = 0, v = a; k < ntask; ++k) {
+              const int nk = len / ntask + (k < len % ntask ? 1 : 0);
+              TaskDesc t{};
+              t.op = (uint8_t)op;
+              t.nunits = (uint8_t)nk;
+              t.layer = (uint16_t)l;
+              t.u0 = (uint32_t)v;
+              t.task_idx = (uint16_t)tidx++;
+              t.slot0 = t.task_idx;
+              t.k0 = 0;
+              t.k1 = (uint16_t)nkb;
+              t.split = kNoSplit;
+              t.kc = (uint16_t)stage_cols(nk * rpu / 8, K, c.max_batch);
+              t.wait_ctr = (uint16_t)wc;
+              t.wait_count = wcount;
+              t.sig_ctr = (uint16_t)sig;
+              P->streams[sm].push_back(t);
+              cum[sm] += (long long)nk * unit_weight_bytes(G, op);
+              v += nk;
+            }
+            a = b;
+          }
+          u += n;
+        }
+      } else {
+      const long long gmax = (long long)max_u * nkb;
+      // ranges long enough that no group falls into more than kMaxPieces of them
+      const int nuse = (int)std::max<long long>(1, std::min<long long>(nsm, W * (kMaxPieces - 1) / gmax));
+      std::vector<long long> cut(nuse + 1);
+      {
+        // cuts at chunk boundaries of the group they fall into
+        long long pos = 0;
+        size_t gi = 0;
+        cut[0] = 0;
+        for (int s2 = 1; s2 < nuse; ++s2) {
+          const long long want = W * s2 / nuse;
+          while (gi < groups.size() && pos + (long long)groups[gi].second * nkb <= want) {
+            pos += (long long)groups[gi].second * nkb;
+            ++gi;
+          }
+          const long long within = want - pos;  // inside group gi
+          const int n = gi < groups.size() ? groups[gi].second : 1;
+          cut[s2] = pos + (within / n) * n;
+        }
+        cut[nuse] = W;
+      }
+      // per group: its start on the line, and the ranges (pieces) it falls into
+      std::vector<long long> gstart(groups.size() + 1, 0);
+      for (size_t g = 0; g < groups.size(); ++g) gstart[g + 1] = gstart[g] + (long long)groups[g].second * nkb;
+      int next_id = 0;
+      std::vector<int> gid(groups.size(), -1), gpieces(groups.size(), 1), gslot0(groups.size(), 0);
+      for (size_t g = 0; g < groups.size(); ++g) {
+        int np = 0;
+        for (int s2 = 0; s2 < nuse; ++s2)
+          if (cut[s2] < gstart[g + 1] && cut[s2 + 1] > gstart[g]) ++np;
+        gpieces[g] = np;
+        if (np > 1) gid[g] = next_id++;
+      }
+      for (int s2 = 0; s2 < nuse; ++s2) {
+        const long long a = cut[s2], b = cut[s2 + 1];
+        if (a >= b) continue;
+        for (size_t g = 0; g < groups.size(); ++g) {
+          if (gstart[g + 1] <= a || gstart[g] >= b) continue;
+          const int n = groups[g].second;
+          const int k0 = (int)((std::max(a, gstart[g]) - gstart[g]) / n);
+          const int k1 = (int)((std::min(b, gstart[g + 1]) - gstart[g]) / n);
+          if (k0 >= k1) continue;
+          TaskDesc t{};
+          t.op = (uint8_t)op;
+          t.nunits = (uint8_t)n;
+          t.layer = (uint16_t)l;
+          t.u0 = (uint32_t)groups[g].first;
+          t.task_idx = (uint16_t)tidx++;
+          t.k0 = (uint16_t)k0;
+          t.k1 = (uint16_t)k1;
+          t.slot0 = t.task_idx;
+          if (gpieces[g] > 1) {
+            int piece = 0;
+            for (int s3 = 0; s3 < s2; ++s3)
+              if (cut[s3] < gstart[g + 1] && cut[s3 + 1] > gstart[g] && cut[s3] < cut[s3 + 1]) ++piece;
+            t.split = split_tag(gid[g], piece, gpieces[g]);
+            if (piece == 0) gslot0[g] = t.task_idx;  // pieces are made in K order: piece 0 first
+            t.slot0 = (uint16_t)gslot0[g];
+          } else {
+            t.split = kNoSplit;
+          }
+          const int cols = std::min(k1 * kBoxCols, K) - k0 * kBoxCols;
+          t.kc = (uint16_t)stage_cols(n * rpu / 8, cols, c.max_batch);
+          t.wait_ctr = (uint16_t)wc;
+          t.wait_count = wcount;
+          t.sig_ctr = (uint16_t)sig;
+          P->streams[s2].push_back(t);
+          cum[s2] += (long long)n * rpu * cols * 2;
+        }
+      }
+      P->max_split_ids = std::max(P->max_split_ids, next_id);
       }
     }
     phase_tasks[pi] = tidx;
@@ -257,14 +367,14 @@ namespace {
 
 // X: fp32 residual; AX: its normalised-gain operand for the next GEMV; AA: attention
 // output operand; AH: SwiGLU output operand.
-enum Buf { B_X, B_Q, B_ATTN, B_H, B_PART, B_LOGITS, B_LMPART, B_KVNEW, B_SSQ, B_AX };
+enum Buf { B_X, B_Q, B_ATTN, B_H, B_PART, B_LOGITS, B_LMPART, B_KVNEW, B_SSQ, B_AX, B_SPLIT };
 
 struct Access {
   int buf, inst;   // inst: layer for KVNEW, ssq instance for SSQ, 0 otherwise
   bool write;
 };
 
-std::vector<Access> accesses(int op, int l, int L) {
+std::vector<Access> accesses_of_phase(int op, int l, int L) {
   switch (op) {
     case OP_EMBED: return {{B_X, 0, true}, {B_AX, 0, true}, {B_SSQ, ssq_inst_embed(), true}};
     case OP_QKV:
@@ -280,6 +390,12 @@ std::vector<Access> accesses(int op, int l, int L) {
       return {{B_AX, 0, false}, {B_SSQ, ssq_inst_down(L - 1), false}, {B_LOGITS, 0, true}, {B_LMPART, 0, true}};
   }
   return {};
+}
+
+std::vector<Access> accesses(int op, int l, int L) {
+  std::vector<Access> v = accesses_of_phase(op, l, L);
+  if (op != OP_EMBED && op != OP_ATTN) v.push_back({B_SPLIT, 0, true});  // K-piece partials and counters
+  return v;
 }
 
 }  // namespace
@@ -300,11 +416,15 @@ int validate_plan(const mk_plan_s& p, std::string* err) {
   };
   const int NP = (int)order.size();
 
-  // 1. each task well formed; units covered exactly once; stages fit a slot
+  // 1. each task well formed; units covered exactly once (a unit cut into K pieces: its two
+  // pieces tile its chunks, carry the same boundary and pieces 0 and 1); stages fit a slot
   std::vector<std::vector<int>> cover(NP);
+  struct Piece { int k0, k1, split, u0, n; };
+  std::vector<std::vector<std::vector<Piece>>> pieces(NP);
   for (int pi = 0; pi < NP; ++pi) {
     int op = order[pi].op;
     cover[pi].assign(op == OP_ATTN ? S : phase_units(G, op), 0);
+    pieces[pi].assign(cover[pi].size(), {});
   }
   std::vector<int> n_sig(nctr, 0);
   std::vector<int> phase_of_sig(nctr, -1);
@@ -321,10 +441,25 @@ int validate_plan(const mk_plan_s& p, std::string* err) {
                 t.layer, t.u0, t.u0 + t.nunits, cover[pi].size());
         return MK_ERR_SCHEDULE_INVALID;
       }
-      for (uint32_t u = t.u0; u < t.u0 + t.nunits; ++u) cover[pi][u]++;
-      if (t.op != OP_EMBED && t.op != OP_ATTN) {
+      const bool gemv = t.op != OP_EMBED && t.op != OP_ATTN;
+      const int nkb = gemv ? (gemv_K(G, t.op) + kBoxCols - 1) / kBoxCols : 0;
+      if (gemv && (t.k0 >= t.k1 || t.k1 > nkb)) {
+        set_err(err, "sm %d task %zu: K chunks [%d, %d) outside [0, %d)", sm, k, t.k0, t.k1, nkb);
+        return MK_ERR_SCHEDULE_INVALID;
+      }
+      if (gemv && (t.split != kNoSplit || t.k0 != 0 || t.k1 != nkb)) {
+        if (t.split == kNoSplit || split_id(t.split) >= p.max_split_ids) {
+          set_err(err, "sm %d task %zu: a K piece without a valid split tag", sm, k);
+          return MK_ERR_SCHEDULE_INVALID;
+        }
+        for (uint32_t u = t.u0; u < t.u0 + t.nunits; ++u)
+          pieces[pi][u].push_back({t.k0, t.k1, t.split, (int)t.u0, t.nunits});
+      } else {
+        for (uint32_t u = t.u0; u < t.u0 + t.nunits; ++u) cover[pi][u]++;
+      }
+      if (gemv) {
         const int rows = t.nunits * rows_per_unit(t.op);
-        const int K = gemv_K(G, t.op);
+        const int K = std::min((int)t.k1 * kBoxCols, gemv_K(G, t.op)) - (int)t.k0 * kBoxCols;
         if (t.nunits > max_units(t.op)) {
           set_err(err, "sm %d task %zu: %d rows exceed %d", sm, k, rows, kMaxBlocks * 8);
           return MK_ERR_SCHEDULE_INVALID;
@@ -348,13 +483,37 @@ int validate_plan(const mk_plan_s& p, std::string* err) {
       }
       n_sig[t.sig_ctr]++;
     }
-  for (int pi = 0; pi < NP; ++pi)
-    for (size_t u = 0; u < cover[pi].size(); ++u)
-      if (cover[pi][u] != 1) {
-        set_err(err, "phase op %d layer %d: unit %zu covered %d times", order[pi].op, order[pi].layer, u,
-                cover[pi][u]);
+  for (int pi = 0; pi < NP; ++pi) {
+    std::vector<long long> id_owner(p.max_split_ids, -1);  // the first unit of the group an id belongs to
+    const int op = order[pi].op;
+    const int nkb = (op != OP_EMBED && op != OP_ATTN) ? (gemv_K(G, op) + kBoxCols - 1) / kBoxCols : 0;
+    for (size_t u = 0; u < cover[pi].size(); ++u) {
+      auto& pc = pieces[pi][u];
+      bool ok = false;
+      if (pc.empty()) ok = cover[pi][u] == 1;
+      else if (cover[pi][u] == 0 && pc.size() >= 2 && pc.size() <= (size_t)kMaxPieces) {
+        // the pieces tile [0, nkb) in K order, pieces 0..P-1 of one id with P pieces
+        std::sort(pc.begin(), pc.end(), [](const Piece& a, const Piece& b) { return a.k0 < b.k0; });
+        ok = pc.front().k0 == 0 && pc.back().k1 == nkb;
+        const int id = split_id((uint16_t)pc[0].split);
+        for (size_t k2 = 0; ok && k2 < pc.size(); ++k2) {
+          const uint16_t sp = (uint16_t)pc[k2].split;
+          ok = split_id(sp) == id && split_piece(sp) == (int)k2 && split_pieces(sp) == (int)pc.size() &&
+               (k2 == 0 || pc[k2 - 1].k1 == pc[k2].k0) && pc[k2].u0 == pc[0].u0 && pc[k2].n == pc[0].n;
+        }
+        // an id names one task group (one u0) in the phase
+        if (ok) {
+          if (id_owner[id] < 0) id_owner[id] = pc[0].u0;
+          else ok = id_owner[id] == pc[0].u0;
+        }
+      }
+      if (!ok) {
+        set_err(err, "phase op %d layer %d: unit %zu covered %d times in full and by %zu K pieces that do not "
+                "pair up", order[pi].op, order[pi].layer, u, cover[pi][u], pc.size());
         return MK_ERR_SCHEDULE_INVALID;
       }
+    }
+  }
 
   // 2. every wait target is exactly the number of signals its counter gets
   for (int sm = 0; sm < nsm; ++sm)
@@ -496,9 +655,10 @@ MK_API int mk_plan_stats(mk_plan_t plan, mk_plan_info* o) {
     int64_t bytes = 0;
     for (const auto& t : s) {
       if (t.op == mk::OP_EMBED || t.op == mk::OP_ATTN) continue;
-      int K = mk::gemv_K(G, t.op);
-      o->n_stages += (K + t.kc - 1) / t.kc;
-      bytes += (int64_t)t.nunits * mk::unit_weight_bytes(G, t.op);
+      const int K = mk::gemv_K(G, t.op);
+      const int cols = std::min((int)t.k1 * mk::kBoxCols, K) - (int)t.k0 * mk::kBoxCols;
+      o->n_stages += (cols + t.kc - 1) / t.kc;
+      bytes += (int64_t)t.nunits * mk::rows_per_unit(t.op) * cols * 2;
     }
     o->weight_bytes_max_sm = std::max(o->weight_bytes_max_sm, bytes);
     if (o->weight_bytes_min_sm < 0 || bytes < o->weight_bytes_min_sm) o->weight_bytes_min_sm = bytes;

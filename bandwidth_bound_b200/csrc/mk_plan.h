@@ -15,6 +15,7 @@ struct mk_plan_s {
   std::vector<int> signalers;                      // per counter: tasks that add to it
   int max_phase_tasks = 0;                         // most tasks in one phase (scratch sizing)
   int n_lm_tasks = 0;
+  int max_split_ids = 0;                           // most K-split task groups in one phase
 };
 
 namespace mk {
