@@ -7,14 +7,16 @@
 //     stream of task descriptors;
 //   * tasks wait on dependency counters in global memory (acquire loads) and
 //     signal them (release read-modify-writes) instead of grid-wide barriers;
-//   * one producer warp streams every weight tile and every prior KV page of the
-//     CTA's whole stream into a ring of shared-memory slots with cp.async.bulk
-//     (completion on mbarriers), running ahead of the activation dependencies;
-//     eight consumer warps compute from the slots.
-// B200 choices: 1-D bulk copies (no tensor maps, no multicast) of contiguous row
-// segments, evict-first L2 policy for streamed bytes, fp32 accumulation, CUDA-core
-// FMA GEMV at batch 1, mma.sync bf16 tensor cores with hi/lo-split activations
-// at batch >= 2, split-K flash-decode with QK^T on tensor cores.
+//   * a shared-memory pool of stage slots is filled ahead of the compute: one
+//     producer warp streams every weight tile and KV page of the CTA's whole stream
+//     (they do not depend on this step's activations), one operand warp adds each
+//     GEMV stage's activation slice once the task's dependency is met, and eight
+//     consumer warps compute from the slots.
+// B200 choices: every copy is a tiled TMA box (cp.async.bulk.tensor, no multicast)
+// with completion on mbarriers; evict-first L2 policy for streamed bytes; fp32
+// accumulation; CUDA-core FMA GEMV at batch 1; mma.sync bf16 tensor cores with hi/lo
+// split activations at batch >= 2; split-K flash-decode attention with both products on
+// tensor cores (ldmatrix fragments from 128-byte-swizzled page boxes).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
