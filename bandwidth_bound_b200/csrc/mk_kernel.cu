@@ -196,6 +196,17 @@ __device__ bool mbar_wait(const KParams& p, uint64_t* bar, uint32_t parity) {
   }
 }
 
+// Non-blocking test that stage `st`'s weights and operands have both landed (lane 0).  The two
+// tests are independent, so their ~200-cycle latencies overlap; issued ahead of a stage's
+// compute, they overlap that too.
+__device__ __forceinline__ uint32_t stage_landed(Smem& sm, uint32_t st) {
+  const int slot = st % kNumSlots;
+  const uint32_t par = (st / kNumSlots) & 1;
+  const uint32_t a = mbar_test(&sm.wfull[slot], par) ? 1u : 0u;
+  const uint32_t b = mbar_test(&sm.ofull[slot], par) ? 1u : 0u;
+  return a & b;
+}
+
 // Warp-uniform variant: lane 0 waits, the result is broadcast.
 __device__ __forceinline__ bool mbar_wait_warp(const KParams& p, uint64_t* bar, uint32_t parity,
                                                unsigned long long* wait_acc = nullptr) {
@@ -585,13 +596,19 @@ __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDes
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[j][mt][e] = 0.f;
 
+  // lane 0 tests each stage's barriers one stage ahead (before the previous stage's compute);
+  // only a stage that had not landed by then takes the blocking wait
+  uint32_t ready = (lane == 0 && !ab && nst > 0) ? stage_landed(sm, stage) : 0u;
   for (int s = 0; s < nst; ++s, ++stage) {
     const int slot = stage % kNumSlots;
     const uint32_t par = (stage / kNumSlots) & 1;
-    unsigned long long* wacc = (p.trace && threadIdx.x == 0) ? &sm.wait_cyc : nullptr;
-    if (!ab) ab = !mbar_wait_warp(p, &sm.wfull[slot], par, wacc);
-    if (!ab) ab = !mbar_wait_warp(p, &sm.ofull[slot], par, wacc);
+    if (!ab && !__shfl_sync(0xffffffffu, ready, 0)) {
+      unsigned long long* wacc = (p.trace && threadIdx.x == 0) ? &sm.wait_cyc : nullptr;
+      ab = !mbar_wait_warp(p, &sm.wfull[slot], par, wacc);
+      if (!ab) ab = !mbar_wait_warp(p, &sm.ofull[slot], par, wacc);
+    }
     if (ab) continue;
+    ready = (lane == 0 && s + 1 < nst) ? stage_landed(sm, stage + 1) : 0u;
     const long long tc0 = (p.trace && threadIdx.x == 0) ? clock64() : 0ll;
     const uint8_t* tile = sm.pool[slot];
     const uint8_t* opnd = tile + (size_t)R * kc * 2;
