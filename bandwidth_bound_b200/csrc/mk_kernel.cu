@@ -545,13 +545,27 @@ __device__ void operand_loader(const KParams& p, Smem& sm, const TaskDesc* ts, i
 // ---------------------------------------------------------------------------------------
 // consumer helpers
 
-// 1/rms of each batch row from the partial sums of squares of instance `inst`.
+// 1/rms of each batch row from the partial sums of squares of instance `inst`.  Each lane
+// keeps eight loads in flight (partials lane + 32 (8 i + j) go to sum j), so a few hundred
+// partials cost one or two L2 round trips; the order of the additions is fixed.
 __device__ void compute_inv_rms(const KParams& p, Smem& sm, int inst, int nparts) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float* base = p.ssq + (size_t)inst * p.ssq_stride;
   for (int bi = warp; bi < p.b; bi += kConsumerWarps) {
-    float s = 0.f;
-    for (int k = lane; k < nparts; k += 32) s += __ldcg(base + (size_t)k * p.max_b + bi);
+    float acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+    for (int k0 = lane; k0 < nparts; k0 += 256) {
+      float v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int k = k0 + 32 * j;
+        v[j] = k < nparts ? __ldcg(base + (size_t)k * p.max_b + bi) : 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[j] += v[j];
+    }
+    float s = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
 #pragma unroll
     for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
     if (lane == 0) sm.inv_rms[bi] = 1.0f / sqrtf(s / (float)p.d + p.eps);
