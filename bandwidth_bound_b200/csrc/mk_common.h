@@ -23,8 +23,8 @@ namespace mk {
 // ---- launch geometry -------------------------------------------------------------------
 constexpr int kConsumerWarps = 8;                       // compute warps per CTA
 constexpr int kThreads = (kConsumerWarps + 2) * 32;     // + the weight/KV producer warp + the operand warp
-constexpr int kSlotBytes = 40 * 1024;                   // one pool stage: weights + their operands, or KV pages
-constexpr int kNumSlots = 5;                            // pool depth (200 KB)
+constexpr int kSlotBytes = 50 * 1024;                   // one pool stage: weights + their operands, or KV pages
+constexpr int kNumSlots = 4;                            // pool depth (200 KB; 4 x 50 KB measured fastest)
 constexpr int kMaxBatch = 16;
 constexpr int kMaxBlocks = 8;                           // 8-row blocks per GEMV task (64 rows)
 constexpr int kPage = 16;                               // tokens per KV page

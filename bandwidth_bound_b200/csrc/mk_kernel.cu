@@ -586,7 +586,7 @@ __device__ __forceinline__ void put_operand(bf16* tiles, float* f, int ld, int b
 // Slot layout of a stage: the weights (per 64-column chunk: 8*G rows of 128 bytes, 16-byte
 // pieces swizzled, piece c of row r at c ^ (r & 7)), then the stage's operands (opnd_*
 // layouts: per bf16 (tile, part) kc * 16 bytes, or kc * 4 bytes of fp32 row 0).  Warp w takes
-// 32-column k blocks w, w+8, ... of every stage; block kb is the even (h = 0) or odd (h = 1)
+// the task's 32-column k blocks w, w+8, ... (counted across stages); block kb is the even (h = 0) or odd (h = 1)
 // 16-byte pieces of chunk kb / 2, so lane (g, tq) reads piece 2*tq + h of row 8j + g -
 // conflict-free - which holds columns 16*tq + 8*h .. +7, and the operand piece of the same
 // columns at `lane` (bf16) or `tq` (fp32, shared by the 8 lanes of one tq).
@@ -627,7 +627,12 @@ __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDes
     const uint8_t* tile = sm.pool[slot];
     const uint8_t* opnd = tile + (size_t)R * kc * 2;
     const int nb = 2 * ((min(kc, kend - kbeg - s * kc) + kBoxCols - 1) / kBoxCols);
-    for (int kb = warp; kb < nb; kb += kConsumerWarps) {
+    // k block q of the task (q = s * nbs + kb) goes to warp q % 8: every warp's accumulator
+    // chain covers an eighth of K whatever the stage width (tensor-core fp32 accumulation
+    // truncates, so its error grows with the chain)
+    const int nbs = 2 * (kc / kBoxCols);
+    for (int kb = (warp + kConsumerWarps - (s * nbs) % kConsumerWarps) % kConsumerWarps; kb < nb;
+         kb += kConsumerWarps) {
       const uint8_t* chunk = tile + (size_t)(kb >> 1) * (R * 128) + ((((2 * tq + (kb & 1)) ^ g)) << 4);
       uint4 A[2 * NMT];
       if constexpr (MT == 0) {
