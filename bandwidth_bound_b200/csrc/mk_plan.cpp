@@ -5,11 +5,13 @@
 // a static validator proves the schedule deadlock-free and race-free before it
 // runs; "Inside the megakernel serving engine": idle SMs take ready work instead
 // of waiting on a wave) is realised here as plain host code:
-//  * every GEMV phase (per layer qkv / oproj / gateup / down, lm head) is cut into
-//    equal ranges of (unit, 64-column chunk) work, one per SM, because each phase
-//    ends at a counter that every SM waits on: its slowest SM sets the pace.  A unit
-//    that a range boundary cuts becomes two K pieces whose partial sums the second
-//    to finish adds; the attention phase is cut into equal token ranges at run time;
+//  * every GEMV phase (per layer qkv / oproj / gateup / down, lm head) ends at a
+//    counter that every SM waits on, so its slowest SM sets the pace.  The phase takes
+//    the cheaper, by a cost model of bytes plus a fixed cost per task and per K piece,
+//    of equal ranges of (unit, 64-column chunk) work - a unit group that a range
+//    boundary cuts becomes K pieces whose partial sums the last to finish adds - and
+//    one task per SM (row groups within one unit of each other, each cut into equal K
+//    pieces); the attention phase is cut into equal token ranges at run time;
 //  * each task waits on exactly one counter (all tasks of the phase it reads)
 //    and adds one to its own phase's counter.
 #include "mk_plan.h"
@@ -22,8 +24,24 @@
 
 namespace mk {
 
-// GEMV phases with less than this many weight bytes per SM keep whole units per task.
+// GEMV phases with less than this many weight bytes per SM keep whole units per task in the
+// equal-range partition.
 constexpr long long kSplitMinBytes = 512 * 1024;
+
+// The plan's cost model for choosing among partitions of a GEMV phase: every phase ends at
+// a counter all SMs wait on, so the estimate that matters is the slowest SM's - its weight
+// and operand bytes plus a fixed cost per task (reduction, epilogue, release, and the pool
+// standing full meanwhile; measured ~7-9 us per extra task at batch 8) and per K piece
+// (partial sums written, counted and re-read), both in byte equivalents.
+constexpr long long kTaskCostBytes = 256 * 1024;
+constexpr long long kPieceCostBytes = 96 * 1024;
+
+// One candidate partition of a GEMV phase: (SM, task) pairs in creation order (a split
+// group's piece 0 before its other pieces), task_idx and slot0 still unset; split ids 0..nids-1.
+struct Cand {
+  std::vector<std::pair<int, TaskDesc>> tasks;
+  int nids = 0;
+};
 
 Geometry geometry(const mk_model_cfg& c) {
   Geometry G;
@@ -214,142 +232,203 @@ int build_plan(const mk_model_cfg& c, const mk_plan_opts* opts, mk_plan_s* P, st
         u += n;
       }
     } else {
-      // GEMV phase: units are grouped into tasks of <= max_u units (QKV groups inside one
-      // head); the work is the line of (group, 64-column chunk) pairs weighted by the group's
-      // units, cut into equal ranges, one per SM.  A group that a cut falls into becomes K
-      // pieces (<= kMaxPieces), each with all of the group's rows; the last piece to finish
-      // adds the partial sums.
       const int U = phase_units(G, op);
       const int K = gemv_K(G, op);
       const int nkb = (K + kBoxCols - 1) / kBoxCols;
       const int rpu = rows_per_unit(op);
-      // groups small enough that every SM gets work and no group needs more than kMaxPieces
-      const int max_u = std::max(1, std::min({max_units(op), P->max_blocks * 8 / rpu, (kMaxPieces - 1) * U / nsm}));
-      const int seg = op == OP_QKV ? G.hd / 16 : U;
-      std::vector<std::pair<int, int>> groups;  // (u0, n)
-      for (int x = 0; x < U;) {
-        const int y = std::min(U, (x / seg + 1) * seg);
-        const int len = y - x, ng = (len + max_u - 1) / max_u;
-        for (int k = 0, v = x; k < ng; ++k) {
-          const int nk = len / ng + (k < len % ng ? 1 : 0);
-          groups.push_back({v, nk});
-          v += nk;
-        }
-        x = y;
-      }
-      const long long W = (long long)U * nkb;
-      if ((long long)U * unit_weight_bytes(G, op) / nsm < kSplitMinBytes) {
-        // a small phase: whole units only (split pieces would add more fixed cost per task than
-        // they save), each SM a contiguous range of U / nsm or U / nsm + 1 units cut into
-        // tasks of <= max_units units inside head segments
-        const int mu = std::max(1, std::min(max_units(op), P->max_blocks * 8 / rpu));
-        // the extra units of the phase go to the SMs with the fewest bytes so far
-        std::vector<int> cnt(nsm, U / nsm), idx(nsm);
-        std::iota(idx.begin(), idx.end(), 0);
-        std::stable_sort(idx.begin(), idx.end(), [&](int a2, int b2) { return cum[a2] < cum[b2]; });
-        for (int k = 0; k < U % nsm; ++k) cnt[idx[k]]++;
-        for (int sm = 0, u = 0; sm < nsm; ++sm) {
-          const int n = cnt[sm];
-          for (int a = u, end = u + n; a < end;) {
-            const int b = std::min(end, (a / seg + 1) * seg);
-            const int len = b - a, ntask = (len + mu - 1) / mu;
-            for (int k = 0, v = a; k < ntask; ++k) {
-              const int nk = len / ntask + (k < len % ntask ? 1 : 0);
-              TaskDesc t{};
-              t.op = (uint8_t)op;
-              t.nunits = (uint8_t)nk;
-              t.layer = (uint16_t)l;
-              t.u0 = (uint32_t)v;
-              t.task_idx = (uint16_t)tidx++;
-              t.slot0 = t.task_idx;
-              t.k0 = 0;
-              t.k1 = (uint16_t)nkb;
-              t.split = kNoSplit;
-              t.kc = (uint16_t)stage_cols(nk * rpu / 8, K, c.max_batch);
-              t.wait_ctr = (uint16_t)wc;
-              t.wait_count = wcount;
-              t.sig_ctr = (uint16_t)sig;
-              P->streams[sm].push_back(t);
-              cum[sm] += (long long)nk * unit_weight_bytes(G, op);
-              v += nk;
-            }
-            a = b;
-          }
-          u += n;
-        }
-      } else {
-      const long long gmax = (long long)max_u * nkb;
-      // ranges long enough that no group falls into more than kMaxPieces of them
-      const int nuse = (int)std::max<long long>(1, std::min<long long>(nsm, W * (kMaxPieces - 1) / gmax));
-      std::vector<long long> cut(nuse + 1);
+      const int seg = op == OP_QKV ? G.hd / 16 : U;  // QKV tasks stay inside one head
+      const int mu = std::max(1, std::min(max_units(op), P->max_blocks * 8 / rpu));
+      auto make_task = [&](int u0, int n, int k0, int k1) {
+        TaskDesc t{};
+        t.op = (uint8_t)op;
+        t.nunits = (uint8_t)n;
+        t.layer = (uint16_t)l;
+        t.u0 = (uint32_t)u0;
+        t.k0 = (uint16_t)k0;
+        t.k1 = (uint16_t)k1;
+        t.split = kNoSplit;
+        const int cols = std::min(k1 * kBoxCols, K) - k0 * kBoxCols;
+        t.kc = (uint16_t)stage_cols(n * rpu / 8, cols, c.max_batch);
+        t.wait_ctr = (uint16_t)wc;
+        t.wait_count = wcount;
+        t.sig_ctr = (uint16_t)sig;
+        return t;
+      };
+      auto task_cost = [&](const TaskDesc& t) {
+        const long long cols = std::min((int)t.k1 * kBoxCols, K) - (long long)t.k0 * kBoxCols;
+        return (long long)t.nunits * rpu * cols * 2 + cols * operand_col_bytes(c.max_batch) + kTaskCostBytes +
+               (t.split != kNoSplit ? kPieceCostBytes : 0);
+      };
+      auto cand_cost = [&](const Cand& cd) {
+        std::vector<long long> per(nsm, 0);
+        for (const auto& st : cd.tasks) per[st.first] += task_cost(st.second);
+        return *std::max_element(per.begin(), per.end());
+      };
+      std::vector<Cand> cands;
+
+      // (1) Equal ranges.  Units are grouped into tasks of <= max_u units (QKV groups inside
+      // one head); the work is the line of (group, 64-column chunk) pairs weighted by the
+      // group's units, cut into equal ranges, one per SM.  A group that a cut falls into
+      // becomes K pieces (<= kMaxPieces), each with all of the group's rows; the last piece
+      // to finish adds the partial sums.
       {
-        // cuts at chunk boundaries of the group they fall into
-        long long pos = 0;
-        size_t gi = 0;
-        cut[0] = 0;
-        for (int s2 = 1; s2 < nuse; ++s2) {
-          const long long want = W * s2 / nuse;
-          while (gi < groups.size() && pos + (long long)groups[gi].second * nkb <= want) {
-            pos += (long long)groups[gi].second * nkb;
-            ++gi;
+        Cand cd;
+        // groups small enough that every SM gets work and no group needs more than kMaxPieces
+        const int max_u = std::max(1, std::min({max_units(op), P->max_blocks * 8 / rpu, (kMaxPieces - 1) * U / nsm}));
+        std::vector<std::pair<int, int>> groups;  // (u0, n)
+        for (int x = 0; x < U;) {
+          const int y = std::min(U, (x / seg + 1) * seg);
+          const int len = y - x, ng = (len + max_u - 1) / max_u;
+          for (int k = 0, v = x; k < ng; ++k) {
+            const int nk = len / ng + (k < len % ng ? 1 : 0);
+            groups.push_back({v, nk});
+            v += nk;
           }
-          const long long within = want - pos;  // inside group gi
-          const int n = gi < groups.size() ? groups[gi].second : 1;
-          cut[s2] = pos + (within / n) * n;
+          x = y;
         }
-        cut[nuse] = W;
-      }
-      // per group: its start on the line, and the ranges (pieces) it falls into
-      std::vector<long long> gstart(groups.size() + 1, 0);
-      for (size_t g = 0; g < groups.size(); ++g) gstart[g + 1] = gstart[g] + (long long)groups[g].second * nkb;
-      int next_id = 0;
-      std::vector<int> gid(groups.size(), -1), gpieces(groups.size(), 1), gslot0(groups.size(), 0);
-      for (size_t g = 0; g < groups.size(); ++g) {
-        int np = 0;
-        for (int s2 = 0; s2 < nuse; ++s2)
-          if (cut[s2] < gstart[g + 1] && cut[s2 + 1] > gstart[g]) ++np;
-        gpieces[g] = np;
-        if (np > 1) gid[g] = next_id++;
-      }
-      for (int s2 = 0; s2 < nuse; ++s2) {
-        const long long a = cut[s2], b = cut[s2 + 1];
-        if (a >= b) continue;
-        for (size_t g = 0; g < groups.size(); ++g) {
-          if (gstart[g + 1] <= a || gstart[g] >= b) continue;
-          const int n = groups[g].second;
-          const int k0 = (int)((std::max(a, gstart[g]) - gstart[g]) / n);
-          const int k1 = (int)((std::min(b, gstart[g + 1]) - gstart[g]) / n);
-          if (k0 >= k1) continue;
-          TaskDesc t{};
-          t.op = (uint8_t)op;
-          t.nunits = (uint8_t)n;
-          t.layer = (uint16_t)l;
-          t.u0 = (uint32_t)groups[g].first;
-          t.task_idx = (uint16_t)tidx++;
-          t.k0 = (uint16_t)k0;
-          t.k1 = (uint16_t)k1;
-          t.slot0 = t.task_idx;
-          if (gpieces[g] > 1) {
-            int piece = 0;
-            for (int s3 = 0; s3 < s2; ++s3)
-              if (cut[s3] < gstart[g + 1] && cut[s3 + 1] > gstart[g] && cut[s3] < cut[s3 + 1]) ++piece;
-            t.split = split_tag(gid[g], piece, gpieces[g]);
-            if (piece == 0) gslot0[g] = t.task_idx;  // pieces are made in K order: piece 0 first
-            t.slot0 = (uint16_t)gslot0[g];
-          } else {
-            t.split = kNoSplit;
+        const long long W = (long long)U * nkb;
+        if ((long long)U * unit_weight_bytes(G, op) / nsm < kSplitMinBytes) {
+          // a small phase: whole units only, each SM a contiguous range of U / nsm or
+          // U / nsm + 1 units cut into tasks of <= max_units units inside head segments; the
+          // extra units of the phase go to the SMs with the fewest bytes so far
+          std::vector<int> cnt(nsm, U / nsm), idx(nsm);
+          std::iota(idx.begin(), idx.end(), 0);
+          std::stable_sort(idx.begin(), idx.end(), [&](int a2, int b2) { return cum[a2] < cum[b2]; });
+          for (int k = 0; k < U % nsm; ++k) cnt[idx[k]]++;
+          for (int sm = 0, u = 0; sm < nsm; ++sm) {
+            const int n = cnt[sm];
+            for (int a2 = u, end = u + n; a2 < end;) {
+              const int b2 = std::min(end, (a2 / seg + 1) * seg);
+              const int len = b2 - a2, ntask = (len + mu - 1) / mu;
+              for (int k = 0, v = a2; k < ntask; ++k) {
+                const int nk = len / ntask + (k < len % ntask ? 1 : 0);
+                cd.tasks.push_back({sm, make_task(v, nk, 0, nkb)});
+                v += nk;
+              }
+              a2 = b2;
+            }
+            u += n;
           }
-          const int cols = std::min(k1 * kBoxCols, K) - k0 * kBoxCols;
-          t.kc = (uint16_t)stage_cols(n * rpu / 8, cols, c.max_batch);
-          t.wait_ctr = (uint16_t)wc;
-          t.wait_count = wcount;
-          t.sig_ctr = (uint16_t)sig;
-          P->streams[s2].push_back(t);
-          cum[s2] += (long long)n * rpu * cols * 2;
+        } else {
+          const long long gmax = (long long)max_u * nkb;
+          // ranges long enough that no group falls into more than kMaxPieces of them
+          const int nuse = (int)std::max<long long>(1, std::min<long long>(nsm, W * (kMaxPieces - 1) / gmax));
+          std::vector<long long> cut(nuse + 1);
+          {
+            // cuts at chunk boundaries of the group they fall into
+            long long pos = 0;
+            size_t gi = 0;
+            cut[0] = 0;
+            for (int s2 = 1; s2 < nuse; ++s2) {
+              const long long want = W * s2 / nuse;
+              while (gi < groups.size() && pos + (long long)groups[gi].second * nkb <= want) {
+                pos += (long long)groups[gi].second * nkb;
+                ++gi;
+              }
+              const long long within = want - pos;  // inside group gi
+              const int n = gi < groups.size() ? groups[gi].second : 1;
+              cut[s2] = pos + (within / n) * n;
+            }
+            cut[nuse] = W;
+          }
+          // per group: its start on the line, and the ranges (pieces) it falls into
+          std::vector<long long> gstart(groups.size() + 1, 0);
+          for (size_t g = 0; g < groups.size(); ++g) gstart[g + 1] = gstart[g] + (long long)groups[g].second * nkb;
+          std::vector<int> gid(groups.size(), -1), gpieces(groups.size(), 1);
+          for (size_t g = 0; g < groups.size(); ++g) {
+            int np = 0;
+            for (int s2 = 0; s2 < nuse; ++s2)
+              if (cut[s2] < gstart[g + 1] && cut[s2 + 1] > gstart[g]) ++np;
+            gpieces[g] = np;
+            if (np > 1) gid[g] = cd.nids++;
+          }
+          for (int s2 = 0; s2 < nuse; ++s2) {
+            const long long a2 = cut[s2], b2 = cut[s2 + 1];
+            if (a2 >= b2) continue;
+            for (size_t g = 0; g < groups.size(); ++g) {
+              if (gstart[g + 1] <= a2 || gstart[g] >= b2) continue;
+              const int n = groups[g].second;
+              const int k0 = (int)((std::max(a2, gstart[g]) - gstart[g]) / n);
+              const int k1 = (int)((std::min(b2, gstart[g + 1]) - gstart[g]) / n);
+              if (k0 >= k1) continue;
+              TaskDesc t = make_task(groups[g].first, n, k0, k1);
+              if (gpieces[g] > 1) {
+                int piece = 0;
+                for (int s3 = 0; s3 < s2; ++s3)
+                  if (cut[s3] < gstart[g + 1] && cut[s3 + 1] > gstart[g] && cut[s3] < cut[s3 + 1]) ++piece;
+                t.split = split_tag(gid[g], piece, gpieces[g]);
+              }
+              cd.tasks.push_back({s2, t});
+            }
+          }
         }
+        cands.push_back(std::move(cd));
       }
-      P->max_split_ids = std::max(P->max_split_ids, next_id);
+
+      // (2) One task per SM: n row groups whose sizes differ by at most one unit (QKV: a
+      // head's units split among its groups), each cut into m equal K pieces, n * m <= nsm.
+      // Slightly unequal bytes, but no SM pays for a second task.
+      for (int m = 1; m <= kMaxPieces && m <= nkb; ++m) {
+        const int n = nsm / m;
+        const int nseg = (U + seg - 1) / seg;
+        if (n < nseg) continue;
+        std::vector<std::pair<int, int>> groups;  // (u0, n)
+        bool ok = true;
+        for (int sg = 0; sg < nseg && ok; ++sg) {
+          const int x = sg * seg, len = std::min(U, x + seg) - x;
+          // this segment's share of the n groups, by its units
+          const int g_lo = (int)((long long)n * x / U), g_hi = (int)((long long)n * (x + len) / U);
+          const int ng = std::min(len, std::max(1, g_hi - g_lo));
+          if ((len + ng - 1) / ng > mu) { ok = false; break; }
+          for (int k = 0, v = x; k < ng; ++k) {
+            const int nk = len / ng + (k < len % ng ? 1 : 0);
+            groups.push_back({v, nk});
+            v += nk;
+          }
+        }
+        if (!ok || (int)groups.size() * m > nsm) continue;
+        Cand cd;
+        for (const auto& gr : groups) {
+          const int id = m > 1 ? cd.nids++ : -1;
+          for (int q = 0; q < m; ++q) {
+            const int k0 = nkb * q / m, k1 = nkb * (q + 1) / m;
+            TaskDesc t = make_task(gr.first, gr.second, k0, k1);
+            if (m > 1) t.split = split_tag(id, q, m);
+            cd.tasks.push_back({0, t});
+          }
+        }
+        // the largest tasks to the SMs with the fewest bytes so far, keeping the step's
+        // totals level (task order, and so piece order, is unchanged)
+        std::vector<int> ti(cd.tasks.size()), si(nsm);
+        std::iota(ti.begin(), ti.end(), 0);
+        std::iota(si.begin(), si.end(), 0);
+        std::stable_sort(ti.begin(), ti.end(), [&](int x, int y) {
+          return task_cost(cd.tasks[x].second) > task_cost(cd.tasks[y].second);
+        });
+        std::stable_sort(si.begin(), si.end(), [&](int x, int y) { return cum[x] < cum[y]; });
+        for (size_t k = 0; k < ti.size(); ++k) cd.tasks[ti[k]].first = si[k];
+        cands.push_back(std::move(cd));
       }
+
+      size_t best = 0;
+      for (size_t k = 1; k < cands.size(); ++k)
+        if (cand_cost(cands[k]) < cand_cost(cands[best])) best = k;
+      const Cand& cd = cands[best];
+      std::vector<int> slot0_of(cd.nids, -1);
+      for (const auto& st : cd.tasks) {
+        TaskDesc t = st.second;
+        t.task_idx = (uint16_t)tidx++;
+        t.slot0 = t.task_idx;
+        if (t.split != kNoSplit) {
+          const int id = split_id(t.split);
+          if (split_piece(t.split) == 0) slot0_of[id] = t.task_idx;  // piece 0 comes first
+          t.slot0 = (uint16_t)slot0_of[id];
+        }
+        P->streams[st.first].push_back(t);
+        const int cols = std::min((int)t.k1 * kBoxCols, K) - (int)t.k0 * kBoxCols;
+        cum[st.first] += (long long)t.nunits * rpu * cols * 2;
+      }
+      P->max_split_ids = std::max(P->max_split_ids, cd.nids);
     }
     phase_tasks[pi] = tidx;
     tasks_of_counter[sig] += tidx;

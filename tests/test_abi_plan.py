@@ -57,10 +57,10 @@ def test_default_plans_validate(lib, m, max_batch):
 def test_weight_bytes_balanced_across_sms(lib, m):
     st = mk.Plan(mk.model_cfg(m, 8, 4097)).stats()
     lo, hi = st["weight_bytes_min_sm"], st["weight_bytes_max_sm"]
-    # large GEMV phases are cut into equal ranges of (task group, 64-column chunk) work (SMs
-    # differ by at most one chunk of one group, <= 64 rows x 64 columns x 2 bytes, per phase);
-    # small phases into whole units, the extra unit going to the SMs with the fewest bytes so
-    # far: over the step the SMs stay within one unit plus one chunk per phase
+    # each GEMV phase takes the cheaper of equal ranges of (task group, 64-column chunk) work
+    # and one task per SM (row groups within one unit of each other, cut into equal K pieces);
+    # either way the larger shares go to the SMs with the fewest bytes so far, so over the
+    # step the SMs stay within one unit plus one chunk per phase
     chunk = 64 * 64 * 2
     unit = max(8 * m.ffn * 2, 16 * m.hidden * 2)
     assert hi - lo <= unit + chunk * (4 * m.n_layers + 1), (lo, hi)
