@@ -234,7 +234,7 @@ MK_API int mk_create_from_plan(mk_plan_t plan, const mk_weight_ptrs* w, int32_t 
   int regs = 0, lmem = 0, maxthr = 0;
   cudaError_t ce = mk::kernel_attributes(&regs, &lmem, &maxthr);
   if (ce != cudaSuccess) { release(h); return cuda_fail(nullptr, ce, "kernel attributes"); }
-  if (maxthr < mk::kThreads) { release(h); return fail(nullptr, MK_ERR_CUDA, "kernel cannot run its 320 threads"); }
+  if (maxthr < mk::kThreads) { release(h); return fail(nullptr, MK_ERR_CUDA, "kernel cannot run its " + std::to_string(mk::kThreads) + " threads"); }
 
   const mk::Geometry G = mk::geometry(c);
   const int S = plan->num_sms * plan->attn_slots_per_sm;
@@ -592,7 +592,7 @@ int static_setup(StaticState& s, const mk_model_cfg& c, const mk_weight_ptrs* w,
   int regs = 0, lmem = 0, maxthr = 0;
   cudaError_t ce = mk::kernel_attributes(&regs, &lmem, &maxthr);
   if (ce != cudaSuccess) return cuda_fail(nullptr, ce, "kernel attributes");
-  if (maxthr < mk::kThreads) return fail(nullptr, MK_ERR_CUDA, "kernel cannot run its 320 threads");
+  if (maxthr < mk::kThreads) return fail(nullptr, MK_ERR_CUDA, "kernel cannot run its " + std::to_string(mk::kThreads) + " threads");
 
   mk_plan_opts o{};
   o.num_sms = prop.multiProcessorCount;

@@ -22,7 +22,11 @@ namespace mk {
 
 // ---- launch geometry -------------------------------------------------------------------
 constexpr int kConsumerWarps = 8;                       // compute warps per CTA
-constexpr int kThreads = (kConsumerWarps + 2) * 32;     // + the weight/KV producer warp + the operand warp
+constexpr int kProducerWarp = kConsumerWarps;           // weight and KV copies
+constexpr int kOperandWarp = kConsumerWarps + 1;        // GEMV operand copies
+constexpr int kSignalWarp = kConsumerWarps + 2;         // releases finished tasks' counters
+constexpr int kThreads = (kConsumerWarps + 3) * 32;
+constexpr int kSigRing = 4;                             // finished tasks the consumers may run ahead of their release
 constexpr int kSlotBytes = 50 * 1024;                   // one pool stage: weights + their operands, or KV pages
 constexpr int kNumSlots = 4;                            // pool depth (200 KB; 4 x 50 KB measured fastest)
 constexpr int kMaxBatch = 16;

@@ -39,10 +39,13 @@ struct Smem {
   alignas(8) uint64_t wfull[kNumSlots];                  // weight/KV bytes of the stage landed
   alignas(8) uint64_t ofull[kNumSlots];                  // the stage's operand bytes landed (operand warp)
   alignas(8) uint64_t empty[kNumSlots];                  // all consumer warps done with the stage
+  alignas(8) uint64_t sigfull[kSigRing];                 // consumer warps: task done, its writes ordered before
+  alignas(8) uint64_t sigempty[kSigRing];                // signal warp: that task's counter released
+  int sigab[kSigRing];                                   // the consumers gave up on that task (no release)
+  int lm_last;                                           // this CTA released the step's last LM-head task
   int attn_R, bad, flag, flag2;  // attn_R: tokens per attention range (this step)
   unsigned long long wait_cyc;  // tracing: SM cycles warp 0 spent waiting for pool slots in the current task
   unsigned long long tm[3];     // tracing: compute, reduce, epilogue SM cycles of the current task (warp 0)
-  int inv_inst;                // ssq instance whose 1/rms sm.inv_rms holds (-1: none)
 };
 
 size_t kernel_smem_bytes() { return sizeof(Smem); }
@@ -731,17 +734,19 @@ __device__ __forceinline__ const bf16* next_gain(const KParams& p, int op, int l
 // ---------------------------------------------------------------------------------------
 // consumer task bodies
 
-__device__ void gemv_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_t& stage, bool& ab) {
+__device__ void gemv_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_t& stage, bool& ab, int& inv_inst) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool norm = t.op == OP_QKV || t.op == OP_GATEUP || t.op == OP_LMHEAD;
   const int inst = t.op == OP_GATEUP ? ssq_inst_oproj(t.layer)
                    : t.op == OP_QKV  ? (t.layer == 0 ? ssq_inst_embed() : ssq_inst_down(t.layer - 1))
                                      : ssq_inst_down(p.L - 1);
-  // tasks of one phase share the 1/rms of their input: compute it once per phase
-  const bool fresh = norm && !ab && sm.inv_inst != inst;
-  if (fresh) compute_inv_rms(p, sm, inst, (int)t.wait_count);
-  cbar();
-  if (fresh && threadIdx.x == 0) sm.inv_inst = inst;
+  // tasks of one phase share the 1/rms of their input: compute it once per phase (inv_inst is
+  // the same in every consumer thread, so the barrier is taken by all or none)
+  if (norm && inst != inv_inst) {
+    if (!ab) compute_inv_rms(p, sm, inst, (int)t.wait_count);
+    cbar();
+    inv_inst = inst;
+  }
   const int G = t.nunits * rows_per_unit(t.op) / 8;
   if (p.b == 1) gemv_dispatch<0>(p, sm, t, stage, ab, G);
   else if (p.b <= 8) gemv_dispatch<1>(p, sm, t, stage, ab, G);
@@ -1188,90 +1193,110 @@ __device__ __noinline__ void attn_task(const KParams& p, Smem& sm, const TaskDes
 __device__ void consumer(const KParams& p, Smem& sm, const TaskDesc* ts, int nt) {
   uint32_t stage = 0;
   bool ab = false;
-  int met_ctr = -1;          // thread 0: the last counter/target seen satisfied (counters only grow)
+  // the last counter/target seen satisfied (counters only grow) and the ssq instance whose
+  // 1/rms sm.inv_rms holds: the same in every consumer thread
+  int met_ctr = -1, inv_inst = -1;
   uint32_t met_target = 0;
   for (int ti = 0; ti < nt; ++ti) {
     const TaskDesc t = ts[ti];
-    // dependency wait: one thread polls, the others wait at the consumer barrier
+    // dependency wait, when the task's counter target is not met already: one thread polls,
+    // the others wait at the consumer barrier
     unsigned long long tr0 = 0, tr1 = 0;
-    if (threadIdx.x == 0) {
-      if (p.trace) { tr0 = gtimer(); sm.wait_cyc = 0; sm.tm[0] = sm.tm[1] = sm.tm[2] = 0; }
-      bool ok = !ab;
-      if (ok && t.wait_ctr != kNoCounter) {
-        const uint32_t target = t.wait_count * p.epoch;
-        if (t.wait_ctr != met_ctr || target != met_target) {
-          ok = wait_counter(p, t.wait_ctr, t.wait_count);
-          met_ctr = t.wait_ctr;
-          met_target = target;
-        }
-      }
-      sm.flag = ok ? 0 : 1;
-      if (p.trace) tr1 = gtimer();
+    if (threadIdx.x == 0 && p.trace) { tr0 = gtimer(); sm.wait_cyc = 0; sm.tm[0] = sm.tm[1] = sm.tm[2] = 0; }
+    const uint32_t target = t.wait_count * p.epoch;
+    if (t.wait_ctr != kNoCounter && (t.wait_ctr != met_ctr || target != met_target)) {
+      if (threadIdx.x == 0) sm.flag = (!ab && wait_counter(p, t.wait_ctr, t.wait_count)) ? 0 : 1;
+      cbar();
+      ab = ab || sm.flag;
+      met_ctr = t.wait_ctr;
+      met_target = target;
+      cbar();  // sm.flag is rewritten by the next poll
     }
-    cbar();
-    ab = ab || sm.flag;
+    if (threadIdx.x == 0 && p.trace) tr1 = gtimer();
     switch (t.op) {
       case OP_EMBED: embed_task(p, sm, t, ab); break;
       case OP_ATTN:
         if (p.hd == 64) attn_task<64>(p, sm, t, stage, ab);
         else attn_task<128>(p, sm, t, stage, ab);
         break;
-      default: gemv_task(p, sm, t, stage, ab); break;
+      default: gemv_task(p, sm, t, stage, ab, inv_inst); break;
     }
-    cbar();
+    cbar();  // every consumer write of the task is done
     if (threadIdx.x == 0) {
-      const long long ts0 = p.trace ? clock64() : 0ll;
-      if (!ab) {
-        // release: everything the consumer warps wrote before the barrier above is visible to
-        // whoever acquires the counter; bulk copies (async proxy) may read it next
-        asm volatile("fence.proxy.async.global;" ::: "memory");
-        if (t.op == OP_LMHEAD && p.argmax) {
-          const uint32_t old = atom_add_acqrel(p.ctr + t.sig_ctr, 1u);
-          sm.flag = old + 1u == (uint32_t)p.n_lm_tasks * p.epoch ? 1 : 0;
-        } else {
-          red_release_add(p.ctr + t.sig_ctr, 1u);  // nobody here needs the old value: no round trip
-          sm.flag = 0;
-        }
-      } else {
-        sm.flag = 0;
-      }
+      // hand the task to the signal warp, which releases its counter; the consumers go on
+      const int e = ti % kSigRing;
+      bool ok = !ab;
+      if (ti >= kSigRing) ok = mbar_wait(p, &sm.sigempty[e], ((ti / kSigRing) - 1) & 1) && ok;
+      sm.sigab[e] = ok ? 0 : 1;
+      mbar_arrive(&sm.sigfull[e]);
       if (p.trace) {
         unsigned long long* r = p.trace + 8ull * (p.task_off[blockIdx.x] + ti);
-        const long long ce = clock64();
-        const unsigned long long te = gtimer();
         r[0] = tr0;
         r[1] = tr1;
-        r[2] = te;
+        r[2] = gtimer();
         r[3] = (unsigned long long)t.op | ((unsigned long long)t.layer << 8) |
                ((unsigned long long)blockIdx.x << 24) | (min(sm.wait_cyc, 0xFFFFFFull) << 40);
         r[4] = sm.tm[0];
         r[5] = sm.tm[1];
         r[6] = sm.tm[2];
-        r[7] = (unsigned long long)(ce - ts0);
       }
     }
-    cbar();
-    if (sm.flag) {
-      // the last LM-head task of the step reduces the per-task argmax candidates
-      const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-      for (int bi = warp; bi < p.b; bi += kConsumerWarps) {
-        float best = -INFINITY;
-        int bidx = 0x7fffffff;
-        for (int k = lane; k < p.n_lm_tasks; k += 32) {
-          const float2 c = __ldcg(p.lmpart + (size_t)k * p.max_b + bi);
-          const int ci = __float_as_int(c.y);
-          if (c.x > best || (c.x == best && ci < bidx)) { best = c.x; bidx = ci; }
-        }
+  }
+  // once the signal warp has released every task: if this CTA's LM-head task was the step's
+  // last, reduce the per-task argmax candidates (one batch row per warp)
+  if (threadIdx.x == 0 && nt > 0 && p.argmax)
+    sm.flag = mbar_wait(p, &sm.sigempty[(nt - 1) % kSigRing], ((nt - 1) / kSigRing) & 1) ? sm.lm_last : 0;
+  cbar();
+  if (nt > 0 && p.argmax && sm.flag) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int bi = warp; bi < p.b; bi += kConsumerWarps) {
+      float best = -INFINITY;
+      int bidx = 0x7fffffff;
+      for (int k = lane; k < p.n_lm_tasks; k += 32) {
+        const float2 c = __ldcg(p.lmpart + (size_t)k * p.max_b + bi);
+        const int ci = __float_as_int(c.y);
+        if (c.x > best || (c.x == best && ci < bidx)) { best = c.x; bidx = ci; }
+      }
 #pragma unroll
-        for (int o = 16; o; o >>= 1) {
-          const float ov = __shfl_xor_sync(0xffffffffu, best, o);
-          const int oi = __shfl_xor_sync(0xffffffffu, bidx, o);
-          if (ov > best || (ov == best && oi < bidx)) { best = ov; bidx = oi; }
-        }
-        if (lane == 0) p.argmax[bi] = bidx;
+      for (int o = 16; o; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, best, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bidx, o);
+        if (ov > best || (ov == best && oi < bidx)) { best = ov; bidx = oi; }
       }
+      if (lane == 0) p.argmax[bi] = bidx;
     }
-    cbar();
+  }
+}
+
+// The signal warp: for each task of the CTA's stream, in order, once the consumer warps have
+// handed it over, make the task's writes visible and add one to its counter.  Generic-proxy
+// writes that other SMs' bulk copies (async proxy) read next need the proxy fence; the
+// release makes everything the consumers wrote before their barrier and hand-over visible to
+// whoever acquires the counter.  Whether the step's last LM-head task was released here is
+// left in sm.lm_last for the consumer warps.
+__device__ void signaler(const KParams& p, Smem& sm, const TaskDesc* ts, int nt) {
+  const int lane = threadIdx.x & 31;
+  for (int ti = 0; ti < nt; ++ti) {
+    const TaskDesc t = ts[ti];
+    const int e = ti % kSigRing;
+    if (!mbar_wait_warp(p, &sm.sigfull[e], (ti / kSigRing) & 1)) break;
+    int last = 0;
+    if (lane == 0) {
+      const long long ts0 = p.trace ? clock64() : 0ll;
+      if (!sm.sigab[e]) {
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        if (t.op == OP_LMHEAD && p.argmax) {
+          const uint32_t old = atom_add_acqrel(p.ctr + t.sig_ctr, 1u);
+          last = old + 1u == (uint32_t)p.n_lm_tasks * p.epoch ? 1 : 0;
+        } else {
+          red_release_add(p.ctr + t.sig_ctr, 1u);  // nobody here needs the old value: no round trip
+        }
+      }
+      if (p.trace) p.trace[8ull * (p.task_off[blockIdx.x] + ti) + 7] = (unsigned long long)(clock64() - ts0);
+      if (last) sm.lm_last = 1;
+      mbar_arrive(&sm.sigempty[e]);  // releases sm.lm_last to the consumers' wait
+    }
+    __syncwarp();
   }
 }
 
@@ -1287,6 +1312,11 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
       mbar_init(&sm.ofull[s], 1);
       mbar_init(&sm.empty[s], kConsumerWarps);
     }
+    for (int e = 0; e < kSigRing; ++e) {
+      mbar_init(&sm.sigfull[e], 1);
+      mbar_init(&sm.sigempty[e], 1);
+    }
+    sm.lm_last = 0;
     fence_mbar_init();
     // scalar input checks (page ids are checked where they are used)
     int bad = 0;
@@ -1300,15 +1330,15 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
     }
     if (bad) raise_error(p, -6 /* MK_ERR_BOUNDS */);
     sm.bad = bad;
-    sm.inv_inst = -1;
     if (!bad) sm.attn_R = attn_setup(p);
   }
   __syncthreads();
   if (sm.bad) return;
   const uint32_t o0 = p.task_off[blockIdx.x], o1 = p.task_off[blockIdx.x + 1];
   const int warp = threadIdx.x >> 5;
-  if (warp == kConsumerWarps) producer(p, sm, p.tasks + o0, (int)(o1 - o0));
-  else if (warp == kConsumerWarps + 1) operand_loader(p, sm, p.tasks + o0, (int)(o1 - o0));
+  if (warp == kProducerWarp) producer(p, sm, p.tasks + o0, (int)(o1 - o0));
+  else if (warp == kOperandWarp) operand_loader(p, sm, p.tasks + o0, (int)(o1 - o0));
+  else if (warp == kSignalWarp) signaler(p, sm, p.tasks + o0, (int)(o1 - o0));
   else consumer(p, sm, p.tasks + o0, (int)(o1 - o0));
 }
 
