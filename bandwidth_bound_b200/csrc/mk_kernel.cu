@@ -43,7 +43,10 @@ struct Smem {
   alignas(8) uint64_t sigempty[kSigRing];                // signal warp: that task's counter released
   int sigab[kSigRing];                                   // the consumers gave up on that task (no release)
   int lm_last;                                           // this CTA released the step's last LM-head task
-  int attn_R, bad, flag, flag2;  // attn_R: tokens per attention range (this step)
+  int attn_R, bad, flag, flag2;  // attn_R: tokens per attention range on the pair line (this step), 0: pair-aligned
+  int attn_n[kMaxBatch];         // pair-aligned: ranges per (sequence i, kv head) pair
+  int attn_Ri[kMaxBatch];        // pair-aligned: tokens per range of sequence i (a multiple of 16)
+  int attn_u0[kMaxBatch + 1];    // pair-aligned: first range of sequence i
   unsigned long long wait_cyc;  // tracing: SM cycles warp 0 spent waiting for pool slots in the current task
   unsigned long long tm[3];     // tracing: compute, reduce, epilogue SM cycles of the current task (warp 0)
 };
@@ -278,11 +281,17 @@ __device__ __forceinline__ void issue_gemv_chunk(const KParams& p, const TaskDes
   }
 }
 
-// Split-K attention work.  The (sequence i, kv head h) pairs are laid end to end, pair
-// (i, h) taking ceil16(len_i) token places; attention range u covers places [u R, u R + R)
-// of that line.  Its pieces are the parts of the pairs it overlaps, cut at 16-token
-// (page) boundaries, so every range holds the same number of KV bytes whatever the
-// lengths, and a piece is the unit of split-K state (one log-sum-exp partial).
+// Split-K attention work, partitioned at run time from this step's lengths in one of two ways.
+//  * Pair-aligned (whenever every (sequence i, kv head h) pair can have a range of its own):
+//    the pairs of sequence i get attn_n[i] ranges each, every range one piece of attn_Ri[i]
+//    tokens inside one pair.  attn_n is water-filled over the ranges: a round adds one range
+//    to every pair of the sequence whose ranges are longest.  No range pays for a second
+//    piece, and a pair's few pieces finish together.
+//  * Otherwise the pairs are laid end to end, pair (i, h) taking ceil16(len_i) token places;
+//    attention range u covers places [u R, u R + R) of that line, and its pieces are the
+//    parts of the pairs it overlaps, cut at 16-token (page) boundaries, so every range holds
+//    the same number of KV bytes whatever the lengths.
+// A piece is the unit of split-K state (one log-sum-exp partial).
 struct AttnPiece {
   int i, h;    // sequence, kv head
   int c, nc;   // piece index within the pair, pieces of the pair
@@ -291,7 +300,25 @@ struct AttnPiece {
 };
 
 // Piece j (in order) of range u, or false past the last one.
-__device__ bool attn_piece(const KParams& p, int R, int u, int j, AttnPiece& a) {
+__device__ bool attn_piece(const KParams& p, const Smem& sm, int u, int j, AttnPiece& a) {
+  const int R = sm.attn_R;
+  if (R == 0) {
+    if (j > 0 || u >= sm.attn_u0[p.b]) return false;
+    int i = 0;
+    while (u >= sm.attn_u0[i + 1]) ++i;
+    const int ni = sm.attn_n[i], Ri = sm.attn_Ri[i];
+    const int r = u - sm.attn_u0[i];
+    const int n = p.lens[i];
+    a.i = i;
+    a.h = r / ni;
+    a.c = r - a.h * ni;
+    a.n = n;
+    a.t0 = a.c * Ri;
+    if (a.t0 >= n) return false;
+    a.t1 = min(a.t0 + Ri, n);
+    a.nc = (n + Ri - 1) / Ri;
+    return true;
+  }
   const long long lo = (long long)u * R, hi = lo + R;
   long long off = 0;
   for (int i = 0; i < p.b; ++i) {
@@ -322,10 +349,34 @@ __device__ bool attn_piece(const KParams& p, int R, int u, int j, AttnPiece& a) 
   return false;
 }
 
-// Range length R (tokens, a multiple of 16): the padded pair lengths spread evenly over the
-// n_slots ranges, at least one full stage, and short enough that no pair is cut into more
-// than kMaxChunksPerSeq pieces.
-__device__ int attn_setup(const KParams& p) {
+// This step's attention partition into sm (thread 0, after the lengths were checked).  The
+// pair line's range length R is the padded pair lengths spread evenly over the n_slots
+// ranges, at least one full stage, and short enough that no pair is cut into more than
+// kMaxChunksPerSeq pieces.
+__device__ void attn_setup(const KParams& p, Smem& sm) {
+  const int T = attn_stage_tokens(p.hd);
+  if (p.b * p.nkv <= p.n_slots) {
+    int used = p.b * p.nkv;
+    for (int i = 0; i < p.b; ++i) sm.attn_n[i] = 1;
+    for (;;) {
+      int best = -1, bestlen = 0;
+      for (int i = 0; i < p.b; ++i) {
+        const int len = (p.lens[i] + sm.attn_n[i] - 1) / sm.attn_n[i];
+        if (sm.attn_n[i] < kMaxChunksPerSeq && len > bestlen && len > T) { best = i; bestlen = len; }
+      }
+      if (best < 0 || used + p.nkv > p.n_slots) break;
+      ++sm.attn_n[best];
+      used += p.nkv;
+    }
+    sm.attn_u0[0] = 0;
+    for (int i = 0; i < p.b; ++i) {
+      const int len = (p.lens[i] + sm.attn_n[i] - 1) / sm.attn_n[i];
+      sm.attn_Ri[i] = (len + kPage - 1) / kPage * kPage;
+      sm.attn_u0[i + 1] = sm.attn_u0[i] + p.nkv * sm.attn_n[i];
+    }
+    sm.attn_R = 0;
+    return;
+  }
   long long tot = 0;
   int mx = kPage;
   for (int i = 0; i < p.b; ++i) {
@@ -335,11 +386,11 @@ __device__ int attn_setup(const KParams& p) {
   }
   long long R = (tot + p.n_slots - 1) / p.n_slots;
   R = (R + kPage - 1) / kPage * kPage;
-  const long long rmin = attn_stage_tokens(p.hd);
+  const long long rmin = T;
   const long long rcap = ((mx + kMaxChunksPerSeq - 3) / (kMaxChunksPerSeq - 2) + kPage - 1) / kPage * kPage;
   if (R < rmin) R = rmin;
   if (R < rcap) R = rcap;
-  return (int)R;
+  sm.attn_R = (int)R;
 }
 
 // ---------------------------------------------------------------------------------------
@@ -420,7 +471,7 @@ __device__ void producer(const KParams& p, Smem& sm, const TaskDesc* ts, int nt)
     const TaskDesc t = ts[wt];
     if (t.op == OP_ATTN) {
       AttnPiece a;
-      for (int j = 0; !fail && attn_piece(p, sm.attn_R, (int)t.u0, j, a); ++j) {
+      for (int j = 0; !fail && attn_piece(p, sm, (int)t.u0, j, a); ++j) {
         const int ns = (a.t1 - a.t0 + T - 1) / T;
         for (int k = 0; k < ns; ++k, ++wk) {
           const int slot = wk % kNumSlots;
@@ -477,7 +528,7 @@ __device__ void operand_loader(const KParams& p, Smem& sm, const TaskDesc* ts, i
     if (t.op == OP_EMBED) continue;
     if (t.op == OP_ATTN) {
       AttnPiece a;
-      for (int j = 0; !fail && attn_piece(p, sm.attn_R, (int)t.u0, j, a); ++j) {
+      for (int j = 0; !fail && attn_piece(p, sm, (int)t.u0, j, a); ++j) {
         const int ns = (a.t1 - a.t0 + T - 1) / T;
         for (int k = 0; k < ns; ++k, ++wk) {
           const int slot = wk % kNumSlots;
@@ -986,7 +1037,7 @@ __device__ __noinline__ void attn_task(const KParams& p, Smem& sm, const TaskDes
   const bool tr = p.trace && threadIdx.x == 0;
   uint32_t ks = 0;  // stage count within the task: picks the warp group
   AttnPiece a;
-  for (int j = 0; attn_piece(p, sm.attn_R, (int)t.u0, j, a); ++j) {
+  for (int j = 0; attn_piece(p, sm, (int)t.u0, j, a); ++j) {
     const long long tc0 = tr ? clock64() : 0ll;
     const unsigned long long wait0 = tr ? sm.wait_cyc : 0ull;
     // Q fragments of head g_ of this kv group
@@ -1330,7 +1381,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
     }
     if (bad) raise_error(p, -6 /* MK_ERR_BOUNDS */);
     sm.bad = bad;
-    if (!bad) sm.attn_R = attn_setup(p);
+    if (!bad) attn_setup(p, sm);
   }
   __syncthreads();
   if (sm.bad) return;
