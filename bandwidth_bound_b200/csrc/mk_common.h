@@ -136,7 +136,8 @@ constexpr int kOpMapsPerKind = 2 * kMaxTiles + 1;
 MK_HD int opmap_index(int n_layers, int kind, int q) { return num_tmaps(n_layers) + kind * kOpMapsPerKind + q; }
 MK_HD int num_all_tmaps(int n_layers) { return num_tmaps(n_layers) + 3 * kOpMapsPerKind; }
 
-// Tokens per attention stage: K rows then V rows of the same tokens, 32 KB total.
-MK_HD int attn_stage_tokens(int head_dim) { return head_dim == 64 ? 128 : 64; }
+// Tokens per attention stage: K rows then V rows of the same tokens, 32 KB (head_dim 64) or
+// 48 KB (head_dim 128: six 16-token warp groups on one stage, most of a 50 KB slot).
+MK_HD int attn_stage_tokens(int head_dim) { return head_dim == 64 ? 128 : 96; }
 
 }  // namespace mk

@@ -1023,7 +1023,7 @@ __device__ __forceinline__ uint32_t split_pair(float x, float y, bool lo) {
 //     piece of (i, h) to finish combines all its pieces into the O-projection operand.
 template <int HD>
 __device__ __noinline__ void attn_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_t& stage, bool& ab) {
-  constexpr int T = HD == 64 ? 128 : 64;      // tokens per stage (K then V: 32 KB)
+  constexpr int T = HD == 64 ? 128 : 96;      // tokens per stage (K then V: 32 / 48 KB)
   constexpr int WPS = T / 16;                 // warps per stage, one 16-token group each
   constexpr int NG = kConsumerWarps / WPS;    // stages in flight across warp groups
   constexpr int NK = HD / 16;                 // k steps of Q K^T
