@@ -123,7 +123,8 @@ static std::string build_tensor_maps(const mk_model_cfg& c, const mk_weight_ptrs
 
 // Tensor maps of the GEMV operand buffers (appended after the weight maps): per operand kind,
 // bf16 tile parts q = 2 * mt + part as rows of 64 values (boxes of 8 rows = 64 columns of one
-// tile part), then the fp32 batch row 0 as rows of 32 values (boxes of 2 rows = 64 columns).
+// tile part), then the fp32 batch rows 0..kFmaRows-1 as lines of 32 values, ld / 32 lines per
+// batch row (boxes of 2 lines = 64 columns).
 static std::string encode_operand_maps(std::vector<CUtensorMap>& maps, int L, int ntiles,
                                        const __nv_bfloat16* const tiles[3], const float* const rows[3],
                                        const int lds[3]) {
@@ -143,7 +144,7 @@ static std::string encode_operand_maps(std::vector<CUtensorMap>& maps, int L, in
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
       if (r != CUDA_SUCCESS) return "cuTensorMapEncodeTiled failed for an operand buffer";
     }
-    cuuint64_t dims[2] = {32, (cuuint64_t)ld / 32};
+    cuuint64_t dims[2] = {32, (cuuint64_t)mk::kFmaRows * ld / 32};  // fp32 rows 0..kFmaRows-1, ld / 32 lines each
     cuuint64_t strides[1] = {128};
     cuuint32_t box[2] = {32, 2};
     CUresult r = encode(&maps[mk::opmap_index(L, kind, mk::kOpMapsPerKind - 1)], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
@@ -262,7 +263,7 @@ MK_API int mk_create_from_plan(mk_plan_t plan, const mk_weight_ptrs* w, int32_t 
   // operands: bf16 hi/lo tiles of 8 batch rows (operand_index layout) and the fp32 batch row 0,
   // zero padded to whole 64-column boxes
   const int ntiles = (mb + 7) / 8;
-  auto opbytes = [&](int ld) { return (size_t)ntiles * 2 * ld * 8 * 2 + (size_t)ld * 4; };
+  auto opbytes = [&](int ld) { return (size_t)ntiles * 2 * ld * 8 * 2 + (size_t)mk::kFmaRows * ld * 4; };
   const size_t o_ax = take(opbytes(ld_x)), o_aa = take(opbytes(ld_a)), o_ah = take(opbytes(ld_h));
   const int ssq_stride = plan->max_phase_tasks * mb;
   const size_t o_ssq = take(sizeof(float) * mk::num_ssq_inst(G.L) * ssq_stride);
@@ -623,7 +624,7 @@ int static_setup(StaticState& s, const mk_model_cfg& c, const mk_weight_ptrs* w,
   const int ld_x = mk::round_up(G.d, mk::kBoxCols), ld_a = mk::round_up(G.qdim, mk::kBoxCols),
             ld_h = mk::round_up(G.F, mk::kBoxCols);
   const int ntiles = (mb + 7) / 8;
-  auto opbytes = [&](int ld) { return (size_t)ntiles * 2 * ld * 8 * 2 + (size_t)ld * 4; };
+  auto opbytes = [&](int ld) { return (size_t)ntiles * 2 * ld * 8 * 2 + (size_t)mk::kFmaRows * ld * 4; };
   const size_t o_ax = take(opbytes(ld_x)), o_aa = take(opbytes(ld_a)), o_ah = take(opbytes(ld_h));
   const int ssq_stride = plan.max_phase_tasks * mb;
   const size_t o_ssq = take(sizeof(float) * mk::num_ssq_inst(G.L) * ssq_stride);

@@ -30,6 +30,7 @@ constexpr int kSigRing = 4;                             // finished tasks the co
 constexpr int kSlotBytes = 50 * 1024;                   // one pool stage: weights + their operands, or KV pages
 constexpr int kNumSlots = 4;                            // pool depth (200 KB; 4 x 50 KB measured fastest)
 constexpr int kMaxBatch = 16;
+constexpr int kFmaRows = 4;                             // batches up to this size run the GEMVs on fp32 FMA
 constexpr int kMaxBlocks = 8;                           // 8-row blocks per GEMV task (64 rows)
 constexpr int kPage = 16;                               // tokens per KV page
 constexpr int kMaxChunksPerSeq = 32;                    // split-K chunks per (sequence, kv head)
@@ -95,8 +96,8 @@ MK_HD uint32_t ceil_div(uint32_t a, uint32_t b) { return (a + b - 1) / b; }
 MK_HD int round_up(int a, int b) { return (a + b - 1) / b * b; }
 
 // Operand bytes per K column of one stage for a batch of up to max_batch rows: bf16 hi and
-// lo parts of every 8-row batch tile (16 bytes each per column).  The batch-1 path uses the
-// first 4 bytes (fp32) of the same room.
+// lo parts of every 8-row batch tile (16 bytes each per column).  The fp32 path (batch <=
+// kFmaRows) uses at most 16 bytes (4 rows x fp32) of the same room.
 MK_HD int operand_col_bytes(int max_batch) { return 32 * ((max_batch + 7) / 8); }
 
 // K columns per pool stage of a GEMV task with `blocks` 8-row blocks: the largest multiple of
@@ -116,7 +117,8 @@ MK_HD int stage_cols(int blocks, int K, int max_batch) {
 //   bf16 tiles: per batch tile mt (rows 8mt..8mt+7) and part (0 hi, 1 lo), block kb is 512
 //   contiguous bytes: 32 pieces of 16 bytes, piece 4 * row + tq = the 8 columns of group
 //   2tq + h of batch row `row` - lane (g, tq) reads piece `lane`;
-//   fp32 batch row 0: block kb is 128 bytes, piece tq = the 8 values of group 2tq + h.
+//   fp32 batch rows 0..kFmaRows-1, each ld values: block kb is 128 bytes, piece tq = the 8
+//   values of group 2tq + h.
 MK_HD int opnd_block(int k) { return ((k >> 6) << 1) | ((k >> 3) & 1); }
 MK_HD size_t opnd_tile_index(int mt, int part, int k, int row, int ld) {
   return ((((size_t)(mt * 2 + part) * (ld / 32) + opnd_block(k)) * 32 + row * 4 + ((k >> 4) & 3)) * 8 + (k & 7));
@@ -130,7 +132,7 @@ MK_HD int tmap_index(int layer, int mat, int n) { return (layer * kNumMats + mat
 MK_HD int num_tmaps(int n_layers) { return (n_layers + 1) * kNumMats * kMaxBlocks; }
 
 // Operand tensor maps, after the weight maps: per operand kind (0 normed x, 1 attention
-// output, 2 SwiGLU output), 2 * tiles bf16 maps (tile mt, part) then the fp32 row-0 map.
+// output, 2 SwiGLU output), 2 * tiles bf16 maps (tile mt, part) then the map of the fp32 rows.
 constexpr int kMaxTiles = (kMaxBatch + 7) / 8;
 constexpr int kOpMapsPerKind = 2 * kMaxTiles + 1;
 MK_HD int opmap_index(int n_layers, int kind, int q) { return num_tmaps(n_layers) + kind * kOpMapsPerKind + q; }

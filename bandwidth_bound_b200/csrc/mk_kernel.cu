@@ -563,12 +563,18 @@ __device__ void operand_loader(const KParams& p, Smem& sm, const TaskDesc* ts, i
       uint8_t* dst = sm.pool[slot] + (size_t)R * t.kc * 2;
       const int k0 = kbeg + ws * t.kc;
       const int nch = (min((int)t.kc, kend - k0) + kBoxCols - 1) / kBoxCols;
-      if (p.b == 1) {
-        if (lane == 0) mbar_expect_tx(&sm.ofull[slot], (uint32_t)nch * 256u);
+      if (p.b <= kFmaRows) {
+        // fp32 rows 0..NB-1: per chunk c, row r's 256 bytes at (c * NB + r) * 256
+        const int NB = p.b == 1 ? 1 : (p.b == 2 ? 2 : 4);
+        const int rows_per_row = (kind == 0 ? p.ld_x : (kind == 1 ? p.ld_a : p.ld_h)) / 32;
+        const int nbox = NB * nch;
+        if (lane == 0) mbar_expect_tx(&sm.ofull[slot], (uint32_t)nbox * 256u);
         __syncwarp();
-        for (int c = lane; c < nch; c += 32)
-          tma_2d(dst + (size_t)c * 256, maps + opmap_index(p.L, kind, kOpMapsPerKind - 1), 0, k0 / 32 + 2 * c,
-                 &sm.ofull[slot], pol);
+        for (int e = lane; e < nbox; e += 32) {
+          const int c = e / NB, r = e - c * NB;
+          tma_2d(dst + (size_t)e * 256, maps + opmap_index(p.L, kind, kOpMapsPerKind - 1), 0,
+                 r * rows_per_row + k0 / 32 + 2 * c, &sm.ofull[slot], pol);
+        }
       } else {
         const int nbox = 2 * ntile * nch;
         if (lane == 0) mbar_expect_tx(&sm.ofull[slot], (uint32_t)nbox * 1024u);
@@ -626,14 +632,18 @@ __device__ void compute_inv_rms(const KParams& p, Smem& sm, int inst, int nparts
   }
 }
 
-// Store one GEMV operand value (batch row bi, column k): bf16 hi part and bf16 lo part
-// (the remainder) into the tile layout, and fp32 for batch row 0.
-__device__ __forceinline__ void put_operand(bf16* tiles, float* f, int ld, int bi, int k, float v) {
+// Store one GEMV operand value (batch row bi, column k) in the layout this step's GEMVs read:
+// fp32 rows for batches up to kFmaRows (the FMA path), else its bf16 hi part and the bf16 lo
+// part of the remainder in the tile layout.
+__device__ __forceinline__ void put_operand(const KParams& p, bf16* tiles, float* f, int ld, int bi, int k, float v) {
+  if (p.b <= kFmaRows) {
+    f[(size_t)bi * ld + opnd_row0_index(k)] = v;
+    return;
+  }
   const bf16 h = __float2bfloat16_rn(v);
   const int mt = bi >> 3, row = bi & 7;
   tiles[opnd_tile_index(mt, 0, k, row, ld)] = h;
   tiles[opnd_tile_index(mt, 1, k, row, ld)] = __float2bfloat16_rn(v - __bfloat162float(h));
-  if (bi == 0) f[opnd_row0_index(k)] = v;
 }
 
 // Stream the task's stages through the eight warps and reduce into sm.ep[row][batch].
@@ -644,9 +654,10 @@ __device__ __forceinline__ void put_operand(bf16* tiles, float* f, int ld, int b
 // 16-byte pieces of chunk kb / 2, so lane (g, tq) reads piece 2*tq + h of row 8j + g -
 // conflict-free - which holds columns 16*tq + 8*h .. +7, and the operand piece of the same
 // columns at `lane` (bf16) or `tq` (fp32, shared by the 8 lanes of one tq).
-// MT = 0: CUDA-core FMA (batch 1); MT = 1, 2: mma.sync with MT tiles of 8 batch rows, rows
-// 0-7 of the M = 16 tile the bf16 hi parts, rows 8-15 the lo parts.
-template <int MT, int G>
+// MT = 0: CUDA-core FMA on fp32 activations for NB (1, 2 or 4 >= batch) rows, the operands of
+// chunk c row r at (c * NB + r) * 256 bytes; MT = 1, 2: mma.sync with MT tiles of 8 batch
+// rows, rows 0-7 of the M = 16 tile the bf16 hi parts, rows 8-15 the lo parts.
+template <int MT, int G, int NB = 1>
 __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDesc t, uint32_t& stage, bool& ab) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, tq = lane & 3;
@@ -688,11 +699,14 @@ __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDes
     for (int kb = (warp + kConsumerWarps - (s * nbs) % kConsumerWarps) % kConsumerWarps; kb < nb;
          kb += kConsumerWarps) {
       const uint8_t* chunk = tile + (size_t)(kb >> 1) * (R * 128) + ((((2 * tq + (kb & 1)) ^ g)) << 4);
-      uint4 A[2 * NMT];
+      uint4 A[MT == 0 ? 2 * NB : 2 * NMT];
       if constexpr (MT == 0) {
-        const uint8_t* ap = opnd + (size_t)kb * 128 + tq * 32;
-        A[0] = *reinterpret_cast<const uint4*>(ap);
-        A[1] = *reinterpret_cast<const uint4*>(ap + 16);
+#pragma unroll
+        for (int r = 0; r < NB; ++r) {
+          const uint8_t* ap = opnd + ((size_t)(kb >> 1) * NB + r) * 256 + (kb & 1) * 128 + tq * 32;
+          A[2 * r] = *reinterpret_cast<const uint4*>(ap);
+          A[2 * r + 1] = *reinterpret_cast<const uint4*>(ap + 16);
+        }
       } else {
 #pragma unroll
         for (int q = 0; q < 2 * MT; ++q)
@@ -702,18 +716,27 @@ __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDes
       for (int j = 0; j < G; ++j) {
         const uint4 w = *reinterpret_cast<const uint4*>(chunk + (8 * j + g) * 128);
         if constexpr (MT == 0) {
-          float s0 = acc[j][0][0];
-          s0 = fmaf(bf_lo(w.x), __uint_as_float(A[0].x), s0); s0 = fmaf(bf_hi(w.x), __uint_as_float(A[0].y), s0);
-          s0 = fmaf(bf_lo(w.y), __uint_as_float(A[0].z), s0); s0 = fmaf(bf_hi(w.y), __uint_as_float(A[0].w), s0);
-          s0 = fmaf(bf_lo(w.z), __uint_as_float(A[1].x), s0); s0 = fmaf(bf_hi(w.z), __uint_as_float(A[1].y), s0);
-          s0 = fmaf(bf_lo(w.w), __uint_as_float(A[1].z), s0); s0 = fmaf(bf_hi(w.w), __uint_as_float(A[1].w), s0);
-          acc[j][0][0] = s0;
+#pragma unroll
+          for (int r = 0; r < NB; ++r) {
+            const uint4 a0 = A[2 * r], a1 = A[2 * r + 1];
+            float s0 = acc[j][0][r];
+            s0 = fmaf(bf_lo(w.x), __uint_as_float(a0.x), s0); s0 = fmaf(bf_hi(w.x), __uint_as_float(a0.y), s0);
+            s0 = fmaf(bf_lo(w.y), __uint_as_float(a0.z), s0); s0 = fmaf(bf_hi(w.y), __uint_as_float(a0.w), s0);
+            s0 = fmaf(bf_lo(w.z), __uint_as_float(a1.x), s0); s0 = fmaf(bf_hi(w.z), __uint_as_float(a1.y), s0);
+            s0 = fmaf(bf_lo(w.w), __uint_as_float(a1.z), s0); s0 = fmaf(bf_hi(w.w), __uint_as_float(a1.w), s0);
+            acc[j][0][r] = s0;
+          }
         } else {
 #pragma unroll
           for (int mt = 0; mt < MT; ++mt) {
             const uint4 H = A[2 * mt], L = A[2 * mt + 1];
-            mma_bf16(acc[j][mt], H.x, L.x, H.y, L.y, w.x, w.y);
-            mma_bf16(acc[j][mt], H.z, L.z, H.w, L.w, w.z, w.w);
+            // the block's two MMAs into a fresh accumulator, added to the total in fp32
+            // (round to nearest): tensor-core accumulation truncates, so no long chains
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            mma_bf16(d, H.x, L.x, H.y, L.y, w.x, w.y);
+            mma_bf16(d, H.z, L.z, H.w, L.w, w.z, w.w);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[j][mt][e] += d[e];
           }
         }
       }
@@ -732,10 +755,13 @@ __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDes
 #pragma unroll
       for (int j = 0; j < G; ++j) {
         if constexpr (MT == 0) {
-          float v = acc[j][0][0];
-          v += __shfl_xor_sync(0xffffffffu, v, 1);
-          v += __shfl_xor_sync(0xffffffffu, v, 2);
-          if (tq == 0) red[((warp * kMaxBlocks + j) * 8 + 0) * 8 + g] = v;
+#pragma unroll
+          for (int r = 0; r < NB; ++r) {
+            float v = acc[j][0][r];
+            v += __shfl_xor_sync(0xffffffffu, v, 1);
+            v += __shfl_xor_sync(0xffffffffu, v, 2);
+            if (tq == 0) red[((warp * kMaxBlocks + j) * 8 + r) * 8 + g] = v;
+          }
         } else {
           const float2 y = make_float2(acc[j][mt][0] + acc[j][mt][2], acc[j][mt][1] + acc[j][mt][3]);
           *reinterpret_cast<float2*>(&red[((warp * kMaxBlocks + j) * 8 + g) * 8 + 2 * tq]) = y;
@@ -759,17 +785,17 @@ __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDes
   if (p.trace && threadIdx.x == 0) sm.tm[1] += (unsigned long long)(clock64() - tr0);
 }
 
-template <int MT>
+template <int MT, int NB = 1>
 __device__ void gemv_dispatch(const KParams& p, Smem& sm, const TaskDesc& t, uint32_t& stage, bool& ab, int G) {
   switch (G) {
-    case 1: gemv_body<MT, 1>(p, sm, t, stage, ab); break;
-    case 2: gemv_body<MT, 2>(p, sm, t, stage, ab); break;
-    case 3: gemv_body<MT, 3>(p, sm, t, stage, ab); break;
-    case 4: gemv_body<MT, 4>(p, sm, t, stage, ab); break;
-    case 5: gemv_body<MT, 5>(p, sm, t, stage, ab); break;
-    case 6: gemv_body<MT, 6>(p, sm, t, stage, ab); break;
-    case 7: gemv_body<MT, 7>(p, sm, t, stage, ab); break;
-    default: gemv_body<MT, 8>(p, sm, t, stage, ab); break;
+    case 1: gemv_body<MT, 1, NB>(p, sm, t, stage, ab); break;
+    case 2: gemv_body<MT, 2, NB>(p, sm, t, stage, ab); break;
+    case 3: gemv_body<MT, 3, NB>(p, sm, t, stage, ab); break;
+    case 4: gemv_body<MT, 4, NB>(p, sm, t, stage, ab); break;
+    case 5: gemv_body<MT, 5, NB>(p, sm, t, stage, ab); break;
+    case 6: gemv_body<MT, 6, NB>(p, sm, t, stage, ab); break;
+    case 7: gemv_body<MT, 7, NB>(p, sm, t, stage, ab); break;
+    default: gemv_body<MT, 8, NB>(p, sm, t, stage, ab); break;
   }
 }
 
@@ -799,7 +825,9 @@ __device__ void gemv_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_
     inv_inst = inst;
   }
   const int G = t.nunits * rows_per_unit(t.op) / 8;
-  if (p.b == 1) gemv_dispatch<0>(p, sm, t, stage, ab, G);
+  if (p.b == 1) gemv_dispatch<0, 1>(p, sm, t, stage, ab, G);
+  else if (p.b == 2) gemv_dispatch<0, 2>(p, sm, t, stage, ab, G);
+  else if (p.b <= kFmaRows) gemv_dispatch<0, 4>(p, sm, t, stage, ab, G);
   else if (p.b <= 8) gemv_dispatch<1>(p, sm, t, stage, ab, G);
   else gemv_dispatch<2>(p, sm, t, stage, ab, G);
   const long long te0 = (p.trace && threadIdx.x == 0) ? clock64() : 0ll;
@@ -899,7 +927,7 @@ __device__ void gemv_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_
         const float r = sm.inv_rms[bi];
         const float gv = sm.ep[row][bi] * r;
         const float uv = sm.ep[8 * n + row][bi] * r;
-        put_operand(p.ah_t, p.ah_f, p.ld_h, bi, 8 * t.u0 + row, silu_f(gv) * uv);
+        put_operand(p, p.ah_t, p.ah_f, p.ld_h, bi, 8 * t.u0 + row, silu_f(gv) * uv);
       }
     }
   } else if (t.op == OP_OPROJ || t.op == OP_DOWN) {
@@ -917,7 +945,7 @@ __device__ void gemv_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_
         const float xn = __ldcg(xp) + sm.ep[row][bi];
         *xp = xn;
         sm.ep[row][bi] = xn;
-        put_operand(p.ax_t, p.ax_f, p.ld_x, bi, grow, xn * __bfloat162float(gain[grow]));
+        put_operand(p, p.ax_t, p.ax_f, p.ld_x, bi, grow, xn * __bfloat162float(gain[grow]));
         if (dbg) dbg[(size_t)bi * p.d + grow] = xn;
       }
     }
@@ -978,7 +1006,7 @@ __device__ void embed_task(const KParams& p, Smem& sm, const TaskDesc& t, bool a
     for (int c = lane; c < nc; c += 32) {
       const float v = __bfloat162float(e[c0 + c]);
       p.x[(size_t)bi * p.d + c0 + c] = v;
-      put_operand(p.ax_t, p.ax_f, p.ld_x, bi, c0 + c, v * __bfloat162float(gain[c0 + c]));
+      put_operand(p, p.ax_t, p.ax_f, p.ld_x, bi, c0 + c, v * __bfloat162float(gain[c0 + c]));
       if (p.dbg) p.dbg[(size_t)bi * p.d + c0 + c] = v;
       s += v * v;
     }
@@ -1137,8 +1165,16 @@ __device__ __noinline__ void attn_task(const KParams& p, Smem& sm, const TaskDes
         for (int nn = 0; nn < NN / 2; ++nn) {
           uint32_t b0, b1, b2, b3;
           ldsm_x4_t(vb + kv_off(((mi & 1) << 3) + rr, 2 * nn + (mi >> 1)), b0, b1, b2, b3);
-          mma_bf16(o[2 * nn], pa0, pa1, pa2, pa3, b0, b1);
-          mma_bf16(o[2 * nn + 1], pa0, pa1, pa2, pa3, b2, b3);
+          // this stage's P V into fresh accumulators, added to O in fp32 (round to nearest):
+          // tensor-core accumulation truncates, and O lives across all the piece's stages
+          float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+          mma_bf16(d0, pa0, pa1, pa2, pa3, b0, b1);
+          mma_bf16(d1, pa0, pa1, pa2, pa3, b2, b3);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            o[2 * nn][e] += d0[e];
+            o[2 * nn + 1][e] += d1[e];
+          }
         }
       }
       __syncwarp();
@@ -1230,7 +1266,7 @@ __device__ __noinline__ void attn_task(const KParams& p, Smem& sm, const TaskDes
           acc1 = fmaf(wts[h * 32 + c + 1], __ldcg(pc + (c + 1) * pst), acc1);
         }
         if (c < a.nc) acc0 = fmaf(wts[h * 32 + c], __ldcg(pc + c * pst), acc0);
-        put_operand(p.aa_t, p.aa_f, p.ld_a, a.i, (a.h * G + h) * HD + dd, acc0 + acc1);
+        put_operand(p, p.aa_t, p.aa_f, p.ld_a, a.i, (a.h * G + h) * HD + dd, acc0 + acc1);
       }
     }
     cbar();  // sm.red is reused by the next piece

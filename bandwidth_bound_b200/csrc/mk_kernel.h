@@ -34,7 +34,7 @@ struct KParams {
   float *x, *q, *ssq;
   float* part;               // split-K partials [max_b * nkv][kMaxChunksPerSeq][g][hd + 2]
   // GEMV operands, written once by the producing phase: bf16 hi/lo tiles in the layout of
-  // operand_index (all batch rows) and fp32 (batch row 0, for the batch-1 path).
+  // operand_index (all batch rows) and fp32 (batch rows below kFmaRows, for the FMA path).
   // ax: x * gain of the next RMSNorm (input of qkv / gate-up / lm head), aa: attention output,
   // ah: SwiGLU output; ld = K rounded up to 64, padding zero
   __nv_bfloat16 *ax_t, *aa_t, *ah_t;
