@@ -1339,10 +1339,20 @@ __device__ void consumer(const KParams& p, Smem& sm, const TaskDesc* ts, int nt)
     for (int bi = warp; bi < p.b; bi += kConsumerWarps) {
       float best = -INFINITY;
       int bidx = 0x7fffffff;
-      for (int k = lane; k < p.n_lm_tasks; k += 32) {
-        const float2 c = __ldcg(p.lmpart + (size_t)k * p.max_b + bi);
-        const int ci = __float_as_int(c.y);
-        if (c.x > best || (c.x == best && ci < bidx)) { best = c.x; bidx = ci; }
+      // eight candidates' loads in flight per lane; the comparison keeps the lowest index on ties,
+      // so the order of visits does not matter
+      for (int k0 = lane; k0 < p.n_lm_tasks; k0 += 256) {
+        float2 c[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int k = k0 + 32 * u;
+          c[u] = k < p.n_lm_tasks ? __ldcg(p.lmpart + (size_t)k * p.max_b + bi) : make_float2(-INFINITY, __int_as_float(0x7fffffff));
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int ci = __float_as_int(c[u].y);
+          if (c[u].x > best || (c[u].x == best && ci < bidx)) { best = c[u].x; bidx = ci; }
+        }
       }
 #pragma unroll
       for (int o = 16; o; o >>= 1) {
