@@ -16,7 +16,7 @@ Auto-Regressive Model Decode Megakernels" (paperlayer.ai digest of arXiv
   * §3.2 "Unverifiable correctness of kernel fusing": each sequence of a ragged
     batch decodes at its own position.
 
-Readings where the pages are silent (each one is listed in the design doc):
+Readings where the pages are silent:
   * Llama conventions: RMSNorm with eps inside the square root and the gain
     applied afterwards; RoPE in the Hugging Face rotate-half pairing (j, j+hd/2)
     with inv_freq_j = theta^(-2j/hd) and no frequency scaling; keys are cached
