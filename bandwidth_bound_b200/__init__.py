@@ -119,6 +119,22 @@ def model_cfg(m, max_batch: int, max_ctx: int) -> ModelCfg:
                     float(m.rope_theta), float(m.rms_eps), int(max_batch), int(max_ctx), int(m.page_size))
 
 
+def step_bytes(m, ctx_lens: Sequence[int]) -> int:
+    """Bytes one decode step must read from HBM, the numerator of model bandwidth
+    utilisation ("Inside the megakernel serving engine", the MBU definition): every
+    layer's projection weights and its two norm gains, the final norm gain, the whole
+    LM-head matrix (counted even when tied to the embedding), the gathered embedding
+    row of each sequence and the prior K and V entries of every layer, all bf16.
+    Writes and the new token's own K/V, produced on chip, are not counted."""
+    d, L = m.hidden, m.n_layers
+    q_out = m.n_heads * m.head_dim
+    kv_out = m.n_kv_heads * m.head_dim
+    per_layer = d * q_out + 2 * d * kv_out + q_out * d + 3 * d * m.ffn + 2 * d
+    elements = L * per_layer + d + m.vocab * d + len(ctx_lens) * d
+    elements += 2 * L * kv_out * sum(int(s) for s in ctx_lens)
+    return 2 * elements
+
+
 def _check(rc: int, handle=None, what: str = ""):
     if rc != MK_OK:
         lib = load_library()

@@ -95,10 +95,16 @@ MK_HD int max_units(int op) { return (op == OP_QKV || op == OP_GATEUP) ? kMaxBlo
 MK_HD uint32_t ceil_div(uint32_t a, uint32_t b) { return (a + b - 1) / b; }
 MK_HD int round_up(int a, int b) { return (a + b - 1) / b * b; }
 
+// fp32 operand rows a stage carries for a batch of b <= kFmaRows rows (1, 2 or 4).
+MK_HD int fma_rows(int b) { return b == 1 ? 1 : (b == 2 ? 2 : kFmaRows); }
+
 // Operand bytes per K column of one stage for a batch of up to max_batch rows: bf16 hi and
-// lo parts of every 8-row batch tile (16 bytes each per column).  The fp32 path (batch <=
-// kFmaRows) uses at most 16 bytes (4 rows x fp32) of the same room.
-MK_HD int operand_col_bytes(int max_batch) { return 32 * ((max_batch + 7) / 8); }
+// lo parts of every 8-row batch tile (16 bytes each per column), or, when every batch the
+// handle takes runs on the fp32 path (max_batch <= kFmaRows), 4 bytes per fp32 row.  A
+// batch-1 handle thus streams 384 weight columns of a 64-row task per 50 KB stage, not 320.
+MK_HD int operand_col_bytes(int max_batch) {
+  return max_batch <= kFmaRows ? 4 * fma_rows(max_batch) : 32 * ((max_batch + 7) / 8);
+}
 
 // K columns per pool stage of a GEMV task with `blocks` 8-row blocks: the largest multiple of
 // 64 whose weights (blocks * 8 rows) and operands fit one slot, at most K rounded up to 64.

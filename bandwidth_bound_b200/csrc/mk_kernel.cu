@@ -565,7 +565,7 @@ __device__ void operand_loader(const KParams& p, Smem& sm, const TaskDesc* ts, i
       const int nch = (min((int)t.kc, kend - k0) + kBoxCols - 1) / kBoxCols;
       if (p.b <= kFmaRows) {
         // fp32 rows 0..NB-1: per chunk c, row r's 256 bytes at (c * NB + r) * 256
-        const int NB = p.b == 1 ? 1 : (p.b == 2 ? 2 : 4);
+        const int NB = fma_rows(p.b);
         const int rows_per_row = (kind == 0 ? p.ld_x : (kind == 1 ? p.ld_a : p.ld_h)) / 32;
         const int nbox = NB * nch;
         if (lane == 0) mbar_expect_tx(&sm.ofull[slot], (uint32_t)nbox * 256u);

@@ -290,7 +290,6 @@ def _time_steps(fn, steps, stream, flush, per):
 
 def run_mk(args, world, rank, local):
     import bandwidth_bound_b200 as mk
-    import oracle
 
     w = synth.WORKLOADS[args.workload]
     if args.layers:
@@ -314,7 +313,7 @@ def run_mk(args, world, rank, local):
     len_d = pos_d + 1
     logits = torch.empty((b, m.vocab), dtype=torch.float32, device="cuda")
     am = torch.empty((b,), dtype=torch.int32, device="cuda")
-    B = oracle.model_bytes(m, lens)
+    B = mk.step_bytes(m, lens)
     l2 = torch.cuda.get_device_properties(local).L2_cache_size
     flush = None
     l2_note = f"inputs larger than L2 ({B / 1e9:.2f} GB read per step vs {l2 / 1e6:.0f} MB L2)"
@@ -402,16 +401,20 @@ def run_mk(args, world, rank, local):
         "gpu_launches": args.steps * h.launches_per_step(),
     }
     if not args.no_secondary and b > 1:
-        # batch 1 of the same model and context on the same handle (first sequence)
-        b1 = lambda: h.step(tok_d[:1], pos_d[:1], len_d[:1], kv, logits[:1], am[:1], stream=stream,  # noqa: E731
-                            check=False)
+        # batch 1 of the same model, weights and KV cache (first sequence) on a handle built for
+        # batch 1, as a batch-1 server would create it: its stages carry one fp32 operand row,
+        # so each 50 KB stage holds 384 weight columns of a 64-row task instead of 320
+        h1 = mk.Megakernel(m, wts, 1, max_ctx)
+        b1 = lambda: h1.step(tok_d[:1], pos_d[:1], len_d[:1], kv, logits[:1], am[:1], stream=stream,  # noqa: E731
+                             check=False)
         for _ in range(args.warmup):
             b1()
         barrier(world)
         t1, _ = time_steps(b1, min(args.steps, 200), stream, flush)
         ms1 = max_over_ranks(world, t1) / min(args.steps, 200)
-        B1 = oracle.model_bytes(m, lens[:1])
-        line["secondary"] = {"workload": f"{m.name}-b1 (same handle, context {lens[0]})", "ms_per_step": ms1,
+        B1 = mk.step_bytes(m, lens[:1])
+        h1.close()
+        line["secondary"] = {"workload": f"{m.name}-b1 (batch-1 handle, context {lens[0]})", "ms_per_step": ms1,
                              "tokens_per_s": world / (ms1 / 1e3), "mbu": B1 / (ms1 / 1e3) / (NOMINAL_HBM_GBS * 1e9),
                              "achieved_gbs": B1 / (ms1 / 1e3) / 1e9}
     if rank == 0 and not args.no_cpu_baseline:
