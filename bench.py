@@ -304,9 +304,9 @@ def run_mk(args, world, rank, local):
     toks = synth.token_ids(m, b, tag=w.name)
     plan = None
     if args.max_blocks or args.attn_slots:
-        plan = mk.Plan(mk.model_cfg(m, max(b, 8), max_ctx), num_sms=torch.cuda.get_device_properties(local).multi_processor_count,
+        plan = mk.Plan(mk.model_cfg(m, b, max_ctx), num_sms=torch.cuda.get_device_properties(local).multi_processor_count,
                        attn_slots_per_sm=args.attn_slots, max_blocks=args.max_blocks)
-    h = mk.Megakernel(m, wts, max(b, 8), max_ctx, plan=plan)
+    h = mk.Megakernel(m, wts, b, max_ctx, plan=plan)
     stream = torch.cuda.current_stream()
     tok_d = torch.tensor(toks, dtype=torch.int32, device="cuda")
     pos_d = torch.tensor(lens, dtype=torch.int32, device="cuda")
@@ -344,10 +344,14 @@ def run_mk(args, world, rank, local):
 
         np.save(os.path.splitext(args.trace)[0] + ".npy", raw)
         if not args.no_secondary and b > 1:
-            h.set_trace(rec)
-            h.step(tok_d[:1], pos_d[:1], len_d[:1], kv, logits[:1], am[:1], stream=stream, check=False)
+            h1t = mk.Megakernel(m, wts, 1, max_ctx)  # the batch-1 handle of the secondary line
+            rec1 = torch.zeros((h1t.num_tasks(), 8), dtype=torch.int64, device="cuda")
+            h1t.set_trace(rec1)
+            h1t.step(tok_d[:1], pos_d[:1], len_d[:1], kv, logits[:1], am[:1], stream=stream, check=False)
             torch.cuda.synchronize()
-            h.set_trace(None)
+            h1t.set_trace(None)
+            h1t.close()
+            rec = rec1
             with open(args.trace, "a") as f:
                 f.write("--- batch 1 ---\n" + mktrace.summarize(rec.cpu().numpy().view("uint64"), m.n_layers) + "\n")
     clocks = ClockSampler(local)
