@@ -18,6 +18,9 @@ from .decode import (  # noqa: F401
     combine_partials,
     silu,
     decode_step,
+    decode_layer,
+    layer_weights_f64,
+    lm_head,
     model_bytes,
     argmax_lowest,
 )

@@ -138,6 +138,73 @@ def _gather_prior(pool_l: torch.Tensor, table_row, n_prior: int, page: int) -> t
     return to_f64(blk[:, :n_prior, :])
 
 
+def layer_weights_f64(weights: dict, layer: int) -> dict:
+    """The bf16 weights of one layer as float64 CPU tensors (exact)."""
+    return {k: to_f64(t) for k, t in weights["layers"][layer].items()}
+
+
+def decode_layer(cfg, lw: dict, x: torch.Tensor, k_pool_l: torch.Tensor, v_pool_l: torch.Tensor,
+                 page_table, positions, *, round_new_kv: bool = True) -> dict:
+    """One transformer layer of the decode step (§2.1) for a ragged batch.
+
+    lw: float64 weights of the layer (``layer_weights_f64``); x: float64 [b][d] residual
+    stream entering the layer; k_pool_l/v_pool_l: that layer's pools [P][n_kv][page][hd]
+    holding the prior entries; positions[i] = prior entries of sequence i = its new
+    token's position.  Per sequence: RMSNorm, the three projections, RoPE at the
+    sequence's position, the new K/V rounded to bf16 as stored, attention of every
+    query head over the prior keys plus the new one, the O projection and residual,
+    RMSNorm, the SwiGLU MLP and residual.
+
+    Returns {"x": [b][d] after the layer, "k_new"/"v_new" [b][n_kv][hd] (bf16-rounded),
+    "k_new_exact"/"v_new_exact" (before rounding)}.
+    """
+    b = x.shape[0]
+    nq, nkv, hd = cfg.n_heads, cfg.n_kv_heads, cfg.head_dim
+    P = cfg.page_size
+    xn = rmsnorm(x, lw["attn_norm"], cfg.rms_eps)
+    q = (xn @ lw["wq"].T).view(b, nq, hd)
+    k = (xn @ lw["wk"].T).view(b, nkv, hd)
+    v = (xn @ lw["wv"].T).view(b, nkv, hd)
+    attn = torch.zeros((b, nq, hd), dtype=F64)
+    k_new = torch.zeros((b, nkv, hd), dtype=F64)
+    v_new = torch.zeros_like(k_new)
+    k_exact = torch.zeros_like(k_new)
+    v_exact = torch.zeros_like(k_new)
+    for i in range(b):
+        p = int(positions[i])
+        qi = rope(q[i], p, cfg.rope_theta)
+        ki = rope(k[i], p, cfg.rope_theta)
+        vi = v[i]
+        k_exact[i], v_exact[i] = ki, vi
+        kr, vr = bf16_rne(ki), bf16_rne(vi)
+        k_new[i], v_new[i] = kr, vr
+        kin, vin = (kr, vr) if round_new_kv else (ki, vi)
+        Kp = _gather_prior(k_pool_l, page_table[i], p, P)        # [nkv][p][hd]
+        Vp = _gather_prior(v_pool_l, page_table[i], p, P)
+        for h in range(nq):
+            kvh = kv_head_of(h, nq, nkv)
+            Kh = torch.cat([Kp[kvh], kin[kvh][None, :]], dim=0)
+            Vh = torch.cat([Vp[kvh], vin[kvh][None, :]], dim=0)
+            attn[i, h] = attention(qi[h][None, :], Kh, Vh)[0]
+    x = x + attn.reshape(b, nq * hd) @ lw["wo"].T
+    xn = rmsnorm(x, lw["mlp_norm"], cfg.rms_eps)
+    hmid = silu(xn @ lw["w_gate"].T) * (xn @ lw["w_up"].T)
+    x = x + hmid @ lw["w_down"].T
+    return {"x": x, "k_new": k_new, "v_new": v_new, "k_new_exact": k_exact, "v_new_exact": v_exact}
+
+
+def lm_head(cfg, weights: dict, x: torch.Tensor) -> torch.Tensor:
+    """logits = W_lm (rmsnorm(x) * g_final) for x float64 [b][d] -> float64 [b][V]."""
+    xf = rmsnorm(x, to_f64(weights["final_norm"]), cfg.rms_eps)
+    head = weights["lm_head"]
+    V = head.shape[0]
+    logits = torch.empty((x.shape[0], V), dtype=F64)
+    step = 16384
+    for r0 in range(0, V, step):
+        logits[:, r0:r0 + step] = xf @ to_f64(head[r0:r0 + step]).T
+    return logits
+
+
 def decode_step(cfg, weights: dict, k_pool: torch.Tensor, v_pool: torch.Tensor,
                 page_table, token_ids, positions, *, round_new_kv: bool = True,
                 layers: Optional[int] = None, want_logits: bool = True) -> dict:
@@ -159,8 +226,7 @@ def decode_step(cfg, weights: dict, k_pool: torch.Tensor, v_pool: torch.Tensor,
     """
     L = cfg.n_layers if layers is None else layers
     b = len(token_ids)
-    d, nq, nkv, hd = cfg.hidden, cfg.n_heads, cfg.n_kv_heads, cfg.head_dim
-    g = nq // nkv
+    d, nkv, hd = cfg.hidden, cfg.n_kv_heads, cfg.head_dim
     P = cfg.page_size
     kp = k_pool.detach().to("cpu")
     vp = v_pool.detach().to("cpu")
@@ -179,45 +245,18 @@ def decode_step(cfg, weights: dict, k_pool: torch.Tensor, v_pool: torch.Tensor,
         slots.append((int(table[i][p // P]), p % P))
 
     for li in range(L):
-        lw = {k: to_f64(t) for k, t in weights["layers"][li].items()}
-        xn = rmsnorm(x, lw["attn_norm"], cfg.rms_eps)
-        q = (xn @ lw["wq"].T).view(b, nq, hd)
-        k = (xn @ lw["wk"].T).view(b, nkv, hd)
-        v = (xn @ lw["wv"].T).view(b, nkv, hd)
-        attn = torch.zeros((b, nq, hd), dtype=F64)
-        for i in range(b):
-            p = int(positions[i])
-            qi = rope(q[i], p, cfg.rope_theta)
-            ki = rope(k[i], p, cfg.rope_theta)
-            vi = v[i]
-            k_exact[li, i], v_exact[li, i] = ki, vi
-            kr, vr = bf16_rne(ki), bf16_rne(vi)
-            k_new[li, i], v_new[li, i] = kr, vr
-            kin, vin = (kr, vr) if round_new_kv else (ki, vi)
-            Kp = _gather_prior(kp[li], table[i], p, P)              # [nkv][p][hd]
-            Vp = _gather_prior(vp[li], table[i], p, P)
-            for h in range(nq):
-                kvh = kv_head_of(h, nq, nkv)
-                Kh = torch.cat([Kp[kvh], kin[kvh][None, :]], dim=0)
-                Vh = torch.cat([Vp[kvh], vin[kvh][None, :]], dim=0)
-                attn[i, h] = attention(qi[h][None, :], Kh, Vh)[0]
-        x = x + attn.reshape(b, nq * hd) @ lw["wo"].T
-        xn = rmsnorm(x, lw["mlp_norm"], cfg.rms_eps)
-        hmid = silu(xn @ lw["w_gate"].T) * (xn @ lw["w_up"].T)
-        x = x + hmid @ lw["w_down"].T
+        lw = layer_weights_f64(weights, li)
+        r = decode_layer(cfg, lw, x, kp[li], vp[li], table, positions, round_new_kv=round_new_kv)
+        x = r["x"]
+        k_new[li], v_new[li] = r["k_new"], r["v_new"]
+        k_exact[li], v_exact[li] = r["k_new_exact"], r["v_new_exact"]
         hidden.append(x.clone())
         del lw
 
     out = {"hidden": torch.stack(hidden), "k_new": k_new, "v_new": v_new,
            "k_new_exact": k_exact, "v_new_exact": v_exact, "slots": slots}
     if L == cfg.n_layers and want_logits:
-        xf = rmsnorm(x, to_f64(weights["final_norm"]), cfg.rms_eps)
-        head = weights["lm_head"]
-        V = head.shape[0]
-        logits = torch.empty((b, V), dtype=F64)
-        step = 16384
-        for r0 in range(0, V, step):
-            logits[:, r0:r0 + step] = xf @ to_f64(head[r0:r0 + step]).T
+        logits = lm_head(cfg, weights, x)
         out["logits"] = logits
         out["argmax"] = [argmax_lowest(logits[i]) for i in range(b)]
     return out

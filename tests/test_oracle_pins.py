@@ -434,3 +434,20 @@ def test_other_shapes_match_huggingface_llama_float64(shape):
     ref = _hf_reference(m, wts, kv, toks, lens)
     out = oracle.decode_step(m, wts, kv.k_pool, kv.v_pool, kv.page_table, toks, lens, round_new_kv=False)
     assert _compare_to_hf(out, ref) < 1e-10
+
+
+def test_layer_by_layer_run_from_its_own_states_reproduces_the_step():
+    """The re-anchored comparison of the GPU parity tests runs each oracle layer from a given
+    residual stream.  Fed the oracle's own states it must reproduce the whole step exactly."""
+    from parity import Case, run_oracle
+
+    m, wts, kv, toks, lens = _tiny_inputs()
+    c = Case(m, list(lens), toks, 0.1, len(lens), max(lens) + 1, wts, kv)
+    whole = oracle.decode_step(m, wts, kv.k_pool, kv.v_pool, kv.page_table, toks, lens)
+    out = run_oracle(c, kv.k_pool, kv.v_pool, anchor=whole["hidden"])
+    for key in ("k_new", "v_new", "k_new_exact", "v_new_exact"):
+        assert torch.equal(out[key], whole[key])
+        assert torch.equal(out["anchored"][key], whole[key])
+    assert torch.equal(out["hidden"], whole["hidden"])
+    assert torch.equal(out["logits"], whole["logits"])
+    assert out["argmax"] == whole["argmax"] and out["slots"] == whole["slots"]

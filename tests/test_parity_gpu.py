@@ -31,10 +31,42 @@ def _cuda():
 def _run(c, batch=None, handle=None, **kw):
     kb, vb = c.kv.k_pool.cpu(), c.kv.v_pool.cpu()
     out, h = gpu_step(c, handle=handle, batch=batch)
-    ref = run_oracle(c, kb, vb, batch=batch)
+    ref = run_oracle(c, kb, vb, batch=batch, anchor=out["hidden"])
     errs = check_step(c, out, ref, kb, vb, batch=batch, **kw)
     print(c.m.name, len(c.lens) if batch is None else batch, errs)
     return out, ref, h, errs
+
+
+def _new_entries(c, b):
+    """The K and V entries the step appended (bit patterns), [L][b][n_kv][hd] each."""
+    P = c.m.page_size
+    pages = [int(c.kv.page_table[i, c.lens[i] // P]) for i in range(b)]
+    slots = [c.lens[i] % P for i in range(b)]
+    k = torch.stack([c.kv.k_pool[:, pages[i], :, slots[i], :] for i in range(b)], 1)
+    v = torch.stack([c.kv.v_pool[:, pages[i], :, slots[i], :] for i in range(b)], 1)
+    return k.view(torch.int16).cpu(), v.view(torch.int16).cpu()
+
+
+def _run_capture_off_then_on(c):
+    """The step as bench.py times it (no mid-state capture) against the oracle, then the same
+    step with capture on: logits, argmax and the appended K/V must be bit-identical, and the
+    captured run adds the per-layer hidden and re-anchored K/V checks."""
+    b = len(c.lens)
+    kb, vb = c.kv.k_pool.cpu(), c.kv.v_pool.cpu()
+    off, h = gpu_step(c, debug=False)
+    assert off["hidden"] is None
+    k_off, v_off = _new_entries(c, b)
+    on, _ = gpu_step(c, handle=h, debug=True)
+    k_on, v_on = _new_entries(c, b)
+    assert torch.equal(off["logits"], on["logits"])
+    assert torch.equal(off["argmax"], on["argmax"])
+    assert torch.equal(k_off, k_on) and torch.equal(v_off, v_on)
+    ref = run_oracle(c, kb, vb, anchor=on["hidden"])
+    errs_off = check_step(c, off, ref, kb, vb, check_pool=False)
+    errs_on = check_step(c, on, ref, kb, vb, check_pool=False)
+    print(c.m.name, b, "capture off:", errs_off)
+    print(c.m.name, b, "capture on:", errs_on)
+    h.close()
 
 
 def test_tiny_config_b1_position_64():
@@ -113,27 +145,28 @@ def test_llama32_1b_late_arrival_same_handle():
     c = make_case(w.model, w.context_lengths(), max_batch=9, max_ctx=4097, tag=w.name)
     kb, vb = c.kv.k_pool.cpu(), c.kv.v_pool.cpu()
     out8, h = gpu_step(c, batch=8)
-    ref8 = run_oracle(c, kb, vb, batch=8)
+    ref8 = run_oracle(c, kb, vb, batch=8, anchor=out8["hidden"])
     print("b8", check_step(c, out8, ref8, kb, vb, batch=8))
     kb2, vb2 = c.kv.k_pool.cpu(), c.kv.v_pool.cpu()
     out9, _ = gpu_step(c, handle=h, batch=9)
-    ref9 = run_oracle(c, kb2, vb2, batch=9)
+    ref9 = run_oracle(c, kb2, vb2, batch=9, anchor=out9["hidden"])
     print("b9", check_step(c, out9, ref9, kb2, vb2, batch=9))
 
 
 @pytest.mark.slow
 @pytest.mark.parametrize("b", [1, 8])
 def test_llama3_8b_ctx2048(b):
+    """Full size, in the handle configuration bench.py times (max_batch = b, capture off)."""
     w = synth.WORKLOADS[f"llama3-8b-b{b}"]
-    c = make_case(w.model, w.context_lengths(), max_ctx=4096, tag=w.name)
-    _run(c, check_pool=False)
+    c = make_case(w.model, w.context_lengths(), max_ctx=max(w.context_lengths()) + 2, tag=w.name)
+    _run_capture_off_then_on(c)
 
 
 @pytest.mark.slow
 def test_llama2_13b_ragged_b4():
     w = synth.WORKLOADS["llama2-13b-b4"]
-    c = make_case(w.model, w.context_lengths(), max_ctx=4097, tag=w.name)
-    _run(c, check_pool=False)
+    c = make_case(w.model, w.context_lengths(), max_ctx=max(w.context_lengths()) + 2, tag=w.name)
+    _run_capture_off_then_on(c)
 
 
 # --- errors -----------------------------------------------------------------------------
