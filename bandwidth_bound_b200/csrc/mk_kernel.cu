@@ -95,14 +95,6 @@ __device__ __forceinline__ bool mbar_test(uint64_t* b, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
-                                         uint64_t pol) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
-      : "memory");
-}
 // Tiled TMA loads of a box of a weight matrix (128-byte swizzle), completion on an mbarrier.
 __device__ __forceinline__ void tma_2d(void* dst, const void* map, int c0, int c1, uint64_t* bar, uint64_t pol) {
   asm volatile(

@@ -241,7 +241,10 @@ def run_reference(args, world, rank):
     t = statistics.median(per)
     value = w.batch / t
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+            "ms_per_step_kind": "projected: median over samples of (one layer x layers + an LM-head slice scaled "
+                                "to the vocabulary), not a timed full step",
+            "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_desc(w, lens),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cb["cores"], "kind": "oracle",

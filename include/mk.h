@@ -83,7 +83,13 @@ typedef struct mk_weight_ptrs {
  * [n_layers][num_pages][n_kv_heads][page_size][head_dim]; entry t of sequence i
  * lives in physical page page_table[i*max_pages_per_seq + t/page_size], slot
  * t % page_size.  Keys are stored after RoPE.  page_table is device int32
- * [>= batch][max_pages_per_seq]. */
+ * [>= batch][max_pages_per_seq].
+ * Layout choice: inside a page the kv head is the outer index (head-major), not the
+ * token.  One head's 16 tokens x head_dim values are then contiguous, and the kernel
+ * moves one page of one head as a single tiled TMA box with 128-byte swizzle; a
+ * token-major page ([page_size][n_kv_heads][head_dim]) would put that head's rows
+ * n_kv_heads*head_dim*2 bytes apart and take a strided box per page and head.  Callers
+ * holding token-major pages must transpose them once when filling the cache. */
 typedef struct mk_kv_cache {
   void *k_pool, *v_pool;
   const int32_t *page_table;
@@ -126,6 +132,9 @@ MK_API int mk_create_from_plan(mk_plan_t plan, const mk_weight_ptrs *weights, in
                                mk_handle_t *out);
 
 /* One decode step, stream-ordered and asynchronous (one kernel launch).
+ * Besides the logits it returns the greedy next token (argmax_out), reduced inside the
+ * same launch from per-task candidates of the LM head, so a greedy caller needs no
+ * second kernel and no read of the [batch][vocab] logits.
  *   token_ids  device int32 [batch]: the new token of each sequence
  *   positions  device int32 [batch]: p_i = prior entries of sequence i = the new
  *              token's position; sequences may all differ (ragged batch)
@@ -187,7 +196,9 @@ MK_API int mk_get_status(mk_handle_t h);
  * device error starts from a clean state).  Host-synchronous. */
 MK_API int mk_reset(mk_handle_t h);
 
-/* Mid-state capture for checking: when layer_hidden is a device fp32 buffer of
+/* Mid-state capture for checking (the per-task timeline is the separate call
+ * mk_set_trace: the two are set and cleared independently, and a checking run need not
+ * pay for the trace's stores): when layer_hidden is a device fp32 buffer of
  * [n_layers+1][max_batch][hidden], each later step writes the residual stream
  * after the embedding gather (index 0) and after each layer (index l+1) for its
  * batch rows.  NULL turns capture off. */
