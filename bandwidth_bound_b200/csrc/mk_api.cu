@@ -189,6 +189,199 @@ static std::string encode_kv_maps(const mk_model_cfg& c, const mk_kv_cache* kv, 
   return "";
 }
 
+// ---------------------------------------------------------------------------------------
+// Set-up shared by the handle (one cudaMalloc arena) and the allocation-free entry point (one
+// __device__ array): weight checks, device checks, the scratch layout, the uploads and the
+// kernel parameters.  Both paths lay the same pieces out in the same order.
+
+// Check the weight pointers; collect the per-layer device pointers.  "" or an error message.
+static std::string collect_layers(const mk_model_cfg& c, const mk_weight_ptrs* w, std::vector<LayerW>& lw) {
+  if (!w->embed || !w->final_norm || !w->lm_head || !w->attn_norm || !w->wq || !w->wk || !w->wv || !w->wo ||
+      !w->mlp_norm || !w->w_gate || !w->w_up || !w->w_down)
+    return "null weight pointer";
+  const void* all[3] = {w->embed, w->final_norm, w->lm_head};
+  for (const void* p : all)
+    if (!aligned16(p)) return "weights must be 16-byte aligned";
+  lw.assign(c.n_layers > 0 ? c.n_layers : 0, LayerW{});
+  for (int l = 0; l < c.n_layers; ++l) {
+    const void* ps[9] = {w->attn_norm[l], w->wq[l], w->wk[l], w->wv[l], w->wo[l],
+                         w->mlp_norm[l], w->w_gate[l], w->w_up[l], w->w_down[l]};
+    for (const void* p : ps)
+      if (!p || !aligned16(p)) return "layer weight null or not 16-byte aligned";
+    lw[l] = LayerW{(const __nv_bfloat16*)ps[0], (const __nv_bfloat16*)ps[1], (const __nv_bfloat16*)ps[2],
+                   (const __nv_bfloat16*)ps[3], (const __nv_bfloat16*)ps[4], (const __nv_bfloat16*)ps[5],
+                   (const __nv_bfloat16*)ps[6], (const __nv_bfloat16*)ps[7], (const __nv_bfloat16*)ps[8]};
+  }
+  return "";
+}
+
+// The device runs the kernel: sm_100, cooperative launch, enough threads.  MK_OK or a code
+// with g_err set.
+static int check_device(int dev, const char* who) {
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return fail(nullptr, MK_ERR_NO_DEVICE, "no CUDA device");
+  if (prop.major != 10) return fail(nullptr, MK_ERR_NO_DEVICE, "the kernel is built for sm_100a (B200)");
+  if (!prop.cooperativeLaunch) return fail(nullptr, MK_ERR_NO_DEVICE, "device lacks cooperative launch");
+  int regs = 0, lmem = 0, maxthr = 0;
+  cudaError_t ce = mk::kernel_attributes(&regs, &lmem, &maxthr);
+  if (ce != cudaSuccess) return cuda_fail(nullptr, ce, "kernel attributes");
+  if (maxthr < mk::kThreads)
+    return fail(nullptr, MK_ERR_CUDA, std::string(who) + ": kernel cannot run its " + std::to_string(mk::kThreads) +
+                                          " threads");
+  return MK_OK;
+}
+
+// Byte offsets of the scratch pieces (256-byte aligned).  The last three serve only the
+// handle's host-buffer entry point.
+struct Layout {
+  size_t layers, tasks, offs, maps, x, q, ax, aa, ah, ssq, part, lmpart, spart, scnt, ctr, cmb, ctl, status, rope;
+  size_t stage, logits, argmax;
+  size_t total;
+  int ld_x, ld_a, ld_h, ntiles, ssq_stride, nsplit;
+  std::vector<mk::TaskDesc> flat;   // the per-SM streams, concatenated
+  std::vector<uint32_t> offs_host;  // per-SM offsets into flat
+};
+
+static Layout layout_scratch(const mk_plan_s& plan, bool host_step) {
+  const mk_model_cfg& c = plan.cfg;
+  const mk::Geometry G = mk::geometry(c);
+  const int mb = c.max_batch;
+  Layout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off += (bytes + 255) & ~size_t(255); return o; };
+  L.offs_host.assign(plan.num_sms + 1, 0);
+  for (int s = 0; s < plan.num_sms; ++s) {
+    L.flat.insert(L.flat.end(), plan.streams[s].begin(), plan.streams[s].end());
+    L.offs_host[s + 1] = (uint32_t)L.flat.size();
+  }
+  L.layers = take(sizeof(LayerW) * c.n_layers);
+  L.tasks = take(sizeof(mk::TaskDesc) * L.flat.size());
+  L.offs = take(sizeof(uint32_t) * L.offs_host.size());
+  L.maps = take(sizeof(CUtensorMap) * (size_t)mk::num_all_tmaps(G.L));
+  L.x = take(sizeof(float) * mb * G.d);
+  L.q = take(sizeof(float) * mb * G.qdim);
+  L.ld_x = mk::round_up(G.d, mk::kBoxCols);
+  L.ld_a = mk::round_up(G.qdim, mk::kBoxCols);
+  L.ld_h = mk::round_up(G.F, mk::kBoxCols);
+  // operands: bf16 hi/lo tiles of 8 batch rows (opnd_tile_index layout) and fp32 batch rows
+  // 0..kFmaRows-1, zero padded to whole 64-column boxes
+  L.ntiles = (mb + 7) / 8;
+  auto opbytes = [&](int ld) { return (size_t)L.ntiles * 2 * ld * 8 * 2 + (size_t)mk::kFmaRows * ld * 4; };
+  L.ax = take(opbytes(L.ld_x));
+  L.aa = take(opbytes(L.ld_a));
+  L.ah = take(opbytes(L.ld_h));
+  L.ssq_stride = plan.max_phase_tasks * mb;  // per instance: [task of the phase][max_b]
+  L.ssq = take(sizeof(float) * (size_t)mk::num_ssq_inst(G.L) * L.ssq_stride);
+  L.part = take(sizeof(float) * (size_t)mb * G.nkv * mk::kMaxChunksPerSeq * G.g * (G.hd + 2));
+  L.lmpart = take(sizeof(float2) * (size_t)plan.n_lm_tasks * mb);
+  L.nsplit = plan.max_split_ids > 0 ? plan.max_split_ids : 1;
+  L.spart = take(sizeof(float) * (size_t)L.nsplit * mk::kMaxPieces * mk::kMaxBlocks * 8 * mb);
+  L.scnt = take(sizeof(uint32_t) * (size_t)L.nsplit);
+  L.ctr = take(sizeof(uint32_t) * mk::num_counters(G.L));
+  L.cmb = take(sizeof(uint32_t) * (size_t)G.L * mb * G.nkv);
+  L.ctl = take(sizeof(uint32_t) * 2);
+  L.status = take(sizeof(int));
+  L.rope = take(sizeof(float2) * (size_t)c.max_ctx * (G.hd / 2));
+  L.stage = L.logits = L.argmax = 0;
+  if (host_step) {
+    L.stage = take(sizeof(int32_t) * 3 * mb);
+    L.logits = take(sizeof(float) * (size_t)mb * G.V);
+    L.argmax = take(sizeof(int32_t) * mb);
+  }
+  L.total = off;
+  return L;
+}
+
+// Encode the tensor maps of (plan, weights) for scratch at `A`, clear the scratch, upload the
+// tables and compute the RoPE table, in order on `stream`, then synchronise it.
+static int upload_tables(const mk_plan_s& plan, const mk_weight_ptrs* w, const std::vector<LayerW>& lw,
+                         const Layout& L, unsigned char* A, cudaStream_t stream, const char* who) {
+  const mk_model_cfg& c = plan.cfg;
+  const mk::Geometry G = mk::geometry(c);
+  std::vector<CUtensorMap> maps;
+  std::string merr = build_tensor_maps(c, w, maps);
+  if (merr.empty()) {
+    auto tl = [&](size_t o) { return (const __nv_bfloat16*)(A + o); };
+    auto rw = [&](size_t o, int ld) { return (const float*)(A + o + (size_t)L.ntiles * 2 * ld * 8 * 2); };
+    const __nv_bfloat16* tiles[3] = {tl(L.ax), tl(L.aa), tl(L.ah)};
+    const float* rows[3] = {rw(L.ax, L.ld_x), rw(L.aa, L.ld_a), rw(L.ah, L.ld_h)};
+    const int lds[3] = {L.ld_x, L.ld_a, L.ld_h};
+    merr = encode_operand_maps(maps, G.L, L.ntiles, tiles, rows, lds);
+  }
+  if (!merr.empty()) return fail(nullptr, MK_ERR_CUDA, std::string(who) + ": " + merr);
+  cudaError_t ce = cudaMemsetAsync(A, 0, L.total, stream);
+  if (ce == cudaSuccess)
+    ce = cudaMemcpyAsync(A + L.layers, lw.data(), sizeof(LayerW) * c.n_layers, cudaMemcpyHostToDevice, stream);
+  if (ce == cudaSuccess)
+    ce = cudaMemcpyAsync(A + L.tasks, L.flat.data(), sizeof(mk::TaskDesc) * L.flat.size(), cudaMemcpyHostToDevice,
+                         stream);
+  if (ce == cudaSuccess)
+    ce = cudaMemcpyAsync(A + L.offs, L.offs_host.data(), sizeof(uint32_t) * L.offs_host.size(),
+                         cudaMemcpyHostToDevice, stream);
+  if (ce == cudaSuccess)
+    ce = cudaMemcpyAsync(A + L.maps, maps.data(), sizeof(CUtensorMap) * maps.size(), cudaMemcpyHostToDevice, stream);
+  if (ce == cudaSuccess) ce = mk::launch_rope_table((float2*)(A + L.rope), c.max_ctx, G.hd, c.rope_theta, stream);
+  if (ce == cudaSuccess) ce = cudaStreamSynchronize(stream);
+  if (ce != cudaSuccess) return cuda_fail(nullptr, ce, (std::string(who) + ": upload").c_str());
+  return MK_OK;
+}
+
+// Kernel parameters (all but the per-step fields) of a plan laid out at `A`.
+static KParams make_kparams(const mk_plan_s& plan, const mk_weight_ptrs* w, const Layout& L, unsigned char* A,
+                            int* status) {
+  const mk_model_cfg& c = plan.cfg;
+  const mk::Geometry G = mk::geometry(c);
+  KParams k{};
+  k.L = G.L; k.d = G.d; k.nq = G.nq; k.nkv = G.nkv; k.hd = G.hd; k.F = G.F; k.V = G.V; k.g = G.g;
+  k.qdim = G.qdim; k.max_b = c.max_batch; k.max_ctx = c.max_ctx; k.eps = c.rms_eps;
+  k.layers = (const LayerW*)(A + L.layers);
+  k.embed = (const __nv_bfloat16*)w->embed;
+  k.final_norm = (const __nv_bfloat16*)w->final_norm;
+  k.lm_head = (const __nv_bfloat16*)w->lm_head;
+  k.tasks = (const mk::TaskDesc*)(A + L.tasks);
+  k.task_off = (const uint32_t*)(A + L.offs);
+  k.num_sms = plan.num_sms;
+  k.n_slots = plan.num_sms * plan.attn_slots_per_sm;
+  k.n_lm_tasks = plan.n_lm_tasks;
+  k.tmaps = A + L.maps;
+  k.x = (float*)(A + L.x);
+  k.q = (float*)(A + L.q);
+  auto carve = [&](size_t o, int ld, __nv_bfloat16** t, float** f) {
+    *t = (__nv_bfloat16*)(A + o);
+    *f = (float*)(*t + (size_t)L.ntiles * 2 * ld * 8);
+  };
+  carve(L.ax, L.ld_x, &k.ax_t, &k.ax_f);
+  carve(L.aa, L.ld_a, &k.aa_t, &k.aa_f);
+  carve(L.ah, L.ld_h, &k.ah_t, &k.ah_f);
+  k.ld_x = L.ld_x; k.ld_a = L.ld_a; k.ld_h = L.ld_h;
+  k.ssq = (float*)(A + L.ssq);
+  k.ssq_stride = L.ssq_stride;
+  k.part = (float*)(A + L.part);
+  k.lmpart = (float2*)(A + L.lmpart);
+  k.spart = (float*)(A + L.spart);
+  k.scnt = (uint32_t*)(A + L.scnt);
+  k.n_split = L.nsplit;
+  k.ctr = (uint32_t*)(A + L.ctr);
+  k.cmb = (uint32_t*)(A + L.cmb);
+  k.ctl = (uint32_t*)(A + L.ctl);
+  k.host_status = status;
+  k.rope = (const float2*)(A + L.rope);
+  k.timeout_ns = 1000000000ull;
+  k.dbg = nullptr;
+  k.trace = nullptr;
+  return k;
+}
+
+// Zero what the kernel expects at zero after a failed step: dependency, combine and K-piece
+// counters, the abort flag and first error code.
+static cudaError_t clear_counters(const KParams& k, cudaStream_t s) {
+  cudaError_t ce = cudaMemsetAsync(k.ctr, 0, sizeof(uint32_t) * mk::num_counters(k.L), s);
+  if (ce == cudaSuccess) ce = cudaMemsetAsync(k.cmb, 0, sizeof(uint32_t) * (size_t)k.L * k.max_b * k.nkv, s);
+  if (ce == cudaSuccess) ce = cudaMemsetAsync(k.ctl, 0, sizeof(uint32_t) * 2, s);
+  if (ce == cudaSuccess) ce = cudaMemsetAsync(k.scnt, 0, sizeof(uint32_t) * (size_t)k.n_split, s);
+  return ce;
+}
+
 extern "C" {
 
 MK_API int mk_create_from_plan(mk_plan_t plan, const mk_weight_ptrs* w, int32_t flags, mk_handle_t* out) {
@@ -199,160 +392,40 @@ MK_API int mk_create_from_plan(mk_plan_t plan, const mk_weight_ptrs* w, int32_t 
     int rc = mk::validate_plan(*plan, &e);
     if (rc) return fail(nullptr, rc, "schedule rejected: " + e);
   }
-  // weights
-  if (!w->embed || !w->final_norm || !w->lm_head || !w->attn_norm || !w->wq || !w->wk || !w->wv || !w->wo ||
-      !w->mlp_norm || !w->w_gate || !w->w_up || !w->w_down)
-    return fail(nullptr, MK_ERR_INVALID_ARG, "mk_create: null weight pointer");
-  std::vector<LayerW> lw(c.n_layers);
-  const void* all[3] = {w->embed, w->final_norm, w->lm_head};
-  for (const void* p : all)
-    if (!aligned16(p)) return fail(nullptr, MK_ERR_INVALID_ARG, "mk_create: weights must be 16-byte aligned");
-  for (int l = 0; l < c.n_layers; ++l) {
-    const void* ps[9] = {w->attn_norm[l], w->wq[l], w->wk[l], w->wv[l], w->wo[l],
-                         w->mlp_norm[l], w->w_gate[l], w->w_up[l], w->w_down[l]};
-    for (const void* p : ps)
-      if (!p || !aligned16(p))
-        return fail(nullptr, MK_ERR_INVALID_ARG, "mk_create: layer weight null or not 16-byte aligned");
-    lw[l] = LayerW{(const __nv_bfloat16*)ps[0], (const __nv_bfloat16*)ps[1], (const __nv_bfloat16*)ps[2],
-                   (const __nv_bfloat16*)ps[3], (const __nv_bfloat16*)ps[4], (const __nv_bfloat16*)ps[5],
-                   (const __nv_bfloat16*)ps[6], (const __nv_bfloat16*)ps[7], (const __nv_bfloat16*)ps[8]};
-  }
-
+  std::vector<LayerW> lw;
+  e = collect_layers(c, w, lw);
+  if (!e.empty()) return fail(nullptr, MK_ERR_INVALID_ARG, "mk_create: " + e);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return fail(nullptr, MK_ERR_NO_DEVICE, "no CUDA device");
-  cudaDeviceProp prop;
-  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return fail(nullptr, MK_ERR_NO_DEVICE, "no CUDA device");
-  if (prop.major != 10) return fail(nullptr, MK_ERR_NO_DEVICE, "the kernel is built for sm_100a (B200)");
-  if (!prop.cooperativeLaunch) return fail(nullptr, MK_ERR_NO_DEVICE, "device lacks cooperative launch");
-  if (plan->num_sms != prop.multiProcessorCount)
+  int rc = check_device(dev, "mk_create");
+  if (rc) return rc;
+  int nsm = 0;
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  if (plan->num_sms != nsm)
     return fail(nullptr, MK_ERR_INVALID_ARG,
-                "plan built for " + std::to_string(plan->num_sms) + " SMs, device has " +
-                    std::to_string(prop.multiProcessorCount));
+                "plan built for " + std::to_string(plan->num_sms) + " SMs, device has " + std::to_string(nsm));
 
   mk_handle_t h = new mk_handle_s();
   h->plan = *plan;
   h->device = dev;
-  int regs = 0, lmem = 0, maxthr = 0;
-  cudaError_t ce = mk::kernel_attributes(&regs, &lmem, &maxthr);
-  if (ce != cudaSuccess) { release(h); return cuda_fail(nullptr, ce, "kernel attributes"); }
-  if (maxthr < mk::kThreads) { release(h); return fail(nullptr, MK_ERR_CUDA, "kernel cannot run its " + std::to_string(mk::kThreads) + " threads"); }
-
-  const mk::Geometry G = mk::geometry(c);
-  const int S = plan->num_sms * plan->attn_slots_per_sm;
-  const int mb = c.max_batch;
-  // device arena layout (256-byte aligned pieces)
-  size_t off = 0;
-  auto take = [&](size_t bytes) { size_t o = off; off += (bytes + 255) & ~size_t(255); return o; };
-  std::vector<mk::TaskDesc> flat;
-  std::vector<uint32_t> offs(plan->num_sms + 1, 0);
-  for (int s = 0; s < plan->num_sms; ++s) {
-    flat.insert(flat.end(), plan->streams[s].begin(), plan->streams[s].end());
-    offs[s + 1] = (uint32_t)flat.size();
-  }
-  const size_t o_layers = take(sizeof(LayerW) * c.n_layers);
-  const size_t o_tasks = take(sizeof(mk::TaskDesc) * flat.size());
-  const size_t o_offs = take(sizeof(uint32_t) * offs.size());
-  std::vector<CUtensorMap> maps;
-  std::string merr = build_tensor_maps(c, w, maps);
-  if (!merr.empty()) { release(h); return fail(nullptr, MK_ERR_CUDA, merr); }
-  const size_t o_maps = take(sizeof(CUtensorMap) * (size_t)mk::num_all_tmaps(G.L));
-  const size_t o_x = take(sizeof(float) * mb * G.d);
-  const size_t o_q = take(sizeof(float) * mb * G.qdim);
-  const int ld_x = mk::round_up(G.d, mk::kBoxCols), ld_a = mk::round_up(G.qdim, mk::kBoxCols),
-            ld_h = mk::round_up(G.F, mk::kBoxCols);
-  // operands: bf16 hi/lo tiles of 8 batch rows (operand_index layout) and the fp32 batch row 0,
-  // zero padded to whole 64-column boxes
-  const int ntiles = (mb + 7) / 8;
-  auto opbytes = [&](int ld) { return (size_t)ntiles * 2 * ld * 8 * 2 + (size_t)mk::kFmaRows * ld * 4; };
-  const size_t o_ax = take(opbytes(ld_x)), o_aa = take(opbytes(ld_a)), o_ah = take(opbytes(ld_h));
-  const int ssq_stride = plan->max_phase_tasks * mb;
-  const size_t o_ssq = take(sizeof(float) * mk::num_ssq_inst(G.L) * ssq_stride);
-  const size_t o_part = take(sizeof(float) * (size_t)mb * G.nkv * mk::kMaxChunksPerSeq * G.g * (G.hd + 2));
-  const size_t o_lm = take(sizeof(float2) * (size_t)plan->n_lm_tasks * mb);
-  const int nsplit = plan->max_split_ids > 0 ? plan->max_split_ids : 1;
-  const size_t o_spart = take(sizeof(float) * (size_t)nsplit * mk::kMaxPieces * mk::kMaxBlocks * 8 * mb);
-  const size_t o_scnt = take(sizeof(uint32_t) * (size_t)nsplit);
-  const size_t o_ctr = take(sizeof(uint32_t) * mk::num_counters(G.L));
-  const size_t o_cmb = take(sizeof(uint32_t) * (size_t)G.L * mb * G.nkv);
-  const size_t o_ctl = take(sizeof(uint32_t) * 2);
-  const size_t o_rope = take(sizeof(float2) * (size_t)c.max_ctx * (G.hd / 2));
-  const size_t o_stage = take(sizeof(int32_t) * 3 * mb);
-  const size_t o_logits = take(sizeof(float) * (size_t)mb * G.V);
-  const size_t o_argmax = take(sizeof(int32_t) * mb);
-  const size_t total = off;
-
-  ce = cudaMalloc(&h->arena, total);
-  if (ce != cudaSuccess) { release(h); return cuda_fail(nullptr, ce, "cudaMalloc(scratch)"); }
-  ce = cudaMemset(h->arena, 0, total);
+  const Layout L = layout_scratch(*plan, true);
+  cudaError_t ce = cudaMalloc(&h->arena, L.total);
   if (ce == cudaSuccess) ce = cudaHostAlloc((void**)&h->host_status, sizeof(int), cudaHostAllocMapped);
-  if (ce == cudaSuccess) ce = cudaHostAlloc((void**)&h->h_stage, sizeof(int32_t) * 3 * mb, cudaHostAllocDefault);
+  if (ce == cudaSuccess) ce = cudaHostAlloc((void**)&h->h_stage, sizeof(int32_t) * 3 * c.max_batch, cudaHostAllocDefault);
   if (ce != cudaSuccess) { release(h); return cuda_fail(nullptr, ce, "scratch allocation"); }
   *h->host_status = 0;
   int* dev_status = nullptr;
   ce = cudaHostGetDevicePointer((void**)&dev_status, h->host_status, 0);
   if (ce != cudaSuccess) { release(h); return cuda_fail(nullptr, ce, "cudaHostGetDevicePointer"); }
-
-  char* A = (char*)h->arena;
-  {
-    auto tl = [&](size_t o) { return (const __nv_bfloat16*)(A + o); };
-    auto rw = [&](size_t o, int ld) { return (const float*)(A + o + (size_t)ntiles * 2 * ld * 8 * 2); };
-    const __nv_bfloat16* tiles[3] = {tl(o_ax), tl(o_aa), tl(o_ah)};
-    const float* rows[3] = {rw(o_ax, ld_x), rw(o_aa, ld_a), rw(o_ah, ld_h)};
-    const int lds[3] = {ld_x, ld_a, ld_h};
-    merr = encode_operand_maps(maps, G.L, ntiles, tiles, rows, lds);
-    if (!merr.empty()) { release(h); return fail(nullptr, MK_ERR_CUDA, merr); }
-  }
-  ce = cudaMemcpy(A + o_layers, lw.data(), sizeof(LayerW) * c.n_layers, cudaMemcpyHostToDevice);
-  if (ce == cudaSuccess)
-    ce = cudaMemcpy(A + o_tasks, flat.data(), sizeof(mk::TaskDesc) * flat.size(), cudaMemcpyHostToDevice);
-  if (ce == cudaSuccess)
-    ce = cudaMemcpy(A + o_offs, offs.data(), sizeof(uint32_t) * offs.size(), cudaMemcpyHostToDevice);
-  if (ce == cudaSuccess)
-    ce = cudaMemcpy(A + o_maps, maps.data(), sizeof(CUtensorMap) * maps.size(), cudaMemcpyHostToDevice);
-  if (ce == cudaSuccess) ce = mk::launch_rope_table((float2*)(A + o_rope), c.max_ctx, G.hd, c.rope_theta, 0);
-  if (ce == cudaSuccess) ce = cudaDeviceSynchronize();
-  if (ce != cudaSuccess) { release(h); return cuda_fail(nullptr, ce, "upload"); }
-
-  KParams& k = h->kp;
-  k.L = G.L; k.d = G.d; k.nq = G.nq; k.nkv = G.nkv; k.hd = G.hd; k.F = G.F; k.V = G.V; k.g = G.g;
-  k.qdim = G.qdim; k.max_b = mb; k.max_ctx = c.max_ctx; k.eps = c.rms_eps;
-  k.layers = (const LayerW*)(A + o_layers);
-  k.embed = (const __nv_bfloat16*)w->embed;
-  k.final_norm = (const __nv_bfloat16*)w->final_norm;
-  k.lm_head = (const __nv_bfloat16*)w->lm_head;
-  k.tasks = (const mk::TaskDesc*)(A + o_tasks);
-  k.task_off = (const uint32_t*)(A + o_offs);
-  k.num_sms = plan->num_sms;
-  k.n_slots = S;
-  k.n_lm_tasks = plan->n_lm_tasks;
-  k.tmaps = A + o_maps;
-  k.x = (float*)(A + o_x); k.q = (float*)(A + o_q);
-  auto carve = [&](size_t o, int ld, __nv_bfloat16** t, float** f) {
-    *t = (__nv_bfloat16*)(A + o);
-    *f = (float*)(*t + (size_t)ntiles * 2 * ld * 8);
-  };
-  carve(o_ax, ld_x, &k.ax_t, &k.ax_f);
-  carve(o_aa, ld_a, &k.aa_t, &k.aa_f);
-  carve(o_ah, ld_h, &k.ah_t, &k.ah_f);
-  k.ld_x = ld_x; k.ld_a = ld_a; k.ld_h = ld_h;
-  k.ssq = (float*)(A + o_ssq); k.ssq_stride = ssq_stride; k.part = (float*)(A + o_part);
-  k.lmpart = (float2*)(A + o_lm);
-  k.spart = (float*)(A + o_spart);
-  k.scnt = (uint32_t*)(A + o_scnt);
-  k.n_split = nsplit;
-  k.ctr = (uint32_t*)(A + o_ctr); k.cmb = (uint32_t*)(A + o_cmb); k.ctl = (uint32_t*)(A + o_ctl);
-  k.host_status = dev_status;
-  k.rope = (const float2*)(A + o_rope);
-  k.timeout_ns = 1000000000ull;
-  k.dbg = nullptr;
-  k.trace = nullptr;
-  h->d_stage = (int32_t*)(A + o_stage);
-  h->d_logits = (float*)(A + o_logits);
-  h->d_argmax = (int32_t*)(A + o_argmax);
-  // bookkeeping for mk_reset
+  unsigned char* A = (unsigned char*)h->arena;
+  rc = upload_tables(*plan, w, lw, L, A, 0, "mk_create");
+  if (rc) { release(h); return rc; }
+  h->kp = make_kparams(*plan, w, L, A, dev_status);
+  h->d_stage = (int32_t*)(A + L.stage);
+  h->d_logits = (float*)(A + L.logits);
+  h->d_argmax = (int32_t*)(A + L.argmax);
   h->err.clear();
   *out = h;
-  (void)o_ctl;
   return MK_OK;
 }
 
@@ -457,11 +530,7 @@ MK_API int mk_get_status(mk_handle_t h) {
 MK_API int mk_reset(mk_handle_t h) {
   if (!h) return MK_ERR_INVALID_ARG;
   MK_CUDA(h, cudaDeviceSynchronize());
-  KParams& k = h->kp;
-  MK_CUDA(h, cudaMemset(k.ctr, 0, sizeof(uint32_t) * mk::num_counters(k.L)));
-  MK_CUDA(h, cudaMemset(k.cmb, 0, sizeof(uint32_t) * (size_t)k.L * k.max_b * k.nkv));
-  MK_CUDA(h, cudaMemset(k.ctl, 0, sizeof(uint32_t) * 2));
-  MK_CUDA(h, cudaMemset(k.scnt, 0, sizeof(uint32_t) * k.n_split));
+  MK_CUDA(h, clear_counters(h->kp, 0));
   MK_CUDA(h, cudaDeviceSynchronize());
   *(volatile int*)h->host_status = 0;
   h->epoch = 0;
@@ -566,151 +635,34 @@ bool same_key(const StaticState& s, const mk_model_cfg& c, const mk_weight_ptrs*
 }
 
 // Build the schedule and tensor maps for (cfg, weights), lay the scratch out in the static
-// array, clear it and upload the tables.  Host-synchronous on `stream`.
+// array (the same layout as a handle's arena, without the host-buffer pieces), clear it and
+// upload the tables.  Host-synchronous on `stream`.
 int static_setup(StaticState& s, const mk_model_cfg& c, const mk_weight_ptrs* w, int dev, cudaStream_t stream) {
   s.ready = false;
-  if (!w->embed || !w->final_norm || !w->lm_head || !w->attn_norm || !w->wq || !w->wk || !w->wv || !w->wo ||
-      !w->mlp_norm || !w->w_gate || !w->w_up || !w->w_down)
-    return fail(nullptr, MK_ERR_INVALID_ARG, "mk_decode_step_static: null weight pointer");
-  std::vector<LayerW> lw(c.n_layers > 0 ? c.n_layers : 0);
-  const void* all[3] = {w->embed, w->final_norm, w->lm_head};
-  for (const void* p : all)
-    if (!aligned16(p)) return fail(nullptr, MK_ERR_INVALID_ARG, "mk_decode_step_static: weights must be 16-byte aligned");
-  for (int l = 0; l < c.n_layers; ++l) {
-    const void* ps[9] = {w->attn_norm[l], w->wq[l], w->wk[l], w->wv[l], w->wo[l],
-                         w->mlp_norm[l], w->w_gate[l], w->w_up[l], w->w_down[l]};
-    for (const void* p : ps)
-      if (!p || !aligned16(p))
-        return fail(nullptr, MK_ERR_INVALID_ARG, "mk_decode_step_static: layer weight null or not 16-byte aligned");
-    lw[l] = LayerW{(const __nv_bfloat16*)ps[0], (const __nv_bfloat16*)ps[1], (const __nv_bfloat16*)ps[2],
-                   (const __nv_bfloat16*)ps[3], (const __nv_bfloat16*)ps[4], (const __nv_bfloat16*)ps[5],
-                   (const __nv_bfloat16*)ps[6], (const __nv_bfloat16*)ps[7], (const __nv_bfloat16*)ps[8]};
-  }
-  cudaDeviceProp prop;
-  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return fail(nullptr, MK_ERR_NO_DEVICE, "no CUDA device");
-  if (prop.major != 10) return fail(nullptr, MK_ERR_NO_DEVICE, "the kernel is built for sm_100a (B200)");
-  if (!prop.cooperativeLaunch) return fail(nullptr, MK_ERR_NO_DEVICE, "device lacks cooperative launch");
-  int regs = 0, lmem = 0, maxthr = 0;
-  cudaError_t ce = mk::kernel_attributes(&regs, &lmem, &maxthr);
-  if (ce != cudaSuccess) return cuda_fail(nullptr, ce, "kernel attributes");
-  if (maxthr < mk::kThreads) return fail(nullptr, MK_ERR_CUDA, "kernel cannot run its " + std::to_string(mk::kThreads) + " threads");
-
+  std::vector<LayerW> lw;
+  const std::string e = collect_layers(c, w, lw);
+  if (!e.empty()) return fail(nullptr, MK_ERR_INVALID_ARG, "mk_decode_step_static: " + e);
+  int rc = check_device(dev, "mk_decode_step_static");
+  if (rc) return rc;
   mk_plan_opts o{};
-  o.num_sms = prop.multiProcessorCount;
+  cudaDeviceGetAttribute(&o.num_sms, cudaDevAttrMultiProcessorCount, dev);
   mk_plan_s plan;
-  std::string e;
-  int rc = mk::build_plan(c, &o, &plan, &e);
-  if (rc) return fail(nullptr, rc, "plan: " + e);
-  rc = mk::validate_plan(plan, &e);
-  if (rc) return fail(nullptr, rc, "schedule rejected: " + e);
-
-  const mk::Geometry G = mk::geometry(c);
-  const int S = plan.num_sms * plan.attn_slots_per_sm;
-  const int mb = c.max_batch;
-  size_t off = 0;
-  auto take = [&](size_t bytes) { size_t at = off; off += (bytes + 255) & ~size_t(255); return at; };
-  std::vector<mk::TaskDesc> flat;
-  std::vector<uint32_t> offs(plan.num_sms + 1, 0);
-  for (int sm = 0; sm < plan.num_sms; ++sm) {
-    flat.insert(flat.end(), plan.streams[sm].begin(), plan.streams[sm].end());
-    offs[sm + 1] = (uint32_t)flat.size();
-  }
-  const size_t o_layers = take(sizeof(LayerW) * c.n_layers);
-  const size_t o_tasks = take(sizeof(mk::TaskDesc) * flat.size());
-  const size_t o_offs = take(sizeof(uint32_t) * offs.size());
-  const size_t o_maps = take(sizeof(CUtensorMap) * (size_t)mk::num_all_tmaps(G.L));
-  const size_t o_x = take(sizeof(float) * mb * G.d);
-  const size_t o_q = take(sizeof(float) * mb * G.qdim);
-  const int ld_x = mk::round_up(G.d, mk::kBoxCols), ld_a = mk::round_up(G.qdim, mk::kBoxCols),
-            ld_h = mk::round_up(G.F, mk::kBoxCols);
-  const int ntiles = (mb + 7) / 8;
-  auto opbytes = [&](int ld) { return (size_t)ntiles * 2 * ld * 8 * 2 + (size_t)mk::kFmaRows * ld * 4; };
-  const size_t o_ax = take(opbytes(ld_x)), o_aa = take(opbytes(ld_a)), o_ah = take(opbytes(ld_h));
-  const int ssq_stride = plan.max_phase_tasks * mb;
-  const size_t o_ssq = take(sizeof(float) * mk::num_ssq_inst(G.L) * ssq_stride);
-  const size_t o_part = take(sizeof(float) * (size_t)mb * G.nkv * mk::kMaxChunksPerSeq * G.g * (G.hd + 2));
-  const size_t o_lm = take(sizeof(float2) * (size_t)plan.n_lm_tasks * mb);
-  const int nsplit = plan.max_split_ids > 0 ? plan.max_split_ids : 1;
-  const size_t o_spart = take(sizeof(float) * (size_t)nsplit * mk::kMaxPieces * mk::kMaxBlocks * 8 * mb);
-  const size_t o_scnt = take(sizeof(uint32_t) * (size_t)nsplit);
-  const size_t o_ctr = take(sizeof(uint32_t) * mk::num_counters(G.L));
-  const size_t o_cmb = take(sizeof(uint32_t) * (size_t)G.L * mb * G.nkv);
-  const size_t o_ctl = take(sizeof(uint32_t) * 2);
-  const size_t o_status = take(sizeof(int));
-  const size_t o_rope = take(sizeof(float2) * (size_t)c.max_ctx * (G.hd / 2));
-  const size_t total = off;
-  if (total > kStaticScratchBytes)
+  std::string pe;
+  rc = mk::build_plan(c, &o, &plan, &pe);
+  if (rc) return fail(nullptr, rc, "plan: " + pe);
+  rc = mk::validate_plan(plan, &pe);
+  if (rc) return fail(nullptr, rc, "schedule rejected: " + pe);
+  const Layout L = layout_scratch(plan, false);
+  if (L.total > kStaticScratchBytes)
     return fail(nullptr, MK_ERR_INVALID_ARG,
-                "mk_decode_step_static: this model needs " + std::to_string(total) +
+                "mk_decode_step_static: this model needs " + std::to_string(L.total) +
                     " bytes of scratch; the static area holds " + std::to_string(kStaticScratchBytes) +
                     " (lower max_batch or max_ctx, or use mk_create)");
-
-  std::vector<CUtensorMap> maps;
-  std::string merr = build_tensor_maps(c, w, maps);
-  if (!merr.empty()) return fail(nullptr, MK_ERR_CUDA, merr);
-
-  unsigned char* A = s.base;
-  {
-    auto tl = [&](size_t o) { return (const __nv_bfloat16*)(A + o); };
-    auto rw = [&](size_t o, int ld) { return (const float*)(A + o + (size_t)ntiles * 2 * ld * 8 * 2); };
-    const __nv_bfloat16* tiles[3] = {tl(o_ax), tl(o_aa), tl(o_ah)};
-    const float* rows[3] = {rw(o_ax, ld_x), rw(o_aa, ld_a), rw(o_ah, ld_h)};
-    const int lds[3] = {ld_x, ld_a, ld_h};
-    merr = encode_operand_maps(maps, G.L, ntiles, tiles, rows, lds);
-    if (!merr.empty()) return fail(nullptr, MK_ERR_CUDA, merr);
-  }
-  ce = cudaMemsetAsync(A, 0, total, stream);
-  if (ce == cudaSuccess)
-    ce = cudaMemcpyAsync(A + o_layers, lw.data(), sizeof(LayerW) * c.n_layers, cudaMemcpyHostToDevice, stream);
-  if (ce == cudaSuccess)
-    ce = cudaMemcpyAsync(A + o_tasks, flat.data(), sizeof(mk::TaskDesc) * flat.size(), cudaMemcpyHostToDevice,
-                         stream);
-  if (ce == cudaSuccess)
-    ce = cudaMemcpyAsync(A + o_offs, offs.data(), sizeof(uint32_t) * offs.size(), cudaMemcpyHostToDevice, stream);
-  if (ce == cudaSuccess)
-    ce = cudaMemcpyAsync(A + o_maps, maps.data(), sizeof(CUtensorMap) * maps.size(), cudaMemcpyHostToDevice,
-                         stream);
-  if (ce == cudaSuccess)
-    ce = mk::launch_rope_table((float2*)(A + o_rope), c.max_ctx, G.hd, c.rope_theta, stream);
-  if (ce == cudaSuccess) ce = cudaStreamSynchronize(stream);
-  if (ce != cudaSuccess) return cuda_fail(nullptr, ce, "mk_decode_step_static: upload");
-
-  KParams k{};
-  k.L = G.L; k.d = G.d; k.nq = G.nq; k.nkv = G.nkv; k.hd = G.hd; k.F = G.F; k.V = G.V; k.g = G.g;
-  k.qdim = G.qdim; k.max_b = mb; k.max_ctx = c.max_ctx; k.eps = c.rms_eps;
-  k.layers = (const LayerW*)(A + o_layers);
-  k.embed = (const __nv_bfloat16*)w->embed;
-  k.final_norm = (const __nv_bfloat16*)w->final_norm;
-  k.lm_head = (const __nv_bfloat16*)w->lm_head;
-  k.tasks = (const mk::TaskDesc*)(A + o_tasks);
-  k.task_off = (const uint32_t*)(A + o_offs);
-  k.num_sms = plan.num_sms;
-  k.n_slots = S;
-  k.n_lm_tasks = plan.n_lm_tasks;
-  k.tmaps = A + o_maps;
-  k.x = (float*)(A + o_x); k.q = (float*)(A + o_q);
-  auto carve = [&](size_t at, int ld, __nv_bfloat16** t, float** f) {
-    *t = (__nv_bfloat16*)(A + at);
-    *f = (float*)(*t + (size_t)ntiles * 2 * ld * 8);
-  };
-  carve(o_ax, ld_x, &k.ax_t, &k.ax_f);
-  carve(o_aa, ld_a, &k.aa_t, &k.aa_f);
-  carve(o_ah, ld_h, &k.ah_t, &k.ah_f);
-  k.ld_x = ld_x; k.ld_a = ld_a; k.ld_h = ld_h;
-  k.ssq = (float*)(A + o_ssq); k.ssq_stride = ssq_stride; k.part = (float*)(A + o_part);
-  k.lmpart = (float2*)(A + o_lm);
-  k.spart = (float*)(A + o_spart);
-  k.scnt = (uint32_t*)(A + o_scnt);
-  k.n_split = nsplit;
-  k.ctr = (uint32_t*)(A + o_ctr); k.cmb = (uint32_t*)(A + o_cmb); k.ctl = (uint32_t*)(A + o_ctl);
-  k.host_status = (int*)(A + o_status);
-  k.rope = (const float2*)(A + o_rope);
-  k.timeout_ns = 1000000000ull;
-  k.dbg = nullptr;
-  k.trace = nullptr;
-  s.kp = k;
+  rc = upload_tables(plan, w, lw, L, s.base, stream, "mk_decode_step_static");
+  if (rc) return rc;
+  s.kp = make_kparams(plan, w, L, s.base, (int*)(s.base + L.status));
   s.kv_k = s.kv_v = nullptr;
-  s.status = (int*)(A + o_status);
+  s.status = (int*)(s.base + L.status);
   s.cfg = c;
   weight_key(c, w, &s.wkey);
   s.epoch = 0;
@@ -719,14 +671,10 @@ int static_setup(StaticState& s, const mk_model_cfg& c, const mk_weight_ptrs* w,
   return MK_OK;
 }
 
-// Zero what the kernel expects to start at zero after a failed step: the dependency and
-// combine counters, the abort flag and first error code, the status word.
+// Zero what the kernel expects to start at zero after a failed step: the counters, the abort
+// flag and first error code, the status word.
 cudaError_t static_clear(StaticState& s, cudaStream_t stream) {
-  const KParams& k = s.kp;
-  cudaError_t ce = cudaMemsetAsync(k.ctr, 0, sizeof(uint32_t) * mk::num_counters(k.L), stream);
-  if (ce == cudaSuccess) ce = cudaMemsetAsync(k.cmb, 0, sizeof(uint32_t) * (size_t)k.L * k.max_b * k.nkv, stream);
-  if (ce == cudaSuccess) ce = cudaMemsetAsync(k.ctl, 0, sizeof(uint32_t) * 2, stream);
-  if (ce == cudaSuccess) ce = cudaMemsetAsync(k.scnt, 0, sizeof(uint32_t) * k.n_split, stream);
+  cudaError_t ce = clear_counters(s.kp, stream);
   if (ce == cudaSuccess) ce = cudaMemsetAsync(s.status, 0, sizeof(int), stream);
   return ce;
 }
@@ -755,12 +703,17 @@ extern "C" MK_API int mk_decode_step_static(const mk_model_cfg* cfg, const mk_we
   std::lock_guard<std::mutex> lock(g_static_mu[dev]);
   StaticState& s = g_static[dev];
   cudaStream_t st = (cudaStream_t)stream;
-  if (!s.base) {
-    // once per device, with that device current: the address of this device's copy of the array
+  {
+    // the address of this device's copy of the array, looked up with the device current on every
+    // call (it is cheap): if the module was loaded anew (after a device reset), the tables are
+    // gone and the set-up runs again
     void* p = nullptr;
     cudaError_t ce = cudaGetSymbolAddress(&p, g_static_scratch);
     if (ce != cudaSuccess) return cuda_fail(nullptr, ce, "mk_decode_step_static: cudaGetSymbolAddress");
-    s.base = (unsigned char*)p;
+    if ((unsigned char*)p != s.base) {
+      s.base = (unsigned char*)p;
+      s.ready = false;
+    }
   }
   if (!same_key(s, *cfg, weights)) {
     rc = static_setup(s, *cfg, weights, dev, st);

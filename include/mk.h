@@ -172,11 +172,11 @@ MK_API int mk_decode_step_host(mk_handle_t h, const int32_t *token_ids, const in
  * maps, activations, counters, RoPE table).  A model whose scratch exceeds it (it
  * grows with n_layers, max_batch and max_ctx) is rejected with MK_ERR_INVALID_ARG
  * before anything is launched.  No call allocates device or pinned host memory.
- * Set-up: the first call on a device (with that device current) looks the array's
- * address up, builds and validates the schedule, encodes the tensor maps, clears the
- * array and uploads the tables, synchronising `stream`; a later call with another cfg
- * or other weight pointers does the same again.  Make the first call before any
- * stream capture.
+ * Set-up: every call looks the array's address up on the current device; the first
+ * call on a device (and any call after the array moved, as after a device reset, or
+ * with another cfg or other weight pointers) builds and validates the schedule, encodes
+ * the tensor maps, clears the array and uploads the tables, synchronising `stream`.
+ * Make the first call before any stream capture.
  * Each call synchronises `stream` and returns the step's device status (MK_OK,
  * MK_ERR_DEVICE_TIMEOUT, MK_ERR_BOUNDS); after a device error the next call first
  * clears the counters and the status.  All calls on a device share the one array, so
