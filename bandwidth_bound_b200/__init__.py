@@ -88,6 +88,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "mk_create_from_plan": (ctypes.c_int, [vp, ctypes.POINTER(WeightPtrs), i32, ctypes.POINTER(vp)]),
         "mk_decode_step": (ctypes.c_int, [vp, vp, vp, vp, i32, ctypes.POINTER(KvCache), vp, vp, vp]),
         "mk_decode_step_host": (ctypes.c_int, [vp, vp, vp, vp, i32, ctypes.POINTER(KvCache), vp, vp, vp]),
+        "mk_decode_steps": (ctypes.c_int, [vp, i32, vp, vp, i32, ctypes.POINTER(KvCache), ctypes.POINTER(Sampling),
+                                           vp, vp, vp]),
         "mk_decode_step_static": (ctypes.c_int, [ctypes.POINTER(ModelCfg), ctypes.POINTER(WeightPtrs), vp, vp, vp,
                                                  i32, ctypes.POINTER(KvCache), vp, vp, vp]),
         "mk_get_status": (ctypes.c_int, [vp]),
@@ -181,6 +183,14 @@ def _ptr(t) -> int:
     return 0 if t is None else int(t.data_ptr())
 
 
+class Sampling(ctypes.Structure):
+    """mk_sampling: top-k sampling of the next token (top_k <= 1: greedy)."""
+    _fields_ = [("top_k", ctypes.c_int32), ("temperature", ctypes.c_float), ("uniforms", ctypes.c_void_p)]
+
+
+MAX_TOP_K = 256
+
+
 class Megakernel:
     """A handle of the decode megakernel bound to one model's device weights.
 
@@ -230,6 +240,23 @@ class Megakernel:
                                      ctypes.c_void_p(stream.cuda_stream))
         if check:
             _check(rc, self.handle, "mk_decode_step")
+        return rc
+
+    def steps(self, n_steps: int, token_ids, positions, kv, tokens_out, logits=None, stream=None,
+              check: bool = True, top_k: int = 1, temperature: float = 1.0, uniforms=None) -> int:
+        """n_steps steps in one call: step k feeds the token step k-1 chose at positions + k.
+        tokens_out: device int32 [n_steps][batch]; logits (optional): the last step's.
+        top_k > 1 samples among the top_k logits at `temperature` with the device fp32
+        uniforms [n_steps][batch]; otherwise the choice is greedy."""
+        if stream is None:
+            stream = self._torch.cuda.current_stream()
+        kvs = self.kv_struct(kv)
+        smp = Sampling(int(top_k), float(temperature), _ptr(uniforms))
+        rc = self.lib.mk_decode_steps(self.handle, int(n_steps), _ptr(token_ids), _ptr(positions),
+                                      int(token_ids.numel()), ctypes.byref(kvs), ctypes.byref(smp), _ptr(tokens_out),
+                                      _ptr(logits), ctypes.c_void_p(stream.cuda_stream))
+        if check:
+            _check(rc, self.handle, "mk_decode_steps")
         return rc
 
     def step_host(self, token_ids, positions, seq_lens, kv, logits_host=None, argmax_host=None, stream=None,

@@ -4,12 +4,15 @@
 #include <cuda_runtime.h>
 
 #include <cstdio>
+#include <cmath>
 #include <cstring>
 #include <string>
 #include <vector>
 
 #include "mk_kernel.h"
 #include "mk_plan.h"
+
+static_assert(mk::kMaxTopK == MK_MAX_TOP_K, "the kernel's top-k bound is the ABI's");
 
 using mk::KParams;
 static_assert(sizeof(mk::TmaDesc) == sizeof(CUtensorMap), "TMA descriptor size");
@@ -234,7 +237,8 @@ static int check_device(int dev, const char* who) {
 // Byte offsets of the scratch pieces (256-byte aligned).  The last three serve only the
 // handle's host-buffer entry point.
 struct Layout {
-  size_t layers, tasks, offs, maps, x, q, ax, aa, ah, ssq, part, lmpart, spart, scnt, ctr, cmb, ctl, status, rope;
+  size_t layers, tasks, offs, maps, x, q, ax, aa, ah, ssq, part, lmpart, lmrows, spart, scnt, ctr, cmb, ctl, status,
+      rope;
   size_t stage, logits, argmax;
   size_t total;
   int ld_x, ld_a, ld_h, ntiles, ssq_stride, nsplit;
@@ -274,6 +278,7 @@ static Layout layout_scratch(const mk_plan_s& plan, bool host_step) {
   L.ssq = take(sizeof(float) * (size_t)mk::num_ssq_inst(G.L) * L.ssq_stride);
   L.part = take(sizeof(float) * (size_t)mb * G.nkv * mk::kMaxChunksPerSeq * G.g * (G.hd + 2));
   L.lmpart = take(sizeof(float2) * (size_t)plan.n_lm_tasks * mb);
+  L.lmrows = take(sizeof(int2) * (size_t)plan.n_lm_tasks);
   L.nsplit = plan.max_split_ids > 0 ? plan.max_split_ids : 1;
   L.spart = take(sizeof(float) * (size_t)L.nsplit * mk::kMaxPieces * mk::kMaxBlocks * 8 * mb);
   L.scnt = take(sizeof(uint32_t) * (size_t)L.nsplit);
@@ -358,6 +363,7 @@ static KParams make_kparams(const mk_plan_s& plan, const mk_weight_ptrs* w, cons
   k.ssq_stride = L.ssq_stride;
   k.part = (float*)(A + L.part);
   k.lmpart = (float2*)(A + L.lmpart);
+  k.lmrows = (int2*)(A + L.lmrows);
   k.spart = (float*)(A + L.spart);
   k.scnt = (uint32_t*)(A + L.scnt);
   k.n_split = L.nsplit;
@@ -461,7 +467,8 @@ static int check_step_args(mk_handle_t h, const void* tok, const void* pos, cons
 }
 
 static int launch_step(mk_handle_t h, const int32_t* tok, const int32_t* pos, const int32_t* lens, int32_t batch,
-                       const mk_kv_cache* kv, float* logits, int32_t* argmax, cudaStream_t s) {
+                       const mk_kv_cache* kv, float* logits, int32_t* argmax, cudaStream_t s, int step_add = 0,
+                       const mk_sampling* smp = nullptr, const float* uniforms = nullptr) {
   if (kv->k_pool != h->kv_k || kv->v_pool != h->kv_v || kv->num_pages != h->kv_pages) {
     const std::string e = encode_kv_maps(h->plan.cfg, kv, h->kp);
     if (!e.empty()) {
@@ -473,10 +480,15 @@ static int launch_step(mk_handle_t h, const int32_t* tok, const int32_t* pos, co
     h->kv_pages = kv->num_pages;
   }
   KParams p = h->kp;
-  p.tok = tok; p.pos = pos; p.lens = lens; p.b = batch;
+  p.tok = tok; p.pos = pos; p.lens = lens; p.b = batch; p.step_add = step_add;
   p.kpool = (__nv_bfloat16*)kv->k_pool; p.vpool = (__nv_bfloat16*)kv->v_pool;
   p.ptable = kv->page_table; p.num_pages = kv->num_pages; p.mpps = kv->max_pages_per_seq;
   p.logits = logits; p.argmax = argmax;
+  if (smp && smp->top_k > 1) {
+    p.top_k = smp->top_k;
+    p.temperature = smp->temperature;
+    p.uniforms = uniforms;
+  }
   p.epoch = ++h->epoch;
   cudaError_t e = mk::launch_decode(p, s);
   if (e != cudaSuccess) {
@@ -493,6 +505,33 @@ MK_API int mk_decode_step(mk_handle_t h, const int32_t* token_ids, const int32_t
   int rc = check_step_args(h, token_ids, positions, seq_lens, batch, kv, logits_out);
   if (rc) return rc;
   return launch_step(h, token_ids, positions, seq_lens, batch, kv, logits_out, argmax_out, (cudaStream_t)stream);
+}
+
+MK_API int mk_decode_steps(mk_handle_t h, int32_t n_steps, const int32_t* token_ids, const int32_t* positions,
+                           int32_t batch, const mk_kv_cache* kv, const mk_sampling* sampling, int32_t* tokens_out,
+                           float* logits_out, mk_stream_t stream) {
+  if (!h) return fail(nullptr, MK_ERR_INVALID_ARG, "mk_decode_steps: null handle");
+  if (n_steps < 1) return fail(h, MK_ERR_INVALID_ARG, "mk_decode_steps: n_steps must be >= 1");
+  if (!tokens_out) return fail(h, MK_ERR_INVALID_ARG, "mk_decode_steps: null tokens_out");
+  if (sampling && sampling->top_k > 1) {
+    if (sampling->top_k > MK_MAX_TOP_K)
+      return fail(h, MK_ERR_INVALID_ARG, "mk_decode_steps: top_k above MK_MAX_TOP_K");
+    if (!(sampling->temperature > 0.f) || !std::isfinite(sampling->temperature))
+      return fail(h, MK_ERR_INVALID_ARG, "mk_decode_steps: temperature must be finite and > 0");
+    if (!sampling->uniforms) return fail(h, MK_ERR_INVALID_ARG, "mk_decode_steps: null uniforms");
+  }
+  float* logits = logits_out ? logits_out : h->d_logits;
+  int rc = check_step_args(h, token_ids, positions, positions, batch, kv, logits);
+  if (rc) return rc;
+  const cudaStream_t s = (cudaStream_t)stream;
+  for (int32_t k = 0; k < n_steps; ++k) {
+    // step k: the token is step k-1's greedy token, every position k further on
+    const int32_t* tok = k == 0 ? token_ids : tokens_out + (size_t)(k - 1) * batch;
+    rc = launch_step(h, tok, positions, nullptr, batch, kv, logits, tokens_out + (size_t)k * batch, s, k, sampling,
+                     sampling ? sampling->uniforms + (size_t)k * batch : nullptr);
+    if (rc) return rc;
+  }
+  return MK_OK;
 }
 
 MK_API int mk_decode_step_host(mk_handle_t h, const int32_t* token_ids, const int32_t* positions,

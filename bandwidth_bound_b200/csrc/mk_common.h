@@ -34,6 +34,7 @@ constexpr int kFmaRows = 4;                             // batches up to this si
 constexpr int kMaxBlocks = 8;                           // 8-row blocks per GEMV task (64 rows)
 constexpr int kPage = 16;                               // tokens per KV page
 constexpr int kMaxChunksPerSeq = 32;                    // split-K chunks per (sequence, kv head)
+constexpr int kMaxTopK = 256;                           // largest k of top-k sampling
 constexpr int kRedBytes = kConsumerWarps * kMaxBlocks * 8 * 8 * 4;   // 16 KB: one 8-row batch tile at a time
 constexpr int kNoCounter = 0xFFFF;
 constexpr int kBoxCols = 64;                            // weight columns per TMA box (128 bytes, 128B swizzle)

@@ -47,6 +47,9 @@ struct Smem {
   int attn_n[kMaxBatch];         // pair-aligned: ranges per (sequence i, kv head) pair
   int attn_Ri[kMaxBatch];        // pair-aligned: tokens per range of sequence i (a multiple of 16)
   int attn_u0[kMaxBatch + 1];    // pair-aligned: first range of sequence i
+  int in_tok[kMaxBatch];         // this step's token, position and keys attended per sequence,
+  int in_pos[kMaxBatch];         // read once from the step's inputs (positions offset by the
+  int in_len[kMaxBatch];         // step's index in a multi-step run)
   unsigned long long wait_cyc;  // tracing: SM cycles warp 0 spent waiting for pool slots in the current task
   unsigned long long tm[3];     // tracing: compute, reduce, epilogue SM cycles of the current task (warp 0)
 };
@@ -300,7 +303,7 @@ __device__ bool attn_piece(const KParams& p, const Smem& sm, int u, int j, AttnP
     while (u >= sm.attn_u0[i + 1]) ++i;
     const int ni = sm.attn_n[i], Ri = sm.attn_Ri[i];
     const int r = u - sm.attn_u0[i];
-    const int n = p.lens[i];
+    const int n = sm.in_len[i];
     a.i = i;
     a.h = r / ni;
     a.c = r - a.h * ni;
@@ -314,7 +317,7 @@ __device__ bool attn_piece(const KParams& p, const Smem& sm, int u, int j, AttnP
   const long long lo = (long long)u * R, hi = lo + R;
   long long off = 0;
   for (int i = 0; i < p.b; ++i) {
-    const int n = p.lens[i];
+    const int n = sm.in_len[i];
     const int Lp = (n + kPage - 1) / kPage * kPage;
     const long long blk = (long long)p.nkv * Lp;
     if (off + blk > lo) {
@@ -353,7 +356,7 @@ __device__ void attn_setup(const KParams& p, Smem& sm) {
     for (;;) {
       int best = -1, bestlen = 0;
       for (int i = 0; i < p.b; ++i) {
-        const int len = (p.lens[i] + sm.attn_n[i] - 1) / sm.attn_n[i];
+        const int len = (sm.in_len[i] + sm.attn_n[i] - 1) / sm.attn_n[i];
         if (sm.attn_n[i] < kMaxChunksPerSeq && len > bestlen && len > T) { best = i; bestlen = len; }
       }
       if (best < 0 || used + p.nkv > p.n_slots) break;
@@ -362,7 +365,7 @@ __device__ void attn_setup(const KParams& p, Smem& sm) {
     }
     sm.attn_u0[0] = 0;
     for (int i = 0; i < p.b; ++i) {
-      const int len = (p.lens[i] + sm.attn_n[i] - 1) / sm.attn_n[i];
+      const int len = (sm.in_len[i] + sm.attn_n[i] - 1) / sm.attn_n[i];
       sm.attn_Ri[i] = (len + kPage - 1) / kPage * kPage;
       sm.attn_u0[i + 1] = sm.attn_u0[i] + p.nkv * sm.attn_n[i];
     }
@@ -372,7 +375,7 @@ __device__ void attn_setup(const KParams& p, Smem& sm) {
   long long tot = 0;
   int mx = kPage;
   for (int i = 0; i < p.b; ++i) {
-    const int Lp = (p.lens[i] + kPage - 1) / kPage * kPage;
+    const int Lp = (sm.in_len[i] + kPage - 1) / kPage * kPage;
     tot += (long long)p.nkv * Lp;
     mx = max(mx, Lp);
   }
@@ -885,7 +888,7 @@ __device__ void gemv_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_
         const float r = sm.inv_rms[bi];
         const float x1 = sm.ep[row][bi] * r;
         const float x2 = sm.ep[8 * n + row][bi] * r;
-        const int pos = p.pos[bi];
+        const int pos = sm.in_pos[bi];
         if (hh < p.nq + p.nkv) {
           const float2 cs = p.rope[(size_t)pos * half + j];
           const float o1 = x1 * cs.x - x2 * cs.y;
@@ -982,6 +985,7 @@ __device__ void gemv_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_
         }
         if (lane == 0) p.lmpart[(size_t)t.task_idx * p.max_b + bi] = make_float2(best, __int_as_float(bidx));
       }
+      if (threadIdx.x == 0) p.lmrows[t.task_idx] = make_int2(8 * (int)t.u0, min(8 * n, p.V - 8 * (int)t.u0));
     }
   }
   if (p.trace && threadIdx.x == 0) sm.tm[2] += (unsigned long long)(clock64() - te0);
@@ -993,7 +997,7 @@ __device__ void embed_task(const KParams& p, Smem& sm, const TaskDesc& t, bool a
   const int c0 = 8 * t.u0, nc = 8 * t.nunits;
   const bf16* gain = next_gain(p, OP_EMBED, 0);
   for (int bi = warp; bi < p.b; bi += kConsumerWarps) {
-    const bf16* e = p.embed + (size_t)p.tok[bi] * p.d;
+    const bf16* e = p.embed + (size_t)sm.in_tok[bi] * p.d;
     float s = 0.f;
     for (int c = lane; c < nc; c += 32) {
       const float v = __bfloat162float(e[c0 + c]);
@@ -1267,6 +1271,231 @@ __device__ __noinline__ void attn_task(const KParams& p, Smem& sm, const TaskDes
 }
 
 // ---------------------------------------------------------------------------------------
+// top-k sampling of the next token, run by the CTA that released the step's last LM-head task
+
+// Order-preserving keys: a larger logit gives a larger key32; key64 puts the lower vocabulary
+// index first among equal logits, so that all keys of one row differ and "the k largest"
+// is one set.
+__device__ __forceinline__ uint32_t logit_key32(float v) {
+  const uint32_t u = __float_as_uint(v);
+  return u ^ ((uint32_t)((int32_t)u >> 31) | 0x80000000u);
+}
+__device__ __forceinline__ uint64_t logit_key64(float v, int idx) {
+  return ((uint64_t)logit_key32(v) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)idx);
+}
+__device__ __forceinline__ float key64_logit(uint64_t key) {
+  const uint32_t k = (uint32_t)(key >> 32);
+  return __uint_as_float((k & 0x80000000u) ? (k ^ 0x80000000u) : ~k);
+}
+__device__ __forceinline__ int key64_index(uint64_t key) { return (int)(0xFFFFFFFFu - (uint32_t)key); }
+
+// The k-th largest of n keys get(0..n-1) (1 <= k <= n), found by one warp: a radix select,
+// most significant 8 bits first, that stops as soon as every key left in the chosen bin is
+// among the k largest (the k-th is then their minimum).  hist: 256 words of shared memory.
+template <class Get>
+__device__ uint64_t warp_kth_largest(Get get, int n, int k, uint32_t* hist) {
+  const int lane = threadIdx.x & 31;
+  uint64_t prefix = 0, mask = 0;
+  uint32_t rem = (uint32_t)k;
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    for (int i = lane; i < 256; i += 32) hist[i] = 0u;
+    __syncwarp();
+    for (int j = lane; j < n; j += 32) {
+      const uint64_t key = get(j);
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    }
+    __syncwarp();
+    // lane l holds bins 255-8l .. 248-8l: lanes in order walk the bins from the top
+    uint32_t c[8], tot = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) { c[q] = hist[255 - 8 * lane - q]; tot += c[q]; }
+    uint32_t incl = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const uint32_t excl = incl - tot;
+    const bool mine = excl < rem && rem <= incl;
+    const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+    uint32_t digit = 0, above = 0, inbin = 0;
+    if (mine) {
+      uint32_t acc = excl;
+      for (int q = 0; q < 8; ++q) {
+        if (acc + c[q] >= rem) { digit = 255u - 8u * lane - q; above = acc; inbin = c[q]; break; }
+        acc += c[q];
+      }
+    }
+    digit = __shfl_sync(0xffffffffu, digit, src);
+    above = __shfl_sync(0xffffffffu, above, src);
+    inbin = __shfl_sync(0xffffffffu, inbin, src);
+    rem -= above;
+    prefix |= (uint64_t)digit << shift;
+    mask |= (uint64_t)255u << shift;
+    __syncwarp();
+    if (inbin == rem) {
+      uint64_t mn = ~0ull;
+      for (int j = lane; j < n; j += 32) {
+        const uint64_t key = get(j);
+        if ((key & mask) == prefix && key < mn) mn = key;
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) {
+        const uint64_t v = __shfl_xor_sync(0xffffffffu, mn, o);
+        mn = v < mn ? v : mn;
+      }
+      return mn;
+    }
+  }
+  return prefix;
+}
+
+// Per batch row (one warp each): the next token drawn from the top_k logits at temperature T.
+//  1. Every LM-head task left its row maximum (lmpart) and its vocabulary rows (lmrows).  The
+//     k largest logits all lie in the k tasks with the largest maxima: a logit of any other
+//     task is below those k maxima.  So the k-th largest task maximum tau0 bounds the top k
+//     from below.
+//  2. The logits >= tau0 of those tasks are the candidates (shared memory; if there are more
+//     than fit, the selection reads the tasks' rows from global memory instead).
+//  3. The k-th largest candidate tau: the top k are the candidates >= tau, ranked by key.
+//  4. Weights w_r = exp((v_r - v_0) / T) in rank order, summed in that order by one lane; the
+//     token is the first rank whose running sum exceeds u * total (the last rank if rounding
+//     leaves none).
+__device__ __noinline__ void sample_top_k(const KParams& p, Smem& sm) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // per warp: histogram, selected tasks, the top k and their weights, then keys/candidates
+  constexpr int kRegion = kNumSlots * kSlotBytes / kConsumerWarps;
+  uint8_t* base = &sm.pool[0][0] + (size_t)warp * kRegion;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(base);                       // 256 words
+  int* sel = reinterpret_cast<int*>(base + 1024);                           // kMaxTopK task ids
+  uint64_t* top = reinterpret_cast<uint64_t*>(base + 1024 + 4 * kMaxTopK);  // kMaxTopK keys, by rank
+  float* w = reinterpret_cast<float*>(base + 1024 + 12 * kMaxTopK);          // kMaxTopK weights
+  uint64_t* buf = reinterpret_cast<uint64_t*>(base + 1024 + 16 * kMaxTopK);
+  const int cap = (kRegion - 1024 - 16 * kMaxTopK) / 8;
+  const int n = p.n_lm_tasks;
+  const int k = min(p.top_k, min(kMaxTopK, p.V));
+  for (int bi = warp; bi < p.b; bi += kConsumerWarps) {
+    const float2* mx = p.lmpart + bi;  // task j: mx[j * max_b]
+    auto task_key = [&](int j) {
+      const float2 c = __ldcg(mx + (size_t)j * p.max_b);
+      return logit_key64(c.x, __float_as_int(c.y));
+    };
+    // 1. tau0 over the task maxima (from shared memory when they fit)
+    uint64_t tau0;
+    const int kt = min(k, n);
+    if (n <= cap) {
+      for (int j = lane; j < n; j += 32) buf[j] = task_key(j);
+      __syncwarp();
+      tau0 = warp_kth_largest([&](int j) { return buf[j]; }, n, kt, hist);
+    } else {
+      tau0 = warp_kth_largest(task_key, n, kt, hist);
+    }
+    // the selected tasks (ties among maxima only come from tasks without a maximum of their
+    // own, the pieces of a split task that did not finish it: those have no rows and are
+    // skipped); at most kMaxTopK, since keys of tasks with rows all differ
+    int nsel = 0;
+    for (int j0 = 0; j0 < n; j0 += 32) {
+      const int j = j0 + lane;
+      bool s = false;
+      if (j < n) {
+        const uint64_t key = n <= cap ? buf[j] : task_key(j);
+        s = key >= tau0 && isfinite(__ldcg(mx + (size_t)j * p.max_b).x);
+      }
+      const unsigned bal = __ballot_sync(0xffffffffu, s);
+      const int at = nsel + __popc(bal & ((1u << lane) - 1u));
+      if (s && at < kMaxTopK) sel[at] = j;
+      nsel += __popc(bal);
+    }
+    nsel = min(nsel, kMaxTopK);
+    __syncwarp();
+    if (nsel == 0) {  // no finite logit in the row: no token (the next step rejects it as out of range)
+      if (lane == 0) p.argmax[bi] = 0x7fffffff;
+      continue;
+    }
+    // 2. candidates: the selected tasks' logits with key >= tau0
+    int nc = 0;
+    for (int s = 0; s < nsel; ++s) {
+      const int2 rr = __ldcg(p.lmrows + sel[s]);
+      for (int r0 = 0; r0 < rr.y; r0 += 32) {
+        const int r = r0 + lane;
+        uint64_t key = 0;
+        bool c = false;
+        if (r < rr.y) {
+          const int idx = rr.x + r;
+          key = logit_key64(__ldcg(p.logits + (size_t)bi * p.V + idx), idx);
+          c = key >= tau0;
+        }
+        const unsigned bal = __ballot_sync(0xffffffffu, c);
+        const int at = nc + __popc(bal & ((1u << lane) - 1u));
+        if (c && at < cap) buf[at] = key;
+        nc += __popc(bal);
+      }
+    }
+    __syncwarp();
+    // 3. tau = the k-th largest candidate (nc >= k: the k tasks' maxima are candidates)
+    auto row_key = [&](int j) {  // the selected tasks' rows, 64 per task (padding: key 0)
+      const int s = j >> 6, r = j & 63;
+      const int2 rr = __ldcg(p.lmrows + sel[s]);
+      if (r >= rr.y) return (uint64_t)0;
+      return logit_key64(__ldcg(p.logits + (size_t)bi * p.V + rr.x + r), rr.x + r);
+    };
+    const bool in_smem = nc <= cap;
+    const int ktop = min(k, nc);
+    const uint64_t tau = in_smem ? warp_kth_largest([&](int j) { return buf[j]; }, nc, ktop, hist)
+                                 : warp_kth_largest(row_key, 64 * nsel, ktop, hist);
+    // the top k, unordered, then placed by rank (the number of larger keys; all keys differ)
+    int nt = 0;
+    const int nsrc = in_smem ? nc : 64 * nsel;
+    for (int j0 = 0; j0 < nsrc; j0 += 32) {
+      const int j = j0 + lane;
+      const uint64_t key = j < nsrc ? (in_smem ? buf[j] : row_key(j)) : 0ull;
+      const bool c = j < nsrc && key >= tau;
+      const unsigned bal = __ballot_sync(0xffffffffu, c);
+      const int at = nt + __popc(bal & ((1u << lane) - 1u));
+      if (c && at < kMaxTopK) top[at] = key;
+      nt += __popc(bal);
+    }
+    nt = min(nt, ktop);
+    __syncwarp();
+    uint64_t mine[kMaxTopK / 32];
+    int rk[kMaxTopK / 32];
+#pragma unroll
+    for (int q = 0; q < kMaxTopK / 32; ++q) {
+      const int e = 32 * q + lane;
+      mine[q] = e < nt ? top[e] : 0ull;
+      rk[q] = -1;
+      if (e < nt) {
+        int r = 0;
+        for (int f = 0; f < nt; ++f) r += top[f] > mine[q] ? 1 : 0;
+        rk[q] = r;
+      }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int q = 0; q < kMaxTopK / 32; ++q)
+      if (rk[q] >= 0) top[rk[q]] = mine[q];
+    __syncwarp();
+    // 4. weights in rank order and the draw
+    const float v0 = key64_logit(top[0]);
+    for (int r = lane; r < nt; r += 32) w[r] = expf((key64_logit(top[r]) - v0) / p.temperature);
+    __syncwarp();
+    if (lane == 0) {
+      float total = 0.f;
+      for (int r = 0; r < nt; ++r) total += w[r];
+      const float thr = p.uniforms[bi] * total;
+      float cum = 0.f;
+      int pick = nt - 1;
+      for (int r = 0; r < nt; ++r) {
+        cum += w[r];
+        if (cum > thr) { pick = r; break; }
+      }
+      p.argmax[bi] = key64_index(top[pick]);
+    }
+    __syncwarp();
+  }
+}
+
+// ---------------------------------------------------------------------------------------
 // consumer warps: walk the stream
 
 __device__ void consumer(const KParams& p, Smem& sm, const TaskDesc* ts, int nt) {
@@ -1326,7 +1555,9 @@ __device__ void consumer(const KParams& p, Smem& sm, const TaskDesc* ts, int nt)
   if (threadIdx.x == 0 && nt > 0 && p.argmax)
     sm.flag = mbar_wait(p, &sm.sigempty[(nt - 1) % kSigRing], ((nt - 1) / kSigRing) & 1) ? sm.lm_last : 0;
   cbar();
-  if (nt > 0 && p.argmax && sm.flag) {
+  if (nt > 0 && p.argmax && sm.flag && p.top_k > 1) {
+    sample_top_k(p, sm);
+  } else if (nt > 0 && p.argmax && sm.flag) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int bi = warp; bi < p.b; bi += kConsumerWarps) {
       float best = -INFINITY;
@@ -1410,7 +1641,11 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
     // scalar input checks (page ids are checked where they are used)
     int bad = 0;
     for (int i = 0; i < p.b; ++i) {
-      const int tk = p.tok[i], ps = p.pos[i], ln = p.lens[i];
+      const int tk = p.tok[i], ps = p.pos[i] + p.step_add;
+      const int ln = p.lens ? p.lens[i] + p.step_add : ps + 1;
+      sm.in_tok[i] = tk;
+      sm.in_pos[i] = ps;
+      sm.in_len[i] = ln;
       if (tk < 0 || tk >= p.V || ps < 0 || ps >= p.max_ctx || ln != ps + 1 || ps / kPage >= p.mpps) bad = 1;
       else {
         const int pg = p.ptable[i * p.mpps + ps / kPage];
@@ -1418,6 +1653,8 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
       }
     }
     if (bad) raise_error(p, -6 /* MK_ERR_BOUNDS */);
+    // an earlier step of a multi-step run failed: its error stands and this step does nothing
+    if (ld_relaxed(&p.ctl[0]) != 0) bad = 1;
     sm.bad = bad;
     if (!bad) attn_setup(p, sm);
   }

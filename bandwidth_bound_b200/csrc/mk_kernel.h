@@ -42,6 +42,7 @@ struct KParams {
   int ld_x, ld_a, ld_h;
   int ssq_stride;            // floats per ssq instance
   float2* lmpart;            // [n_lm_tasks][max_b] (value, index bits)
+  int2* lmrows;              // [n_lm_tasks] (first vocabulary row, rows) of the task whose maxima lmpart holds
   float* spart;              // K-piece partial sums [split id][kMaxPieces][64 rows][max_b]
   uint32_t* scnt;            // K-piece arrival counters [split id]
   int n_split;               // split ids (entries of scnt)
@@ -49,13 +50,17 @@ struct KParams {
   int* host_status;          // mapped host word
   const float2* rope;        // [max_ctx][hd/2] (cos, sin)
   // this step
-  const int *tok, *pos, *lens;
+  const int *tok, *pos, *lens;  // lens may be null: pos + 1
   int b;
+  int step_add;                 // added to every position (and length): step index of a multi-step run
   __nv_bfloat16 *kpool, *vpool;
   const int* ptable;
   int num_pages, mpps;
   float* logits;
-  int* argmax;
+  int* argmax;                 // the step's next token per sequence: greedy, or drawn from the top_k
+  int top_k;                   // <= 1: greedy; 2..kMaxTopK: sample among the top_k logits
+  float temperature;           // > 0 (sampling only)
+  const float* uniforms;       // [b] in [0, 1): this step's draw per sequence (sampling only)
   float* dbg;
   uint32_t epoch;
   unsigned long long timeout_ns;

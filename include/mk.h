@@ -153,6 +153,49 @@ MK_API int mk_decode_step(mk_handle_t h, const int32_t *token_ids, const int32_t
                           const int32_t *seq_lens, int32_t batch, const mk_kv_cache *kv,
                           float *logits_out, int32_t *argmax_out, mk_stream_t stream);
 
+/* Top-k sampling of the next token (the engine's sampler, ForgeMegakernel §4.3), done
+ * inside the step's launch by the CTA that releases the LM head's last task, one warp per
+ * sequence.  For sequence i of step s, with u = uniforms[s][i]:
+ *   the k = top_k largest logits (equal logits: the lower vocabulary index first), ranked
+ *   from the largest, v_0 >= v_1 >= ... >= v_{k-1};
+ *   weights w_r = exp((v_r - v_0) / temperature), in fp32;
+ *   the token is the one of the first rank r whose running sum w_0 + ... + w_r, added in
+ *   rank order in fp32, exceeds u * (w_0 + ... + w_{k-1}) (rank k-1 if rounding leaves none).
+ * The caller draws the uniforms (any generator), so a run is reproducible from its inputs. */
+#define MK_MAX_TOP_K 256
+typedef struct mk_sampling {
+  int32_t top_k;          /* <= 1: greedy (argmax, lowest index of the max); 2 .. MK_MAX_TOP_K */
+  float temperature;      /* finite, > 0 */
+  const float *uniforms;  /* device fp32 [n_steps][batch], each in [0, 1) */
+} mk_sampling;
+
+/* n_steps decode steps in one call, with no host round trip between them (the engine's
+ * generation loop behind the launch: ForgeMegakernel §4.3).  Step k (0-based) takes as its
+ * token the one step k-1 chose (step 0: token_ids), sits at position positions[i] + k,
+ * appends its K/V entry there and attends to the positions[i] + k + 1 keys up to and
+ * including it.
+ *   n_steps    >= 1
+ *   token_ids  device int32 [batch]: the first step's tokens
+ *   positions  device int32 [batch]: the first step's positions
+ *   batch, kv  as for mk_decode_step; the page table must already map every position
+ *              the run reaches, positions[i] + n_steps - 1
+ *   sampling   NULL or top_k <= 1: greedy; else top-k sampling as above (host struct; the
+ *              uniforms it points to are device memory)
+ *   tokens_out device int32 [n_steps][batch]: row k = the token step k chose, which is
+ *              also step k+1's input (the rows are read back by the following steps)
+ *   logits_out device fp32 [batch][vocab] or NULL: the last step's logits (every step
+ *              writes there; with NULL they go to the handle's own buffer)
+ * n_steps stream-ordered launches of the step kernel on `stream`; the call does not wait.
+ * Host-side argument errors return before anything is launched.  A step that fails on
+ * the device (for example a position past max_ctx, or one without a page: MK_ERR_BOUNDS)
+ * sets the sticky status, and every later step of the run then returns at once without
+ * touching the cache or tokens_out; read the status with mk_get_status after
+ * synchronising. */
+MK_API int mk_decode_steps(mk_handle_t h, int32_t n_steps, const int32_t *token_ids,
+                           const int32_t *positions, int32_t batch, const mk_kv_cache *kv,
+                           const mk_sampling *sampling, int32_t *tokens_out, float *logits_out,
+                           mk_stream_t stream);
+
 /* The same step from HOST buffers: copies token_ids/positions/seq_lens (host
  * int32 [batch]) to the handle's device staging area, runs the step, copies the
  * logits (host fp32 [batch][vocab], may be NULL) and argmax (host int32 [batch],

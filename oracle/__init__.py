@@ -24,3 +24,4 @@ from .decode import (  # noqa: F401
     model_bytes,
     argmax_lowest,
 )
+from .sampling import boundary_margin, sample_top_k, top_k_ranked  # noqa: F401,E402

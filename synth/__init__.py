@@ -213,10 +213,11 @@ def pages_needed(n_tokens: int, page: int) -> int:
 
 def make_kv_cache(m: ModelConfig, ctx_lens: list[int], device="cpu", seed: int = 1,
                   max_ctx: Optional[int] = None, spare_pages: int = 3, batch_cap: Optional[int] = None,
-                  tag: str = "") -> KVCache:
+                  tag: str = "", room: int = 1) -> KVCache:
     """A paged cache holding ``ctx_lens[i]`` prior entries per sequence.
 
-    Each sequence owns ceil((S_i + 1) / page) pages (room for the new token), the
+    Each sequence owns ceil((S_i + room) / page) pages (room for the new token, or for the
+    ``room`` tokens of a multi-step run), the
     physical pages are a random permutation (so contiguity is never implied),
     ``spare_pages`` pages belong to nobody, and every slot that is not a prior
     entry holds the canary pattern.
@@ -227,7 +228,7 @@ def make_kv_cache(m: ModelConfig, ctx_lens: list[int], device="cpu", seed: int =
     if max_ctx is None:
         max_ctx = max(ctx_lens) + 1
     mpps = pages_needed(max_ctx, P)
-    need = [pages_needed(s + 1, P) for s in ctx_lens]
+    need = [pages_needed(s + room, P) for s in ctx_lens]
     num_pages = sum(need) + spare_pages
     g = _cpu_gen(2, f"{m.name}:pages:{tag}:{num_pages}")
     perm = torch.randperm(num_pages, generator=g)

@@ -31,13 +31,14 @@ class Case:
     extra: dict = field(default_factory=dict)
 
 
-def make_case(m, lens, gain_std=0.0, max_batch=0, max_ctx=0, tag="", weights=None, kv_spare=3) -> Case:
+def make_case(m, lens, gain_std=0.0, max_batch=0, max_ctx=0, tag="", weights=None, kv_spare=3,
+              kv_room=1) -> Case:
     b = len(lens)
     max_batch = max_batch or b
     max_ctx = max_ctx or (max(lens) + 1)
     wts = weights if weights is not None else synth.make_weights(m, device="cuda", gain_std=gain_std)
     kv = synth.make_kv_cache(m, list(lens), device="cuda", max_ctx=max_ctx, spare_pages=kv_spare,
-                             batch_cap=max_batch, tag=tag)
+                             batch_cap=max_batch, tag=tag, room=kv_room)
     toks = synth.token_ids(m, b, tag=tag or m.name)
     return Case(m, list(lens), toks, gain_std, max_batch, max_ctx, wts, kv)
 
@@ -142,8 +143,11 @@ def bf16_ulp_error(gpu: torch.Tensor, ref: torch.Tensor, floor: float = KV_FLOOR
 
 
 def check_step(c: Case, out: dict, ref: dict, k_before, v_before, batch=None, check_pool=True,
-               logit_tol=LOGIT_ABS) -> dict:
-    """Compare one GPU step with the oracle; returns the measured errors."""
+               logit_tol=LOGIT_ABS, e2e_kv_gate=True) -> dict:
+    """Compare one GPU step with the oracle; returns the measured errors.
+
+    e2e_kv_gate=False reports the end-to-end KV comparison without gating on it; it needs the
+    re-anchored comparison (``ref`` from run_oracle with ``anchor``), which then decides."""
     b = len(c.lens) if batch is None else batch
     m = c.m
     P = m.page_size
@@ -217,7 +221,10 @@ def check_step(c: Case, out: dict, ref: dict, k_before, v_before, batch=None, ch
     print("parity:", errs)
     if out["hidden"] is not None:
         assert hidden_fail is None, hidden_fail
-    assert worst_ulp <= KV_ULP, f"new KV entry off by {worst_ulp} bf16 ulp"
+    if e2e_kv_gate:
+        assert worst_ulp <= KV_ULP, f"new KV entry off by {worst_ulp} bf16 ulp"
+    else:
+        assert "anchored" in ref, "without the end-to-end KV gate the re-anchored check is required"
     if "anchored" in ref:
         assert anchored_worst <= KV_ULP, \
             f"{anchored_over} new KV entries off by up to {anchored_worst} bf16 ulp from the oracle's layer run " \
