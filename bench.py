@@ -32,6 +32,7 @@ import synth  # noqa: E402
 
 METRIC = "decode tokens/s"
 NOMINAL_HBM_GBS = 8000.0  # the pages' "~8 TB/s" B200 peak used for MBU
+MULTI_STEPS = 32  # steps per call of the on-device greedy loop line
 
 
 def parse():
@@ -43,6 +44,8 @@ def parse():
     ap.add_argument("--impl", default="mk", choices=["mk", "reference"])
     ap.add_argument("--no-secondary", action="store_true", help="skip the batch-1 line of the same model")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-all-configs", action="store_true", help="skip timing the other named shapes")
+    ap.add_argument("--no-multi-step", action="store_true", help="skip timing the on-device multi-step loop")
     ap.add_argument("--max-blocks", type=int, default=0, help="schedule option: 8-row blocks per GEMV task")
     ap.add_argument("--attn-slots", type=int, default=0, help="schedule option: attention slots per SM")
     ap.add_argument("--trace", default="", help="write a per-task timeline summary of one step to this file")
@@ -301,9 +304,10 @@ def run_mk(args, world, rank, local):
     m = w.model
     lens = w.context_lengths() if not args.layers else synth.WORKLOADS[args.workload].context_lengths()
     b = w.batch
-    max_ctx = max(lens) + 2
+    max_ctx = max(lens) + MULTI_STEPS + 1
     wts = synth.make_weights(m, device="cuda")
-    kv = synth.make_kv_cache(m, lens, device="cuda", max_ctx=max_ctx, batch_cap=max(b, 8))
+    # pages for the multi-step line's positions too (lens .. lens + MULTI_STEPS - 1)
+    kv = synth.make_kv_cache(m, lens, device="cuda", max_ctx=max_ctx, batch_cap=max(b, 8), room=MULTI_STEPS)
     toks = synth.token_ids(m, b, tag=w.name)
     plan = None
     if args.max_blocks or args.attn_slots:
@@ -424,12 +428,100 @@ def run_mk(args, world, rank, local):
         line["secondary"] = {"workload": f"{m.name}-b1 (batch-1 handle, context {lens[0]})", "ms_per_step": ms1,
                              "tokens_per_s": world / (ms1 / 1e3), "mbu": B1 / (ms1 / 1e3) / (NOMINAL_HBM_GBS * 1e9),
                              "achieved_gbs": B1 / (ms1 / 1e3) / 1e9}
+    if not args.no_multi_step:
+        line["multi_step"] = time_multi_step(mk, h, m, tok_d, pos_d, kv, lens, logits, stream, world, ms, flush)
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = {k: v for k, v in cpu_baseline(w, wts, kv, toks, lens).items()
                                 if k != "seconds_per_step"}
+    h.close()
+    if world == 1 and not args.no_all_configs and not args.layers and args.workload == "llama3-8b-b8":
+        # every named shape, each on a handle built for its own batch; the Llama-3-8B lines are
+        # the headline's and the batch-1 line's own measurements
+        rows = [{"workload": w.name, "batch": b, "ms_per_step": ms, "tokens_per_s": value,
+                 "mbu": line["mbu"], "frac_of_measured_copy": line["mbu_vs_measured_copy"], "l2": l2_note}]
+        if "secondary" in line:
+            sec = line["secondary"]
+            rows.append({"workload": "llama3-8b-b1", "batch": 1, "ms_per_step": sec["ms_per_step"],
+                         "tokens_per_s": sec["tokens_per_s"], "mbu": sec["mbu"],
+                         "frac_of_measured_copy": sec["achieved_gbs"] / peaks["hbm_gbs"], "l2": l2_note})
+        del wts, kv
+        torch.cuda.empty_cache()
+        for name in ("tiny-b1", "smollm2-135m-b1", "llama3.2-1b-b9", "llama2-13b-b4"):
+            rows.extend(time_config(mk, name, stream, min(args.steps, 200), args.warmup, peaks))
+        line["all_configs"] = rows
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def time_multi_step(mk, h, m, tok_d, pos_d, kv, lens, logits, stream, world, single_ms, flush) -> dict:
+    """The on-device greedy loop: MULTI_STEPS steps per call (each step's greedy token is the
+    next step's input, at the next position), the host waiting once per call.  Per call the
+    context of every sequence grows by MULTI_STEPS, so the bytes are summed step by step."""
+    n, runs = MULTI_STEPS, 5
+    b = len(lens)
+    toks_out = torch.empty((n, b), dtype=torch.int32, device="cuda")
+
+    def run():
+        h.steps(n, tok_d, pos_d, kv, toks_out, logits, stream=stream, check=False)
+
+    for _ in range(2):
+        run()
+    torch.cuda.synchronize()
+    barrier(world)
+    total, _ = time_steps(run, runs, stream, flush)
+    assert h.status() == mk.MK_OK, f"device status {h.status()}"
+    ms = max_over_ranks(world, total) / (runs * n)
+    B = sum(mk.step_bytes(m, [s + k for s in lens]) for k in range(n)) / n
+    return {"n_steps_per_call": n, "calls": runs, "ms_per_step": ms, "tokens_per_s": world * b / (ms / 1e3),
+            "mbu": B / (ms / 1e3) / (NOMINAL_HBM_GBS * 1e9), "single_step_ms": single_ms,
+            "launches_per_call": n, "host_waits_per_call": 1,
+            "l2": "no flush between the steps of one call" + ("; L2 flushed between calls" if flush else "")}
+
+
+def time_config(mk, name: str, stream, steps: int, warmup: int, peaks: dict) -> list:
+    """ms/step, tokens/s and MBU of one named workload on a handle built for its batch.  The
+    ragged Llama-3.2-1B batch is timed as its 8 first sequences and then with the 9th joined,
+    on the same handle (max_batch 9), as a server would run a late arrival."""
+    w = synth.WORKLOADS[name]
+    m = w.model
+    lens = w.context_lengths()
+    max_ctx = max(lens) + 2
+    wts = synth.make_weights(m, device="cuda")
+    kv = synth.make_kv_cache(m, lens, device="cuda", max_ctx=max_ctx, batch_cap=w.batch)
+    toks = synth.token_ids(m, w.batch, tag=w.name)
+    tok_d = torch.tensor(toks, dtype=torch.int32, device="cuda")
+    pos_d = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    len_d = pos_d + 1
+    logits = torch.empty((w.batch, m.vocab), dtype=torch.float32, device="cuda")
+    am = torch.empty((w.batch,), dtype=torch.int32, device="cuda")
+    h = mk.Megakernel(m, wts, w.batch, max_ctx)
+    l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+    scrub = torch.empty(2 * l2 // 4, dtype=torch.float32, device="cuda")
+    out = []
+    batches = [8, 9] if name == "llama3.2-1b-b9" else [w.batch]
+    for b in batches:
+        B = mk.step_bytes(m, lens[:b])
+        flush = (lambda: scrub.zero_()) if B < 4 * l2 else None
+        fn = lambda: h.step(tok_d[:b], pos_d[:b], len_d[:b], kv, logits[:b], am[:b], stream=stream,  # noqa: E731
+                            check=False)
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        total, per = time_steps(fn, steps, stream, flush)
+        assert h.status() == mk.MK_OK, f"{name}: device status {h.status()}"
+        ms = total / steps
+        out.append({"workload": name if len(batches) == 1 else f"{name} (first {b} of 9 on one handle)",
+                    "batch": b, "ms_per_step": ms, "tokens_per_s": b / (ms / 1e3),
+                    "mbu": B / (ms / 1e3) / (NOMINAL_HBM_GBS * 1e9),
+                    "frac_of_measured_copy": B / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                    "l2": ("L2 flushed between steps (2x L2 buffer written, untimed)" if flush is not None
+                           else f"inputs larger than L2 ({B / 1e9:.2f} GB read per step)")})
+    if len(out) == 2:
+        out[1]["tokens_per_s_vs_batch_8"] = out[1]["tokens_per_s"] / out[0]["tokens_per_s"]
     h.close()
+    del wts, kv, scrub
+    torch.cuda.empty_cache()
+    return out
 
 
 def main():
