@@ -19,9 +19,13 @@ Auto-Regressive Model Decode Megakernels" (paperlayer.ai digest of arXiv
 Readings where the pages are silent:
   * Llama conventions: RMSNorm with eps inside the square root and the gain
     applied afterwards; RoPE in the Hugging Face rotate-half pairing (j, j+hd/2)
-    with inv_freq_j = theta^(-2j/hd) and no frequency scaling; keys are cached
-    after RoPE; query head h reads KV head h // (n_heads / n_kv_heads); SiLU-gated
-    MLP; scores scaled by 1/sqrt(head_dim).
+    with inv_freq_j = theta^(-2j/hd), slowed by the Llama-3.x frequency scaling where
+    the model has one (rope_inv_freq); keys are cached after RoPE; query head h reads
+    KV head h // (n_heads / n_kv_heads); SiLU-gated MLP; scores scaled by
+    1/sqrt(head_dim).
+  * Qwen3 models (QK-norm): each query and key head is RMS-normalised over head_dim
+    with the layer's q_norm / k_norm gain (same epsilon) between the projection and
+    RoPE; the cached key is the normalised, rotated one.
   * The new token sits at position p_i = number of prior entries and attends to
     p_i + 1 keys; its own key and value enter attention as the bf16 values that
     are stored into the cache (round-to-nearest-even of the float64 result).
@@ -59,17 +63,37 @@ def rmsnorm(x: torch.Tensor, gain: torch.Tensor, eps: float) -> torch.Tensor:
     return x / torch.sqrt(ms + eps) * gain
 
 
-def rope_inv_freq(head_dim: int, theta: float) -> torch.Tensor:
-    """inv_freq_j = theta^(-2j/head_dim), j < head_dim/2 (§2.1 RoPE; HF convention)."""
+def rope_inv_freq(head_dim: int, theta: float, scaling=None) -> torch.Tensor:
+    """inv_freq_j = theta^(-2j/head_dim), j < head_dim/2 (§2.1 RoPE; HF convention).
+
+    scaling = (factor, low_freq_factor, high_freq_factor, original_max_position), the
+    Llama-3.x frequency scaling (the Llama 3 models the pages evaluate; the pages do not
+    spell it out, so this follows the published model configuration): with wavelength
+    w_j = 2 pi / inv_freq_j and N the original context, components with w_j < N / high
+    keep their frequency, those with w_j > N / low are slowed by the factor, and those in
+    between blend the two linearly in s = (N / w_j - low) / (high - low).
+    """
     j = torch.arange(head_dim // 2, dtype=F64)
-    return torch.pow(torch.tensor(theta, dtype=F64), -2.0 * j / head_dim)
+    inv = torch.pow(torch.tensor(theta, dtype=F64), -2.0 * j / head_dim)
+    if scaling is None or scaling[0] <= 1.0:
+        return inv
+    factor, low, high, n_orig = (float(s) for s in scaling)
+    out = inv.clone()
+    for i in range(len(inv)):
+        wavelen = 2.0 * math.pi / float(inv[i])
+        if wavelen > n_orig / low:
+            out[i] = inv[i] / factor
+        elif wavelen >= n_orig / high:
+            s = (n_orig / wavelen - low) / (high - low)
+            out[i] = (1.0 - s) * inv[i] / factor + s * inv[i]
+    return out
 
 
-def rope(v: torch.Tensor, pos: int, theta: float) -> torch.Tensor:
+def rope(v: torch.Tensor, pos: int, theta: float, scaling=None) -> torch.Tensor:
     """Rotate pairs (j, j + hd/2) of ``v[..., hd]`` by angle pos * inv_freq_j."""
     hd = v.shape[-1]
     half = hd // 2
-    ang = float(pos) * rope_inv_freq(hd, theta)
+    ang = float(pos) * rope_inv_freq(hd, theta, scaling)
     c, s = torch.cos(ang), torch.sin(ang)
     x1, x2 = v[..., :half], v[..., half:]
     return torch.cat([x1 * c - x2 * s, x2 * c + x1 * s], dim=-1)
@@ -165,6 +189,12 @@ def decode_layer(cfg, lw: dict, x: torch.Tensor, k_pool_l: torch.Tensor, v_pool_
     q = (xn @ lw["wq"].T).view(b, nq, hd)
     k = (xn @ lw["wk"].T).view(b, nkv, hd)
     v = (xn @ lw["wv"].T).view(b, nkv, hd)
+    if getattr(cfg, "qk_norm", False):
+        # Qwen3 QK-norm: each query and key head vector RMS-normalised over head_dim with
+        # its own gain, before RoPE (the Qwen3 models of §5.3 and Appendix A)
+        q = rmsnorm(q, lw["q_norm"], cfg.rms_eps)
+        k = rmsnorm(k, lw["k_norm"], cfg.rms_eps)
+    scaling = getattr(cfg, "rope_scaling", None)
     attn = torch.zeros((b, nq, hd), dtype=F64)
     k_new = torch.zeros((b, nkv, hd), dtype=F64)
     v_new = torch.zeros_like(k_new)
@@ -172,8 +202,8 @@ def decode_layer(cfg, lw: dict, x: torch.Tensor, k_pool_l: torch.Tensor, v_pool_
     v_exact = torch.zeros_like(k_new)
     for i in range(b):
         p = int(positions[i])
-        qi = rope(q[i], p, cfg.rope_theta)
-        ki = rope(k[i], p, cfg.rope_theta)
+        qi = rope(q[i], p, cfg.rope_theta, scaling)
+        ki = rope(k[i], p, cfg.rope_theta, scaling)
         vi = v[i]
         k_exact[i], v_exact[i] = ki, vi
         kr, vr = bf16_rne(ki), bf16_rne(vi)
@@ -274,6 +304,8 @@ def model_bytes(cfg, ctx_lens) -> int:
     d, hd, L = cfg.hidden, cfg.head_dim, cfg.n_layers
     qd, kvd, F, V = cfg.n_heads * hd, cfg.n_kv_heads * hd, cfg.ffn, cfg.vocab
     per_layer = 2 * d + qd * d + 2 * kvd * d + d * qd + 3 * F * d
+    if getattr(cfg, "qk_norm", False):
+        per_layer += 2 * hd  # the q_norm and k_norm gains
     elems = L * per_layer + d + V * d + len(ctx_lens) * d
     elems += sum(int(s) for s in ctx_lens) * L * 2 * kvd
     return 2 * elems

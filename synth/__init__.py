@@ -44,6 +44,10 @@ class ModelConfig:
     rope_theta: float
     rms_eps: float = 1e-5
     page_size: int = 16
+    # Llama-3.x RoPE frequency scaling: (factor, low_freq_factor, high_freq_factor,
+    # original_max_position), or None
+    rope_scaling: Optional[tuple] = None
+    qk_norm: bool = False  # Qwen3-style RMSNorm of each query and key head before RoPE
 
     @property
     def group(self) -> int:
@@ -78,11 +82,18 @@ class Workload:
 
 TINY = ModelConfig("tiny", 2, 256, 4, 2, 64, 688, 2048, False, 10000.0)
 SMOLLM2_135M = ModelConfig("smollm2-135m", 30, 576, 9, 3, 64, 1536, 49152, True, 100000.0)
-LLAMA32_1B = ModelConfig("llama3.2-1b", 16, 2048, 32, 8, 64, 8192, 128256, True, 500000.0)
+LLAMA32_1B = ModelConfig("llama3.2-1b", 16, 2048, 32, 8, 64, 8192, 128256, True, 500000.0,
+                         rope_scaling=(32.0, 1.0, 4.0, 8192))
 LLAMA3_8B = ModelConfig("llama3-8b", 32, 4096, 32, 8, 128, 14336, 128256, False, 500000.0)
 LLAMA2_13B = ModelConfig("llama2-13b", 40, 5120, 40, 40, 128, 13824, 32000, False, 10000.0)
 
-MODELS = {m.name: m for m in (TINY, SMOLLM2_135M, LLAMA32_1B, LLAMA3_8B, LLAMA2_13B)}
+# the Qwen3 shapes the pages evaluate (QK-norm, head_dim 128 with q_dim != hidden at 0.6B)
+QWEN3_0_6B = ModelConfig("qwen3-0.6b", 28, 1024, 16, 8, 128, 3072, 151936, True, 1000000.0, rms_eps=1e-6,
+                         qk_norm=True)
+QWEN3_8B = ModelConfig("qwen3-8b", 36, 4096, 32, 8, 128, 12288, 151936, False, 1000000.0, rms_eps=1e-6,
+                       qk_norm=True)
+
+MODELS = {m.name: m for m in (TINY, SMOLLM2_135M, LLAMA32_1B, LLAMA3_8B, LLAMA2_13B, QWEN3_0_6B, QWEN3_8B)}
 
 WORKLOADS = {
     w.name: w
@@ -93,6 +104,8 @@ WORKLOADS = {
         Workload("llama3-8b-b1", LLAMA3_8B, 1, ("fixed", 2048)),
         Workload("llama3-8b-b8", LLAMA3_8B, 8, ("fixed", 2048)),
         Workload("llama2-13b-b4", LLAMA2_13B, 4, ("uniform", 1024, 4096)),
+        Workload("qwen3-0.6b-b1", QWEN3_0_6B, 1, ("fixed", 128)),
+        Workload("qwen3-8b-b1", QWEN3_8B, 1, ("fixed", 2048)),
     )
 }
 
@@ -169,10 +182,10 @@ def make_weights(m: ModelConfig, device="cpu", seed: int = 0, std: float = 0.02,
     model is tied, "lm_head" is the same tensor object as "embed". ``layers``
     restricts generation to some layer indices (others are None).
     """
-    def gain(name):
+    def gain(name, n=m.hidden):
         if gain_std == 0.0:
-            return torch.ones((m.hidden,), dtype=torch.bfloat16, device=device)
-        return _normal_bf16((m.hidden,), gain_std, 1.0, seed, name, device)
+            return torch.ones((n,), dtype=torch.bfloat16, device=device)
+        return _normal_bf16((n,), gain_std, 1.0, seed, name, device)
 
     out = {"embed": _normal_bf16((m.vocab, m.hidden), std, 0.0, seed, "embed", device),
            "final_norm": gain("final_norm")}
@@ -191,6 +204,9 @@ def make_weights(m: ModelConfig, device="cpu", seed: int = 0, std: float = 0.02,
                 lw[name] = gain(f"L{li}.{name}")
             else:
                 lw[name] = _normal_bf16(shapes[name], std, 0.0, seed, f"L{li}.{name}", device)
+        if m.qk_norm:
+            for name in ("q_norm", "k_norm"):
+                lw[name] = gain(f"L{li}.{name}", m.head_dim)
         out["layers"].append(lw)
     return out
 

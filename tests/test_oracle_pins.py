@@ -380,9 +380,9 @@ def test_rounding_the_new_entry_is_a_small_perturbation(hf_tiny):
     assert 0 < err < 5e-2
 
 
-def _interleaved_rope(v, pos, theta):
+def _interleaved_rope(v, pos, theta, scaling=None):
     hd = v.shape[-1]
-    ang = float(pos) * od.rope_inv_freq(hd, theta)
+    ang = float(pos) * od.rope_inv_freq(hd, theta, scaling)
     c, s = torch.cos(ang), torch.sin(ang)
     x1, x2 = v[..., 0::2], v[..., 1::2]
     out = torch.empty_like(v)
@@ -393,8 +393,8 @@ def _interleaved_rope(v, pos, theta):
 
 MUTANTS = {
     "rope-interleaved": ("rope", lambda orig: _interleaved_rope),
-    "rope-pos-plus-one": ("rope", lambda orig: (lambda v, p, t: orig(v, p + 1, t))),
-    "rope-sign": ("rope", lambda orig: (lambda v, p, t: orig(v, -p, t))),
+    "rope-pos-plus-one": ("rope", lambda orig: (lambda v, p, t, s=None: orig(v, p + 1, t, s))),
+    "rope-sign": ("rope", lambda orig: (lambda v, p, t, s=None: orig(v, -p, t, s))),
     "gqa-modulo": ("kv_head_of", lambda orig: (lambda h, nq, nkv: h % nkv)),
     "no-score-scale": ("attention", lambda orig: (lambda q, K, V: orig(q * math.sqrt(q.shape[-1]), K, V))),
     "eps-outside-sqrt": ("rmsnorm", lambda orig: (lambda x, g, e: x / (torch.sqrt((x * x).mean(-1, keepdim=True)) + e) * g)),
