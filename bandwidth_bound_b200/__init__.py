@@ -43,7 +43,9 @@ class ModelCfg(ctypes.Structure):
                 ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("ffn", ctypes.c_int32),
                 ("vocab", ctypes.c_int32), ("tied", ctypes.c_int32), ("rope_theta", ctypes.c_float),
                 ("rms_eps", ctypes.c_float), ("max_batch", ctypes.c_int32), ("max_ctx", ctypes.c_int32),
-                ("page_size", ctypes.c_int32)]
+                ("page_size", ctypes.c_int32), ("rope_scale_factor", ctypes.c_float),
+                ("rope_low_freq_factor", ctypes.c_float), ("rope_high_freq_factor", ctypes.c_float),
+                ("rope_original_max_pos", ctypes.c_int32), ("qk_norm", ctypes.c_int32)]
 
 
 _PP = ctypes.POINTER(ctypes.c_void_p)
@@ -52,7 +54,8 @@ _PP = ctypes.POINTER(ctypes.c_void_p)
 class WeightPtrs(ctypes.Structure):
     _fields_ = [("embed", ctypes.c_void_p), ("final_norm", ctypes.c_void_p), ("lm_head", ctypes.c_void_p),
                 ("attn_norm", _PP), ("wq", _PP), ("wk", _PP), ("wv", _PP), ("wo", _PP),
-                ("mlp_norm", _PP), ("w_gate", _PP), ("w_up", _PP), ("w_down", _PP)]
+                ("mlp_norm", _PP), ("w_gate", _PP), ("w_up", _PP), ("w_down", _PP),
+                ("q_norm", _PP), ("k_norm", _PP)]
 
 
 class KvCache(ctypes.Structure):
@@ -116,9 +119,25 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
 
 
 def model_cfg(m, max_batch: int, max_ctx: int) -> ModelCfg:
-    """ModelCfg from any object with the synth.ModelConfig fields."""
+    """ModelCfg from any object with the synth.ModelConfig fields (rope_scaling: None or
+    (factor, low_freq_factor, high_freq_factor, original_max_pos); qk_norm: bool)."""
+    sc = getattr(m, "rope_scaling", None) or (1.0, 0.0, 0.0, 0)
     return ModelCfg(m.n_layers, m.hidden, m.n_heads, m.n_kv_heads, m.head_dim, m.ffn, m.vocab, int(m.tied),
-                    float(m.rope_theta), float(m.rms_eps), int(max_batch), int(max_ctx), int(m.page_size))
+                    float(m.rope_theta), float(m.rms_eps), int(max_batch), int(max_ctx), int(m.page_size),
+                    float(sc[0]), float(sc[1]), float(sc[2]), int(sc[3]), int(bool(getattr(m, "qk_norm", False))))
+
+
+_PER_LAYER = ("attn_norm", "wq", "wk", "wv", "wo", "mlp_norm", "w_gate", "w_up", "w_down")
+
+
+def weight_struct(m, weights: dict):
+    """(WeightPtrs, the host pointer arrays it points into - keep them alive) for a weights
+    dict as built by synth.make_weights."""
+    L = m.n_layers
+    names = _PER_LAYER + (("q_norm", "k_norm") if getattr(m, "qk_norm", False) else ())
+    arr = {n: (ctypes.c_void_p * L)(*[_ptr(weights["layers"][i][n]) for i in range(L)]) for n in names}
+    per = [ctypes.cast(arr[n], _PP) if n in arr else None for n in _PER_LAYER + ("q_norm", "k_norm")]
+    return WeightPtrs(_ptr(weights["embed"]), _ptr(weights["final_norm"]), _ptr(weights["lm_head"]), *per), arr
 
 
 def step_bytes(m, ctx_lens: Sequence[int]) -> int:
@@ -132,6 +151,8 @@ def step_bytes(m, ctx_lens: Sequence[int]) -> int:
     q_out = m.n_heads * m.head_dim
     kv_out = m.n_kv_heads * m.head_dim
     per_layer = d * q_out + 2 * d * kv_out + q_out * d + 3 * d * m.ffn + 2 * d
+    if getattr(m, "qk_norm", False):
+        per_layer += 2 * m.head_dim  # the q_norm and k_norm gains
     elements = L * per_layer + d + m.vocab * d + len(ctx_lens) * d
     elements += 2 * L * kv_out * sum(int(s) for s in ctx_lens)
     return 2 * elements
@@ -206,15 +227,7 @@ class Megakernel:
         self.m = m
         self.cfg = model_cfg(m, max_batch, max_ctx)
         self.weights = weights
-        L = m.n_layers
-        arr = {}
-        for name in ("attn_norm", "wq", "wk", "wv", "wo", "mlp_norm", "w_gate", "w_up", "w_down"):
-            a = (ctypes.c_void_p * L)(*[_ptr(weights["layers"][i][name]) for i in range(L)])
-            arr[name] = a
-        self._arrays = arr
-        w = WeightPtrs(_ptr(weights["embed"]), _ptr(weights["final_norm"]), _ptr(weights["lm_head"]),
-                       *[ctypes.cast(arr[n], _PP) for n in ("attn_norm", "wq", "wk", "wv", "wo", "mlp_norm",
-                                                             "w_gate", "w_up", "w_down")])
+        w, self._arrays = weight_struct(m, weights)
         self.handle = ctypes.c_void_p()
         if plan is None:
             rc = self.lib.mk_create(ctypes.byref(self.cfg), ctypes.byref(w), ctypes.byref(self.handle))
@@ -324,12 +337,7 @@ def decode_step_static(m, weights: dict, max_batch: int, max_ctx: int, token_ids
     if stream is None:
         stream = torch.cuda.current_stream()
     cfg = model_cfg(m, max_batch, max_ctx)
-    L = m.n_layers
-    arr = {name: (ctypes.c_void_p * L)(*[_ptr(weights["layers"][i][name]) for i in range(L)])
-           for name in ("attn_norm", "wq", "wk", "wv", "wo", "mlp_norm", "w_gate", "w_up", "w_down")}
-    w = WeightPtrs(_ptr(weights["embed"]), _ptr(weights["final_norm"]), _ptr(weights["lm_head"]),
-                   *[ctypes.cast(arr[n], _PP) for n in ("attn_norm", "wq", "wk", "wv", "wo", "mlp_norm",
-                                                         "w_gate", "w_up", "w_down")])
+    w, arr = weight_struct(m, weights)  # noqa: F841 (arr keeps the pointer arrays alive)
     kvs = Megakernel.kv_struct(kv)
     rc = lib.mk_decode_step_static(ctypes.byref(cfg), ctypes.byref(w), _ptr(token_ids), _ptr(positions),
                                    _ptr(seq_lens), int(token_ids.numel()), ctypes.byref(kvs), _ptr(logits),

@@ -213,7 +213,16 @@ static std::string collect_layers(const mk_model_cfg& c, const mk_weight_ptrs* w
       if (!p || !aligned16(p)) return "layer weight null or not 16-byte aligned";
     lw[l] = LayerW{(const __nv_bfloat16*)ps[0], (const __nv_bfloat16*)ps[1], (const __nv_bfloat16*)ps[2],
                    (const __nv_bfloat16*)ps[3], (const __nv_bfloat16*)ps[4], (const __nv_bfloat16*)ps[5],
-                   (const __nv_bfloat16*)ps[6], (const __nv_bfloat16*)ps[7], (const __nv_bfloat16*)ps[8]};
+                   (const __nv_bfloat16*)ps[6], (const __nv_bfloat16*)ps[7], (const __nv_bfloat16*)ps[8],
+                   nullptr, nullptr};
+    if (c.qk_norm) {
+      if (!w->q_norm || !w->k_norm) return "qk_norm needs the q_norm and k_norm arrays";
+      const void* g[2] = {w->q_norm[l], w->k_norm[l]};
+      for (const void* p : g)
+        if (!p || !aligned16(p)) return "qk-norm gain null or not 16-byte aligned";
+      lw[l].q_norm = (const __nv_bfloat16*)g[0];
+      lw[l].k_norm = (const __nv_bfloat16*)g[1];
+    }
   }
   return "";
 }
@@ -234,11 +243,36 @@ static int check_device(int dev, const char* who) {
   return MK_OK;
 }
 
+// RoPE inverse frequencies, in double: theta^(-2j/hd), then the Llama-3.x frequency scaling
+// when rope_scale_factor > 1 (the rule in mk.h's mk_model_cfg).
+static mk::RopeFreq rope_freq(const mk_model_cfg& c) {
+  mk::RopeFreq f{};
+  const int half = c.head_dim / 2;
+  const double pi = 3.14159265358979323846;
+  for (int j = 0; j < half; ++j) {
+    const double inv = std::pow((double)c.rope_theta, -2.0 * j / c.head_dim);
+    double out = inv;
+    if (c.rope_scale_factor > 1.f) {
+      const double N = c.rope_original_max_pos, factor = c.rope_scale_factor;
+      const double lo = c.rope_low_freq_factor, hi = c.rope_high_freq_factor;
+      const double wavelen = 2.0 * pi / inv;
+      if (wavelen > N / lo) {
+        out = inv / factor;
+      } else if (wavelen >= N / hi) {
+        const double s = (N / wavelen - lo) / (hi - lo);
+        out = (1.0 - s) * inv / factor + s * inv;
+      }
+    }
+    f.inv_freq[j] = out;
+  }
+  return f;
+}
+
 // Byte offsets of the scratch pieces (256-byte aligned).  The last three serve only the
 // handle's host-buffer entry point.
 struct Layout {
   size_t layers, tasks, offs, maps, x, q, ax, aa, ah, ssq, part, lmpart, lmrows, spart, scnt, ctr, cmb, ctl, status,
-      rope;
+      rope, qkss, knew;
   size_t stage, logits, argmax;
   size_t total;
   int ld_x, ld_a, ld_h, ntiles, ssq_stride, nsplit;
@@ -287,6 +321,11 @@ static Layout layout_scratch(const mk_plan_s& plan, bool host_step) {
   L.ctl = take(sizeof(uint32_t) * 2);
   L.status = take(sizeof(int));
   L.rope = take(sizeof(float2) * (size_t)c.max_ctx * (G.hd / 2));
+  L.qkss = L.knew = 0;
+  if (c.qk_norm) {
+    L.qkss = take(sizeof(float) * (size_t)mb * (G.nq + G.nkv) * (G.hd / 16));
+    L.knew = take(sizeof(float) * (size_t)mb * G.nkv * G.hd);
+  }
   L.stage = L.logits = L.argmax = 0;
   if (host_step) {
     L.stage = take(sizeof(int32_t) * 3 * mb);
@@ -325,7 +364,7 @@ static int upload_tables(const mk_plan_s& plan, const mk_weight_ptrs* w, const s
                          cudaMemcpyHostToDevice, stream);
   if (ce == cudaSuccess)
     ce = cudaMemcpyAsync(A + L.maps, maps.data(), sizeof(CUtensorMap) * maps.size(), cudaMemcpyHostToDevice, stream);
-  if (ce == cudaSuccess) ce = mk::launch_rope_table((float2*)(A + L.rope), c.max_ctx, G.hd, c.rope_theta, stream);
+  if (ce == cudaSuccess) ce = mk::launch_rope_table((float2*)(A + L.rope), c.max_ctx, G.hd, rope_freq(c), stream);
   if (ce == cudaSuccess) ce = cudaStreamSynchronize(stream);
   if (ce != cudaSuccess) return cuda_fail(nullptr, ce, (std::string(who) + ": upload").c_str());
   return MK_OK;
@@ -364,6 +403,9 @@ static KParams make_kparams(const mk_plan_s& plan, const mk_weight_ptrs* w, cons
   k.part = (float*)(A + L.part);
   k.lmpart = (float2*)(A + L.lmpart);
   k.lmrows = (int2*)(A + L.lmrows);
+  k.qk_norm = c.qk_norm ? 1 : 0;
+  k.qkss = c.qk_norm ? (float*)(A + L.qkss) : nullptr;
+  k.knew = c.qk_norm ? (float*)(A + L.knew) : nullptr;
   k.spart = (float*)(A + L.spart);
   k.scnt = (uint32_t*)(A + L.scnt);
   k.n_split = L.nsplit;
@@ -655,7 +697,8 @@ std::mutex g_static_mu[kStaticMaxDevices];
 
 void weight_key(const mk_model_cfg& c, const mk_weight_ptrs* w, std::vector<const void*>* out) {
   out->assign({w->embed, w->final_norm, w->lm_head});
-  const void* const* per[9] = {w->attn_norm, w->wq, w->wk, w->wv, w->wo, w->mlp_norm, w->w_gate, w->w_up, w->w_down};
+  const void* const* per[11] = {w->attn_norm, w->wq, w->wk, w->wv, w->wo, w->mlp_norm, w->w_gate, w->w_up,
+                                 w->w_down, c.qk_norm ? w->q_norm : nullptr, c.qk_norm ? w->k_norm : nullptr};
   for (const void* const* a : per)
     for (int l = 0; l < c.n_layers; ++l) out->push_back(a ? a[l] : nullptr);
 }
@@ -665,11 +708,12 @@ bool same_key(const StaticState& s, const mk_model_cfg& c, const mk_weight_ptrs*
   const void* head[3] = {w->embed, w->final_norm, w->lm_head};
   for (int i = 0; i < 3; ++i)
     if (s.wkey[i] != head[i]) return false;
-  const void* const* per[9] = {w->attn_norm, w->wq, w->wk, w->wv, w->wo, w->mlp_norm, w->w_gate, w->w_up, w->w_down};
+  const void* const* per[11] = {w->attn_norm, w->wq, w->wk, w->wv, w->wo, w->mlp_norm, w->w_gate, w->w_up,
+                                 w->w_down, c.qk_norm ? w->q_norm : nullptr, c.qk_norm ? w->k_norm : nullptr};
   size_t k = 3;
-  for (const void* const* a : per)
+  for (int a = 0; a < 11; ++a)
     for (int l = 0; l < c.n_layers; ++l, ++k)
-      if (!a || s.wkey[k] != a[l]) return false;
+      if ((per[a] ? per[a][l] : nullptr) != s.wkey[k]) return false;
   return true;
 }
 

@@ -295,6 +295,16 @@ struct AttnPiece {
 };
 
 // Piece j (in order) of range u, or false past the last one.
+// QK-norm: 1/rms of head `head` (query heads first, then key heads) of batch row bi, from
+// the per-unit partial sums the QKV tasks left, added in unit order.
+__device__ __forceinline__ float head_inv_rms(const KParams& p, int bi, int head) {
+  const int per_head = p.hd >> 4;
+  const float* s = p.qkss + ((size_t)bi * (p.nq + p.nkv) + head) * per_head;
+  float acc = 0.f;
+  for (int u = 0; u < per_head; ++u) acc += __ldcg(s + u);
+  return 1.0f / sqrtf(acc / (float)p.hd + p.eps);
+}
+
 __device__ bool attn_piece(const KParams& p, const Smem& sm, int u, int j, AttnPiece& a) {
   const int R = sm.attn_R;
   if (R == 0) {
@@ -806,6 +816,102 @@ __device__ __forceinline__ const bf16* next_gain(const KParams& p, int op, int l
 // ---------------------------------------------------------------------------------------
 // consumer task bodies
 
+// The QKV epilogue: RoPE on queries and keys (the table holds cos and sin of pos *
+// inv_freq), queries to q, keys and values appended to the cache in bf16.
+__device__ __forceinline__ void qkv_epilogue(const KParams& p, Smem& sm, const TaskDesc& t) {
+  const int nthr = kConsumerWarps * 32;
+  const int n = t.nunits;
+  const int half = p.hd / 2, per_head = p.hd >> 4;
+  const int hh = (int)t.u0 / per_head, m0 = (int)t.u0 - hh * per_head;
+  const int items = n * 8 * p.b;
+  for (int idx = threadIdx.x; idx < items; idx += nthr) {
+    const int bi = idx % p.b;
+    const int row = idx / p.b;  // 0 .. 8n-1 within the first half
+    const int j = 8 * m0 + row;
+    const float r = sm.inv_rms[bi];
+    const float x1 = sm.ep[row][bi] * r;
+    const float x2 = sm.ep[8 * n + row][bi] * r;
+    const int pos = sm.in_pos[bi];
+    if (hh < p.nq + p.nkv) {
+      const float2 cs = p.rope[(size_t)pos * half + j];
+      const float o1 = x1 * cs.x - x2 * cs.y;
+      const float o2 = x2 * cs.x + x1 * cs.y;
+      if (hh < p.nq) {
+        float* qd = p.q + (size_t)bi * p.qdim + (size_t)hh * p.hd;
+        qd[j] = o1;
+        qd[j + half] = o2;
+      } else {
+        const int page = p.ptable[bi * p.mpps + pos / kPage];
+        bf16* kd = p.kpool + ((((size_t)t.layer * p.num_pages + page) * p.nkv + (hh - p.nq)) * kPage +
+                              pos % kPage) * p.hd;
+        kd[j] = __float2bfloat16_rn(o1);
+        kd[j + half] = __float2bfloat16_rn(o2);
+      }
+    } else {
+      const int page = p.ptable[bi * p.mpps + pos / kPage];
+      bf16* vd = p.vpool + ((((size_t)t.layer * p.num_pages + page) * p.nkv + (hh - p.nq - p.nkv)) * kPage +
+                            pos % kPage) * p.hd;
+      vd[j] = __float2bfloat16_rn(x1);
+      vd[j + half] = __float2bfloat16_rn(x2);
+    }
+  }
+}
+
+// The QKV epilogue of a QK-norm model (Qwen3).  Per head vector, its 1/rms over head_dim is
+// a common factor of all its components, so RoPE can be applied first: this task writes
+// RoPE(gain * raw) for its rows - queries to q, keys to knew - and its share of the head's
+// sum of squares (its units' rows of both halves, added in row order) to one slot per unit.
+// Where the whole head is read (attention) the slots are added and the factor applied; the
+// key is stored into the cache there.  Values are appended here as usual.
+__device__ __noinline__ void qkv_epilogue_qk_norm(const KParams& p, Smem& sm, const TaskDesc& t) {
+  const int nthr = kConsumerWarps * 32;
+  const int n = t.nunits;
+  const int half = p.hd / 2, per_head = p.hd >> 4;
+  const int hh = (int)t.u0 / per_head, m0 = (int)t.u0 - hh * per_head;
+  const bool qk = hh < p.nq + p.nkv;
+  if (qk)
+    for (int bi = threadIdx.x; bi < p.b; bi += nthr) {
+      const float r = sm.inv_rms[bi];
+      float s = 0.f;
+      for (int row = 0; row < 8 * n; ++row) {
+        const float x1 = sm.ep[row][bi] * r, x2 = sm.ep[8 * n + row][bi] * r;
+        s += x1 * x1 + x2 * x2;
+      }
+      float* slot = p.qkss + ((size_t)bi * (p.nq + p.nkv) + hh) * per_head + m0;
+      slot[0] = s;
+      for (int u = 1; u < n; ++u) slot[u] = 0.f;
+    }
+  const bf16* gain = !qk ? nullptr : (hh < p.nq ? p.layers[t.layer].q_norm : p.layers[t.layer].k_norm);
+  const int items = n * 8 * p.b;
+  for (int idx = threadIdx.x; idx < items; idx += nthr) {
+    const int bi = idx % p.b;
+    const int row = idx / p.b;
+    const int j = 8 * m0 + row;
+    const float r = sm.inv_rms[bi];
+    float x1 = sm.ep[row][bi] * r;
+    float x2 = sm.ep[8 * n + row][bi] * r;
+    const int pos = sm.in_pos[bi];
+    if (qk) {
+      x1 *= __bfloat162float(gain[j]);
+      x2 *= __bfloat162float(gain[j + half]);
+      const float2 cs = p.rope[(size_t)pos * half + j];
+      const float o1 = x1 * cs.x - x2 * cs.y;
+      const float o2 = x2 * cs.x + x1 * cs.y;
+      float* d = hh < p.nq ? p.q + (size_t)bi * p.qdim + (size_t)hh * p.hd
+                           : p.knew + ((size_t)bi * p.nkv + (hh - p.nq)) * p.hd;
+      d[j] = o1;
+      d[j + half] = o2;
+    } else {
+      const int page = p.ptable[bi * p.mpps + pos / kPage];
+      bf16* vd = p.vpool + ((((size_t)t.layer * p.num_pages + page) * p.nkv + (hh - p.nq - p.nkv)) * kPage +
+                            pos % kPage) * p.hd;
+      vd[j] = __float2bfloat16_rn(x1);
+      vd[j + half] = __float2bfloat16_rn(x2);
+    }
+  }
+}
+
+
 __device__ void gemv_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_t& stage, bool& ab, int& inv_inst) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool norm = t.op == OP_QKV || t.op == OP_GATEUP || t.op == OP_LMHEAD;
@@ -877,42 +983,8 @@ __device__ void gemv_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_
     cbar();
   }
   if (t.op == OP_QKV) {
-    if (!ab) {
-      const int half = p.hd / 2, per_head = p.hd >> 4;
-      const int hh = (int)t.u0 / per_head, m0 = (int)t.u0 - hh * per_head;
-      const int items = n * 8 * p.b;
-      for (int idx = threadIdx.x; idx < items; idx += nthr) {
-        const int bi = idx % p.b;
-        const int row = idx / p.b;  // 0 .. 8n-1 within the first half
-        const int j = 8 * m0 + row;
-        const float r = sm.inv_rms[bi];
-        const float x1 = sm.ep[row][bi] * r;
-        const float x2 = sm.ep[8 * n + row][bi] * r;
-        const int pos = sm.in_pos[bi];
-        if (hh < p.nq + p.nkv) {
-          const float2 cs = p.rope[(size_t)pos * half + j];
-          const float o1 = x1 * cs.x - x2 * cs.y;
-          const float o2 = x2 * cs.x + x1 * cs.y;
-          if (hh < p.nq) {
-            float* qd = p.q + (size_t)bi * p.qdim + (size_t)hh * p.hd;
-            qd[j] = o1;
-            qd[j + half] = o2;
-          } else {
-            const int page = p.ptable[bi * p.mpps + pos / kPage];
-            bf16* kd = p.kpool + ((((size_t)t.layer * p.num_pages + page) * p.nkv + (hh - p.nq)) * kPage +
-                                  pos % kPage) * p.hd;
-            kd[j] = __float2bfloat16_rn(o1);
-            kd[j + half] = __float2bfloat16_rn(o2);
-          }
-        } else {
-          const int page = p.ptable[bi * p.mpps + pos / kPage];
-          bf16* vd = p.vpool + ((((size_t)t.layer * p.num_pages + page) * p.nkv + (hh - p.nq - p.nkv)) * kPage +
-                                pos % kPage) * p.hd;
-          vd[j] = __float2bfloat16_rn(x1);
-          vd[j + half] = __float2bfloat16_rn(x2);
-        }
-      }
-    }
+    if (!ab && p.qk_norm) qkv_epilogue_qk_norm(p, sm, t);
+    else if (!ab) qkv_epilogue(p, sm, t);
   } else if (t.op == OP_GATEUP) {
     if (!ab) {
       const int items = n * 8 * p.b;
@@ -1045,7 +1117,10 @@ __device__ __forceinline__ uint32_t split_pair(float x, float y, bool lo) {
 //   * O += P V with A = P split the same way into hi/lo rows and B = V by ldmatrix.trans;
 //   * the 8 warps' (m, l, O) merge in shared memory into one log-sum-exp partial; the last
 //     piece of (i, h) to finish combines all its pieces into the O-projection operand.
-template <int HD>
+// QKN (QK-norm models): queries are scaled by their head's 1/rms, and the new key is
+// normalised and stored here.  A template argument, so that models without QK-norm run code
+// with none of it.
+template <int HD, bool QKN>
 __device__ __noinline__ void attn_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_t& stage, bool& ab) {
   constexpr int T = HD == 64 ? 128 : 96;      // tokens per stage (K then V: 32 / 48 KB)
   constexpr int WPS = T / 16;                 // warps per stage, one 16-token group each
@@ -1069,12 +1144,16 @@ __device__ __noinline__ void attn_task(const KParams& p, Smem& sm, const TaskDes
     {
       const bool hv = g_ < G && !ab;
       const float* qs = p.q + (size_t)a.i * p.qdim + (size_t)(a.h * G + (hv ? g_ : 0)) * HD + 2 * tq;
+      const float rq = (QKN && hv) ? head_inv_rms(p, a.i, a.h * G + g_) : 1.f;
 #pragma unroll
       for (int kk = 0; kk < NK; ++kk) {
         float2 v0 = make_float2(0.f, 0.f), v1 = make_float2(0.f, 0.f);
         if (hv) {
           v0 = __ldcg(reinterpret_cast<const float2*>(qs + 16 * kk));
           v1 = __ldcg(reinterpret_cast<const float2*>(qs + 16 * kk + 8));
+          if (QKN) {
+            v0.x *= rq; v0.y *= rq; v1.x *= rq; v1.y *= rq;
+          }
         }
         qa[kk][0] = split_pair(v0.x, v0.y, false);
         qa[kk][1] = split_pair(v0.x, v0.y, true);
@@ -1103,7 +1182,21 @@ __device__ __noinline__ void attn_task(const KParams& p, Smem& sm, const TaskDes
           const int page = p.ptable[a.i * p.mpps + newpos / kPage];
           const size_t off = ((((size_t)t.layer * p.num_pages + page) * p.nkv + a.h) * kPage + r) * HD;
           constexpr int CH = HD / 8;
-          if (lane < 2 * CH) {
+          if (QKN && lane < CH) {
+            // QK-norm: the key is normalised here, where the whole head vector is complete,
+            // then stored into the cache (this task alone holds the new position of its pair)
+            const float rk = head_inv_rms(p, a.i, p.nq + a.h);
+            const float* src = p.knew + ((size_t)a.i * p.nkv + a.h) * HD + lane * 8;
+            const float4 f0 = __ldcg(reinterpret_cast<const float4*>(src));
+            const float4 f1 = __ldcg(reinterpret_cast<const float4*>(src + 4));
+            uint4 v;
+            v.x = pack_bf16(f0.x * rk, f0.y * rk);
+            v.y = pack_bf16(f0.z * rk, f0.w * rk);
+            v.z = pack_bf16(f1.x * rk, f1.y * rk);
+            v.w = pack_bf16(f1.z * rk, f1.w * rk);
+            *reinterpret_cast<uint4*>(p.kpool + off + lane * 8) = v;
+            *reinterpret_cast<uint4*>(kpg + kv_off(r, lane)) = v;
+          } else if (lane < 2 * CH) {
             const int ch = lane % CH;
             const uint4 v = __ldcg(reinterpret_cast<const uint4*>((lane < CH ? p.kpool : p.vpool) + off + ch * 8));
             *reinterpret_cast<uint4*>((lane < CH ? kpg : vpg) + kv_off(r, ch)) = v;
@@ -1524,8 +1617,13 @@ __device__ void consumer(const KParams& p, Smem& sm, const TaskDesc* ts, int nt)
     switch (t.op) {
       case OP_EMBED: embed_task(p, sm, t, ab); break;
       case OP_ATTN:
-        if (p.hd == 64) attn_task<64>(p, sm, t, stage, ab);
-        else attn_task<128>(p, sm, t, stage, ab);
+        if (p.hd == 64) {
+          if (p.qk_norm) attn_task<64, true>(p, sm, t, stage, ab);
+          else attn_task<64, false>(p, sm, t, stage, ab);
+        } else {
+          if (p.qk_norm) attn_task<128, true>(p, sm, t, stage, ab);
+          else attn_task<128, false>(p, sm, t, stage, ab);
+        }
         break;
       default: gemv_task(p, sm, t, stage, ab, inv_inst); break;
     }
@@ -1668,14 +1766,14 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
   else consumer(p, sm, p.tasks + o0, (int)(o1 - o0));
 }
 
-// RoPE table: (cos, sin) of pos * theta^(-2j/hd), computed in double, stored as fp32.
-__global__ void rope_table_kernel(float2* table, int max_ctx, int hd, double theta) {
+// RoPE table: (cos, sin) of pos * inv_freq_j, computed in double, stored as fp32.
+__global__ void rope_table_kernel(float2* table, int max_ctx, int hd, const RopeFreq f) {
   const int half = hd / 2;
   const long long n = (long long)max_ctx * half;
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < n;
        idx += (long long)gridDim.x * blockDim.x) {
     const int pos = (int)(idx / half), j = (int)(idx % half);
-    const double inv = pow(theta, -2.0 * j / hd);
+    const double inv = f.inv_freq[j];
     double sn, cs;
     sincos((double)pos * inv, &sn, &cs);
     table[idx] = make_float2((float)cs, (float)sn);
@@ -1696,8 +1794,8 @@ cudaError_t launch_decode(const KParams& p, cudaStream_t s) {
   return cudaLaunchKernelEx(&cfg, mk_decode_kernel, p);
 }
 
-cudaError_t launch_rope_table(float2* table, int max_ctx, int hd, double theta, cudaStream_t s) {
-  rope_table_kernel<<<256, 256, 0, s>>>(table, max_ctx, hd, theta);
+cudaError_t launch_rope_table(float2* table, int max_ctx, int hd, const RopeFreq& f, cudaStream_t s) {
+  rope_table_kernel<<<256, 256, 0, s>>>(table, max_ctx, hd, f);
   return cudaGetLastError();
 }
 

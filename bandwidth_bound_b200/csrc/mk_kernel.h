@@ -10,6 +10,7 @@ namespace mk {
 
 struct LayerW {
   const __nv_bfloat16 *attn_norm, *wq, *wk, *wv, *wo, *mlp_norm, *wg, *wu, *wd;
+  const __nv_bfloat16 *q_norm, *k_norm;  // QK-norm gains [hd] (null without QK-norm)
 };
 
 struct alignas(64) TmaDesc {  // the driver's opaque 128-byte TMA descriptor (CUtensorMap)
@@ -49,6 +50,12 @@ struct KParams {
   uint32_t *ctr, *cmb, *ctl; // counters, split-K combine counters, {abort, status}
   int* host_status;          // mapped host word
   const float2* rope;        // [max_ctx][hd/2] (cos, sin)
+  // QK-norm: per (batch row, q or k head) partial sums of squares of the raw head vector,
+  // one slot per 16-row QKV unit of the head [max_b][nq + nkv][hd / 16]; the new keys
+  // rotated but not yet normalised [max_b][nkv][hd] (the attention task holding the new
+  // position normalises and stores them)
+  int qk_norm;
+  float *qkss, *knew;
   // this step
   const int *tok, *pos, *lens;  // lens may be null: pos + 1
   int b;
@@ -69,7 +76,10 @@ struct KParams {
 
 size_t kernel_smem_bytes();
 cudaError_t launch_decode(const KParams& p, cudaStream_t s);
-cudaError_t launch_rope_table(float2* table, int max_ctx, int hd, double theta, cudaStream_t s);
+struct RopeFreq {
+  double inv_freq[64];  // per rotation pair j < hd / 2
+};
+cudaError_t launch_rope_table(float2* table, int max_ctx, int hd, const RopeFreq& f, cudaStream_t s);
 cudaError_t kernel_attributes(int* regs, int* local_bytes, int* max_threads);
 
 }  // namespace mk

@@ -106,6 +106,13 @@ int check_cfg(const mk_model_cfg& c, std::string* err) {
     set_err(err, "model cfg: rms_eps must be > 0 and rope_theta > 1");
     return MK_ERR_INVALID_ARG;
   }
+  if (c.rope_scale_factor > 1.f &&
+      !(c.rope_low_freq_factor > 0.f && c.rope_high_freq_factor > c.rope_low_freq_factor &&
+        c.rope_original_max_pos > 0)) {
+    set_err(err, "model cfg: RoPE scaling needs 0 < low_freq_factor < high_freq_factor and original_max_pos > 0");
+    return MK_ERR_INVALID_ARG;
+  }
+  if (c.qk_norm != 0 && c.qk_norm != 1) { set_err(err, "model cfg: qk_norm must be 0 or 1"); return MK_ERR_INVALID_ARG; }
   if (c.page_size != kPage) { set_err(err, "page_size must be %d", kPage); return MK_ERR_UNSUPPORTED_CFG; }
   if (c.head_dim != 64 && c.head_dim != 128) { set_err(err, "head_dim must be 64 or 128"); return MK_ERR_UNSUPPORTED_CFG; }
   if (c.n_heads % c.n_kv_heads) { set_err(err, "n_heads must be a multiple of n_kv_heads"); return MK_ERR_UNSUPPORTED_CFG; }

@@ -446,7 +446,7 @@ def run_mk(args, world, rank, local):
                          "frac_of_measured_copy": sec["achieved_gbs"] / peaks["hbm_gbs"], "l2": l2_note})
         del wts, kv
         torch.cuda.empty_cache()
-        for name in ("tiny-b1", "smollm2-135m-b1", "llama3.2-1b-b9", "llama2-13b-b4"):
+        for name in ("tiny-b1", "smollm2-135m-b1", "llama3.2-1b-b9", "llama2-13b-b4", "qwen3-0.6b-b1", "qwen3-8b-b1"):
             rows.extend(time_config(mk, name, stream, min(args.steps, 200), args.warmup, peaks))
         line["all_configs"] = rows
     if rank == 0:

@@ -64,19 +64,32 @@ typedef struct mk_model_cfg {
   int32_t max_batch;   /* largest batch a step may use */
   int32_t max_ctx;     /* largest position + 1 a sequence may reach */
   int32_t page_size;   /* KV tokens per page; must be 16 */
+  /* Llama-3.x RoPE frequency scaling ("rope_type llama3"); rope_scale_factor <= 1 turns it
+   * off.  With wavelength w_j = 2 pi / inv_freq_j and the original context length N:
+   * w_j < N / high_freq_factor keeps inv_freq_j; w_j > N / low_freq_factor divides it by
+   * the factor; in between s = (N / w_j - low) / (high - low) blends the two,
+   * (1 - s) inv_freq_j / factor + s inv_freq_j.  The table is built once, in double. */
+  float rope_scale_factor, rope_low_freq_factor, rope_high_freq_factor;
+  int32_t rope_original_max_pos;
+  /* 1: Qwen3-style QK-norm - every query and key head vector is RMS-normalised over
+   * head_dim (epsilon rms_eps) and multiplied by the layer's gain q_norm / k_norm before
+   * RoPE; the stored key is the normalised, rotated one.  0: none. */
+  int32_t qk_norm;
 } mk_model_cfg;
 
 /* Device pointers to bf16 weights.  The per-layer members are HOST arrays of
  * n_layers device pointers each.  Shapes ([out][in]): embed, lm_head [vocab][hidden];
  * final_norm, attn_norm[l], mlp_norm[l] [hidden]; wq [n_heads*head_dim][hidden];
  * wk, wv [n_kv_heads*head_dim][hidden]; wo [hidden][n_heads*head_dim];
- * w_gate, w_up [ffn][hidden]; w_down [hidden][ffn].  Every pointer 16-byte aligned.
+ * w_gate, w_up [ffn][hidden]; w_down [hidden][ffn]; q_norm[l], k_norm[l] [head_dim]
+ * (only with cfg.qk_norm; NULL arrays otherwise).  Every pointer 16-byte aligned.
  * The handle keeps the device pointers (not the host arrays); the weights must
  * outlive the handle. */
 typedef struct mk_weight_ptrs {
   const void *embed, *final_norm, *lm_head;
   const void *const *attn_norm, *const *wq, *const *wk, *const *wv, *const *wo;
   const void *const *mlp_norm, *const *w_gate, *const *w_up, *const *w_down;
+  const void *const *q_norm, *const *k_norm;
 } mk_weight_ptrs;
 
 /* Paged KV cache (device, caller-owned).  k_pool and v_pool are bf16

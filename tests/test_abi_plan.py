@@ -32,12 +32,14 @@ def test_library_exports_every_declared_entry_point(lib):
 
 
 def test_cfg_struct_sizes_match_header():
-    assert ctypes.sizeof(mk.ModelCfg) == 13 * 4
+    assert ctypes.sizeof(mk.ModelCfg) == 18 * 4
     assert ctypes.sizeof(mk.KvCache) == 3 * 8 + 2 * 4
-    assert ctypes.sizeof(mk.WeightPtrs) == 12 * 8
+    assert ctypes.sizeof(mk.WeightPtrs) == 14 * 8
+    assert ctypes.sizeof(mk.Sampling) == 2 * 4 + 8
 
 
-ALL_MODELS = [synth.TINY, synth.SMOLLM2_135M, synth.LLAMA32_1B, synth.LLAMA3_8B, synth.LLAMA2_13B]
+ALL_MODELS = [synth.TINY, synth.SMOLLM2_135M, synth.LLAMA32_1B, synth.LLAMA3_8B, synth.LLAMA2_13B, synth.QWEN3_0_6B,
+              synth.QWEN3_8B]
 
 
 @pytest.mark.parametrize("m", ALL_MODELS, ids=lambda m: m.name)
