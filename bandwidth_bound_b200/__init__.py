@@ -91,6 +91,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "mk_create_from_plan": (ctypes.c_int, [vp, ctypes.POINTER(WeightPtrs), i32, ctypes.POINTER(vp)]),
         "mk_decode_step": (ctypes.c_int, [vp, vp, vp, vp, i32, ctypes.POINTER(KvCache), vp, vp, vp]),
         "mk_decode_step_host": (ctypes.c_int, [vp, vp, vp, vp, i32, ctypes.POINTER(KvCache), vp, vp, vp]),
+        "mk_verify_step": (ctypes.c_int, [vp, vp, vp, vp, vp, i32, ctypes.POINTER(KvCache), vp, vp, vp]),
         "mk_decode_steps": (ctypes.c_int, [vp, i32, vp, vp, i32, ctypes.POINTER(KvCache), ctypes.POINTER(Sampling),
                                            vp, vp, vp]),
         "mk_decode_step_static": (ctypes.c_int, [ctypes.POINTER(ModelCfg), ctypes.POINTER(WeightPtrs), vp, vp, vp,
@@ -253,6 +254,20 @@ class Megakernel:
                                      ctypes.c_void_p(stream.cuda_stream))
         if check:
             _check(rc, self.handle, "mk_decode_step")
+        return rc
+
+    def verify(self, token_ids, positions, seq_lens, group_first, kv, logits, argmax=None, stream=None,
+               check: bool = True) -> int:
+        """A multi-token step: rows of one sequence (group_first) at consecutive positions,
+        attending causally to each other's new tokens."""
+        if stream is None:
+            stream = self._torch.cuda.current_stream()
+        kvs = self.kv_struct(kv)
+        rc = self.lib.mk_verify_step(self.handle, _ptr(token_ids), _ptr(positions), _ptr(seq_lens), _ptr(group_first),
+                                     int(token_ids.numel()), ctypes.byref(kvs), _ptr(logits), _ptr(argmax),
+                                     ctypes.c_void_p(stream.cuda_stream))
+        if check:
+            _check(rc, self.handle, "mk_verify_step")
         return rc
 
     def steps(self, n_steps: int, token_ids, positions, kv, tokens_out, logits=None, stream=None,

@@ -510,7 +510,8 @@ static int check_step_args(mk_handle_t h, const void* tok, const void* pos, cons
 
 static int launch_step(mk_handle_t h, const int32_t* tok, const int32_t* pos, const int32_t* lens, int32_t batch,
                        const mk_kv_cache* kv, float* logits, int32_t* argmax, cudaStream_t s, int step_add = 0,
-                       const mk_sampling* smp = nullptr, const float* uniforms = nullptr) {
+                       const mk_sampling* smp = nullptr, const float* uniforms = nullptr,
+                       const int32_t* group_first = nullptr) {
   if (kv->k_pool != h->kv_k || kv->v_pool != h->kv_v || kv->num_pages != h->kv_pages) {
     const std::string e = encode_kv_maps(h->plan.cfg, kv, h->kp);
     if (!e.empty()) {
@@ -523,6 +524,7 @@ static int launch_step(mk_handle_t h, const int32_t* tok, const int32_t* pos, co
   }
   KParams p = h->kp;
   p.tok = tok; p.pos = pos; p.lens = lens; p.b = batch; p.step_add = step_add;
+  p.group_first = group_first;
   p.kpool = (__nv_bfloat16*)kv->k_pool; p.vpool = (__nv_bfloat16*)kv->v_pool;
   p.ptable = kv->page_table; p.num_pages = kv->num_pages; p.mpps = kv->max_pages_per_seq;
   p.logits = logits; p.argmax = argmax;
@@ -574,6 +576,17 @@ MK_API int mk_decode_steps(mk_handle_t h, int32_t n_steps, const int32_t* token_
     if (rc) return rc;
   }
   return MK_OK;
+}
+
+MK_API int mk_verify_step(mk_handle_t h, const int32_t* token_ids, const int32_t* positions,
+                          const int32_t* seq_lens, const int32_t* group_first, int32_t batch, const mk_kv_cache* kv,
+                          float* logits_out, int32_t* argmax_out, mk_stream_t stream) {
+  if (!h) return fail(nullptr, MK_ERR_INVALID_ARG, "mk_verify_step: null handle");
+  if (!group_first) return fail(h, MK_ERR_INVALID_ARG, "mk_verify_step: null group_first");
+  int rc = check_step_args(h, token_ids, positions, seq_lens, batch, kv, logits_out);
+  if (rc) return rc;
+  return launch_step(h, token_ids, positions, seq_lens, batch, kv, logits_out, argmax_out, (cudaStream_t)stream, 0,
+                     nullptr, nullptr, group_first);
 }
 
 MK_API int mk_decode_step_host(mk_handle_t h, const int32_t* token_ids, const int32_t* positions,

@@ -50,6 +50,8 @@ struct Smem {
   int in_tok[kMaxBatch];         // this step's token, position and keys attended per sequence,
   int in_pos[kMaxBatch];         // read once from the step's inputs (positions offset by the
   int in_len[kMaxBatch];         // step's index in a multi-step run)
+  int in_grow0[kMaxBatch];       // multi-token step: first batch row of the row's sequence
+  int in_fresh[kMaxBatch];       // first position written by this step in the row's sequence
   unsigned long long wait_cyc;  // tracing: SM cycles warp 0 spent waiting for pool slots in the current task
   unsigned long long tm[3];     // tracing: compute, reduce, epilogue SM cycles of the current task (warp 0)
 };
@@ -1176,17 +1178,22 @@ __device__ __noinline__ void attn_task(const KParams& p, Smem& sm, const TaskDes
         uint8_t* kpg = sm.pool[slot] + grp * PAGE;
         uint8_t* vpg = sm.pool[slot] + T * HD * 2 + grp * PAGE;
         bool wrote = false;
-        if (newpos >= g0 && newpos < g0 + 16) {
-          // the new token's K/V, written by this layer's QKV tasks after the page was fetched
-          const int r = newpos - g0;
-          const int page = p.ptable[a.i * p.mpps + newpos / kPage];
-          const size_t off = ((((size_t)t.layer * p.num_pages + page) * p.nkv + a.h) * kPage + r) * HD;
+        // positions this step wrote: the row's own new token and, in a multi-token step, the
+        // earlier new tokens of its sequence (rows grow0.. of the batch) - fetched before they
+        // were written, so taken again from where this step's QKV tasks left them
+        const int fresh = sm.in_fresh[a.i];
+        const int q0 = max(fresh, g0), q1 = min(newpos, g0 + 15);
+        for (int q = q0; q <= q1; ++q) {
+          const int r = q - g0;
+          const int page = p.ptable[a.i * p.mpps + q / kPage];
+          const size_t off = ((((size_t)t.layer * p.num_pages + page) * p.nkv + a.h) * kPage + q % kPage) * HD;
           constexpr int CH = HD / 8;
           if (QKN && lane < CH) {
-            // QK-norm: the key is normalised here, where the whole head vector is complete,
-            // then stored into the cache (this task alone holds the new position of its pair)
-            const float rk = head_inv_rms(p, a.i, p.nq + a.h);
-            const float* src = p.knew + ((size_t)a.i * p.nkv + a.h) * HD + lane * 8;
+            // QK-norm: the key is normalised here, where the whole head vector is complete;
+            // the task holding a row's own new position stores it into the cache
+            const int row = sm.in_grow0[a.i] + (q - fresh);  // the batch row whose token sits at q
+            const float rk = head_inv_rms(p, row, p.nq + a.h);
+            const float* src = p.knew + ((size_t)row * p.nkv + a.h) * HD + lane * 8;
             const float4 f0 = __ldcg(reinterpret_cast<const float4*>(src));
             const float4 f1 = __ldcg(reinterpret_cast<const float4*>(src + 4));
             uint4 v;
@@ -1194,7 +1201,7 @@ __device__ __noinline__ void attn_task(const KParams& p, Smem& sm, const TaskDes
             v.y = pack_bf16(f0.z * rk, f0.w * rk);
             v.z = pack_bf16(f1.x * rk, f1.y * rk);
             v.w = pack_bf16(f1.z * rk, f1.w * rk);
-            *reinterpret_cast<uint4*>(p.kpool + off + lane * 8) = v;
+            if (q == newpos) *reinterpret_cast<uint4*>(p.kpool + off + lane * 8) = v;
             *reinterpret_cast<uint4*>(kpg + kv_off(r, lane)) = v;
           } else if (lane < 2 * CH) {
             const int ch = lane % CH;
@@ -1744,6 +1751,15 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
       sm.in_tok[i] = tk;
       sm.in_pos[i] = ps;
       sm.in_len[i] = ln;
+      // rows of one sequence in a multi-token step: consecutive, at consecutive positions
+      const int g0 = p.group_first ? p.group_first[i] : i;
+      sm.in_grow0[i] = g0;
+      sm.in_fresh[i] = ps;
+      if (g0 < 0 || g0 > i) bad = 1;
+      else if (g0 < i) {
+        sm.in_fresh[i] = sm.in_fresh[g0];
+        if (sm.in_grow0[g0] != g0 || ps != sm.in_pos[g0] + (i - g0)) bad = 1;
+      }
       if (tk < 0 || tk >= p.V || ps < 0 || ps >= p.max_ctx || ln != ps + 1 || ps / kPage >= p.mpps) bad = 1;
       else {
         const int pg = p.ptable[i * p.mpps + ps / kPage];

@@ -60,6 +60,7 @@ struct KParams {
   const int *tok, *pos, *lens;  // lens may be null: pos + 1
   int b;
   int step_add;                 // added to every position (and length): step index of a multi-step run
+  const int* group_first;       // multi-token step: first row of each row's sequence (null: every row its own)
   __nv_bfloat16 *kpool, *vpool;
   const int* ptable;
   int num_pages, mpps;

@@ -166,6 +166,25 @@ MK_API int mk_decode_step(mk_handle_t h, const int32_t *token_ids, const int32_t
                           const int32_t *seq_lens, int32_t batch, const mk_kv_cache *kv,
                           float *logits_out, int32_t *argmax_out, mk_stream_t stream);
 
+/* A multi-token step in one launch: several new tokens of one sequence at once, as when a
+ * draft's tokens are verified (speculative decoding) or a prompt is fed in chunks.  Each
+ * new token is a batch row; the rows of one sequence are consecutive and sit at
+ * consecutive positions.  Row r attends causally: to its sequence's prior entries and to
+ * the new tokens of the rows before it in its sequence, and appends its own K/V at its
+ * position.  The projections read every weight once for all rows, as for a batch.
+ *   group_first device int32 [batch]: the first row of row r's sequence (r itself for a
+ *               sequence with one new token); rows first..r must satisfy
+ *               positions[r] = positions[first] + (r - first)
+ *   page_table  rows r of one sequence must map the same pages (the caller repeats the
+ *               sequence's row); entries up to each row's position must be present
+ *   the rest as for mk_decode_step (seq_lens[r] = positions[r] + 1; logits and argmax per
+ *   row, i.e. per new token).
+ * A group_first that breaks these rules is reported as MK_ERR_BOUNDS on the device. */
+MK_API int mk_verify_step(mk_handle_t h, const int32_t *token_ids, const int32_t *positions,
+                          const int32_t *seq_lens, const int32_t *group_first, int32_t batch,
+                          const mk_kv_cache *kv, float *logits_out, int32_t *argmax_out,
+                          mk_stream_t stream);
+
 /* Top-k sampling of the next token (the engine's sampler, ForgeMegakernel §4.3), done
  * inside the step's launch by the CTA that releases the LM head's last task, one warp per
  * sequence.  For sequence i of step s, with u = uniforms[s][i]:
