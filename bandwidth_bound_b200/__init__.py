@@ -96,6 +96,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                            vp, vp, vp]),
         "mk_decode_step_static": (ctypes.c_int, [ctypes.POINTER(ModelCfg), ctypes.POINTER(WeightPtrs), vp, vp, vp,
                                                  i32, ctypes.POINTER(KvCache), vp, vp, vp]),
+        "mk_route_pick": (ctypes.c_int, [ctypes.POINTER(i32), ctypes.POINTER(i32), i32, i32, i32]),
+        "mk_router_create": (ctypes.c_int, [ctypes.POINTER(vp), i32, ctypes.POINTER(vp)]),
+        "mk_router_step": (ctypes.c_int, [vp, vp, vp, vp, i32, i32, ctypes.POINTER(KvCache), vp, vp,
+                                          ctypes.POINTER(i32), vp]),
+        "mk_router_destroy": (ctypes.c_int, [vp]),
         "mk_get_status": (ctypes.c_int, [vp]),
         "mk_reset": (ctypes.c_int, [vp]),
         "mk_set_debug": (ctypes.c_int, [vp, vp]),
@@ -337,6 +342,49 @@ class Megakernel:
             self.close()
         except Exception:
             pass
+
+
+def route_pick(bounds, batch: int, max_position: int) -> int:
+    """The router's rule on [(max_batch, max_ctx), ...]: index of the handle a step goes to,
+    or a negative status when none covers it."""
+    lib = load_library()
+    n = len(bounds)
+    mb = (ctypes.c_int32 * n)(*[int(b) for b, _ in bounds])
+    mc = (ctypes.c_int32 * n)(*[int(c) for _, c in bounds])
+    return lib.mk_route_pick(mb, mc, n, int(batch), int(max_position))
+
+
+class Router:
+    """Steps routed among handles of one model built for different bounds (mk_router_*)."""
+
+    def __init__(self, handles):
+        import torch
+
+        self.lib = load_library()
+        self._torch = torch
+        self.handles = list(handles)
+        arr = (ctypes.c_void_p * len(self.handles))(*[h.handle.value for h in self.handles])
+        self.ptr = ctypes.c_void_p()
+        _check(self.lib.mk_router_create(arr, len(self.handles), ctypes.byref(self.ptr)), None, "mk_router_create")
+
+    def step(self, token_ids, positions, seq_lens, max_position: int, kv, logits, argmax=None, stream=None,
+             check: bool = True):
+        """One step on the picked handle; returns (status, picked index)."""
+        if stream is None:
+            stream = self._torch.cuda.current_stream()
+        picked = ctypes.c_int32(-1)
+        kvs = Megakernel.kv_struct(kv)
+        rc = self.lib.mk_router_step(self.ptr, _ptr(token_ids), _ptr(positions), _ptr(seq_lens),
+                                     int(token_ids.numel()), int(max_position), ctypes.byref(kvs), _ptr(logits),
+                                     _ptr(argmax), ctypes.byref(picked), ctypes.c_void_p(stream.cuda_stream))
+        if check:
+            _check(rc, None, "mk_router_step")
+        return rc, picked.value
+
+    def close(self):
+        if self.ptr:
+            self.lib.mk_router_destroy(self.ptr)
+            self.ptr = ctypes.c_void_p()
 
 
 def decode_step_static(m, weights: dict, max_batch: int, max_ctx: int, token_ids, positions, seq_lens, kv,

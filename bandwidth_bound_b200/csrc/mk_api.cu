@@ -670,6 +670,61 @@ MK_API int mk_destroy(mk_handle_t h) {
 
 MK_API const char* mk_last_error(mk_handle_t h) { return h ? h->err.c_str() : g_err.c_str(); }
 
+MK_API int mk_route_pick(const int32_t* max_batch, const int32_t* max_ctx, int32_t n, int32_t batch,
+                         int32_t max_position) {
+  if (!max_batch || !max_ctx || n < 1 || batch < 1 || max_position < 0) return MK_ERR_INVALID_ARG;
+  int best = -1;
+  for (int i = 0; i < n; ++i) {
+    if (max_batch[i] < batch || max_ctx[i] <= max_position) continue;
+    if (best < 0 || max_batch[i] < max_batch[best] ||
+        (max_batch[i] == max_batch[best] && max_ctx[i] < max_ctx[best]))
+      best = i;
+  }
+  return best < 0 ? MK_ERR_INVALID_ARG : best;
+}
+
+struct mk_router_s {
+  std::vector<mk_handle_t> handles;
+  std::vector<int32_t> max_batch, max_ctx;
+};
+
+MK_API int mk_router_create(const mk_handle_t* handles, int32_t n, mk_router_t* out) {
+  if (!handles || n < 1 || !out) return fail(nullptr, MK_ERR_INVALID_ARG, "mk_router_create: bad arguments");
+  mk_router_t r = new mk_router_s();
+  for (int i = 0; i < n; ++i) {
+    if (!handles[i]) { delete r; return fail(nullptr, MK_ERR_INVALID_ARG, "mk_router_create: null handle"); }
+    const mk_model_cfg& c = handles[i]->plan.cfg;
+    const mk_model_cfg& c0 = handles[0]->plan.cfg;
+    if (c.n_layers != c0.n_layers || c.hidden != c0.hidden || c.vocab != c0.vocab || c.n_heads != c0.n_heads ||
+        c.n_kv_heads != c0.n_kv_heads || c.head_dim != c0.head_dim || c.ffn != c0.ffn) {
+      delete r;
+      return fail(nullptr, MK_ERR_INVALID_ARG, "mk_router_create: handles of different models");
+    }
+    r->handles.push_back(handles[i]);
+    r->max_batch.push_back(c.max_batch);
+    r->max_ctx.push_back(c.max_ctx);
+  }
+  *out = r;
+  return MK_OK;
+}
+
+MK_API int mk_router_step(mk_router_t r, const int32_t* token_ids, const int32_t* positions, const int32_t* seq_lens,
+                          int32_t batch, int32_t max_position, const mk_kv_cache* kv, float* logits_out,
+                          int32_t* argmax_out, int32_t* picked, mk_stream_t stream) {
+  if (!r) return fail(nullptr, MK_ERR_INVALID_ARG, "mk_router_step: null router");
+  const int i = mk_route_pick(r->max_batch.data(), r->max_ctx.data(), (int32_t)r->handles.size(), batch,
+                              max_position);
+  if (i < 0) return fail(nullptr, MK_ERR_INVALID_ARG, "mk_router_step: no handle covers this batch and position");
+  if (picked) *picked = i;
+  return mk_decode_step(r->handles[i], token_ids, positions, seq_lens, batch, kv, logits_out, argmax_out, stream);
+}
+
+MK_API int mk_router_destroy(mk_router_t r) {
+  if (!r) return MK_ERR_INVALID_ARG;
+  delete r;
+  return MK_OK;
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------------------------------

@@ -303,6 +303,31 @@ MK_API int mk_launches_per_step(mk_handle_t h);
 
 MK_API int mk_destroy(mk_handle_t h);
 
+/* ---- routing among handles specialised by bounds ------------------------------------ */
+
+/* A handle is built for bounds (cfg.max_batch, cfg.max_ctx); its schedule is specialised to
+ * them - a handle for batch <= 4 stages fp32 operand rows and so more weight columns per
+ * pool stage than one for batch 8 - the counterpart of the pages' per-kernel compile-time
+ * batch size and context bound with requests routed among kernels (ForgeMegakernel §5.3,
+ * Figure 5).  A router holds several handles of one model (same weights) and sends each
+ * step to the handle with the smallest max_batch >= batch, ties broken by the smallest
+ * max_ctx > max_position, then by the lower index.
+ *   mk_route_pick: the rule alone, on host arrays of the n handles' bounds; returns the
+ *   index, or MK_ERR_INVALID_ARG when no handle fits.  No GPU needed.
+ *   mk_router_create: copies the n handle pointers (the router does not own the handles;
+ *   they must outlive it).  mk_router_step: max_position is the largest positions[i]
+ *   (host int: the positions themselves are device memory); the other arguments as for
+ *   mk_decode_step, run on the picked handle, whose index goes to *picked (may be NULL). */
+typedef struct mk_router_s *mk_router_t;
+MK_API int mk_route_pick(const int32_t *max_batch, const int32_t *max_ctx, int32_t n, int32_t batch,
+                         int32_t max_position);
+MK_API int mk_router_create(const mk_handle_t *handles, int32_t n, mk_router_t *out);
+MK_API int mk_router_step(mk_router_t r, const int32_t *token_ids, const int32_t *positions,
+                          const int32_t *seq_lens, int32_t batch, int32_t max_position,
+                          const mk_kv_cache *kv, float *logits_out, int32_t *argmax_out,
+                          int32_t *picked, mk_stream_t stream);
+MK_API int mk_router_destroy(mk_router_t r);
+
 /* Message of the last failure on h (NULL: of the last handle-less call). */
 MK_API const char *mk_last_error(mk_handle_t h);
 
