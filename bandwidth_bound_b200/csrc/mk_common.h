@@ -30,7 +30,8 @@ constexpr int kSigRing = 4;                             // finished tasks the co
 constexpr int kSlotBytes = 50 * 1024;                   // one pool stage: weights + their operands, or KV pages
 constexpr int kNumSlots = 4;                            // pool depth (200 KB; 4 x 50 KB measured fastest)
 constexpr int kMaxBatch = 16;
-constexpr int kFmaRows = 4;                             // batches up to this size run the GEMVs on fp32 FMA
+constexpr int kFmaRows = 2;                             // batches up to this size run the GEMVs on fp32 FMA
+constexpr int kTriRows = 4;                             // batches up to this size split activations in three bf16 parts
 constexpr int kMaxBlocks = 8;                           // 8-row blocks per GEMV task (64 rows)
 constexpr int kPage = 16;                               // tokens per KV page
 constexpr int kMaxChunksPerSeq = 32;                    // split-K chunks per (sequence, kv head)
@@ -96,8 +97,8 @@ MK_HD int max_units(int op) { return (op == OP_QKV || op == OP_GATEUP) ? kMaxBlo
 MK_HD uint32_t ceil_div(uint32_t a, uint32_t b) { return (a + b - 1) / b; }
 MK_HD int round_up(int a, int b) { return (a + b - 1) / b * b; }
 
-// fp32 operand rows a stage carries for a batch of b <= kFmaRows rows (1, 2 or 4).
-MK_HD int fma_rows(int b) { return b == 1 ? 1 : (b == 2 ? 2 : kFmaRows); }
+// fp32 operand rows a stage carries for a batch of b <= kFmaRows rows (1 or 2).
+MK_HD int fma_rows(int b) { return b == 1 ? 1 : kFmaRows; }
 
 // Operand bytes per K column of one stage for a batch of up to max_batch rows: bf16 hi and
 // lo parts of every 8-row batch tile (16 bytes each per column), or, when every batch the

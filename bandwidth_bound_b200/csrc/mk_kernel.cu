@@ -640,17 +640,27 @@ __device__ void compute_inv_rms(const KParams& p, Smem& sm, int inst, int nparts
 }
 
 // Store one GEMV operand value (batch row bi, column k) in the layout this step's GEMVs read:
-// fp32 rows for batches up to kFmaRows (the FMA path), else its bf16 hi part and the bf16 lo
-// part of the remainder in the tile layout.
+// fp32 rows for batches up to kFmaRows (the FMA path); else bf16 parts in the tile layout.
+// Up to kTriRows batch rows, three parts (hi, mid, lo: ~24 bits, as fp32) fill the 16 rows of
+// one MMA tile - hi in rows 0-3, mid in rows 4-7, lo in rows 8-11; above that, two parts (hi
+// in rows 0-7, lo in rows 8-15; ~16 bits).  Each part is the bf16 rounding of what the parts
+// before it left over, which is exact in fp32.
 __device__ __forceinline__ void put_operand(const KParams& p, bf16* tiles, float* f, int ld, int bi, int k, float v) {
   if (p.b <= kFmaRows) {
     f[(size_t)bi * ld + opnd_row0_index(k)] = v;
     return;
   }
   const bf16 h = __float2bfloat16_rn(v);
+  const float r1 = v - __bfloat162float(h);
   const int mt = bi >> 3, row = bi & 7;
   tiles[opnd_tile_index(mt, 0, k, row, ld)] = h;
-  tiles[opnd_tile_index(mt, 1, k, row, ld)] = __float2bfloat16_rn(v - __bfloat162float(h));
+  if (p.b <= kTriRows) {
+    const bf16 m = __float2bfloat16_rn(r1);
+    tiles[opnd_tile_index(0, 0, k, row + 4, ld)] = m;
+    tiles[opnd_tile_index(0, 1, k, row, ld)] = __float2bfloat16_rn(r1 - __bfloat162float(m));
+  } else {
+    tiles[opnd_tile_index(mt, 1, k, row, ld)] = __float2bfloat16_rn(r1);
+  }
 }
 
 // Stream the task's stages through the eight warps and reduce into sm.ep[row][batch].
@@ -661,10 +671,10 @@ __device__ __forceinline__ void put_operand(const KParams& p, bf16* tiles, float
 // 16-byte pieces of chunk kb / 2, so lane (g, tq) reads piece 2*tq + h of row 8j + g -
 // conflict-free - which holds columns 16*tq + 8*h .. +7, and the operand piece of the same
 // columns at `lane` (bf16) or `tq` (fp32, shared by the 8 lanes of one tq).
-// MT = 0: CUDA-core FMA on fp32 activations for NB (1, 2 or 4 >= batch) rows, the operands of
+// MT = 0: CUDA-core FMA on fp32 activations for NB (1 or 2 = batch) rows, the operands of
 // chunk c row r at (c * NB + r) * 256 bytes; MT = 1, 2: mma.sync with MT tiles of 8 batch
-// rows, rows 0-7 of the M = 16 tile the bf16 hi parts, rows 8-15 the lo parts.
-template <int MT, int G, int NB = 1>
+// rows, the M = 16 tile holding the bf16 parts of the activations (put_operand).
+template <int MT, int G, int NB = 1, bool TRI = false>
 __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDesc t, uint32_t& stage, bool& ab) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, tq = lane & 3;
@@ -770,7 +780,12 @@ __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDes
             if (tq == 0) red[((warp * kMaxBlocks + j) * 8 + r) * 8 + g] = v;
           }
         } else {
-          const float2 y = make_float2(acc[j][mt][0] + acc[j][mt][2], acc[j][mt][1] + acc[j][mt][3]);
+          float2 y = make_float2(acc[j][mt][0] + acc[j][mt][2], acc[j][mt][1] + acc[j][mt][3]);
+          if constexpr (TRI) {
+            // three-part activations: batch row g's mid part is D row g + 4, held by lane + 16
+            y.x += __shfl_down_sync(0xffffffffu, acc[j][mt][0], 16);
+            y.y += __shfl_down_sync(0xffffffffu, acc[j][mt][1], 16);
+          }
           *reinterpret_cast<float2*>(&red[((warp * kMaxBlocks + j) * 8 + g) * 8 + 2 * tq]) = y;
         }
       }
@@ -792,17 +807,18 @@ __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDes
   if (p.trace && threadIdx.x == 0) sm.tm[1] += (unsigned long long)(clock64() - tr0);
 }
 
-template <int MT, int NB = 1>
+// TRI (MT = 1 only): the activations are in three parts (batches up to kTriRows, put_operand).
+template <int MT, int NB = 1, bool TRI = false>
 __device__ void gemv_dispatch(const KParams& p, Smem& sm, const TaskDesc& t, uint32_t& stage, bool& ab, int G) {
   switch (G) {
-    case 1: gemv_body<MT, 1, NB>(p, sm, t, stage, ab); break;
-    case 2: gemv_body<MT, 2, NB>(p, sm, t, stage, ab); break;
-    case 3: gemv_body<MT, 3, NB>(p, sm, t, stage, ab); break;
-    case 4: gemv_body<MT, 4, NB>(p, sm, t, stage, ab); break;
-    case 5: gemv_body<MT, 5, NB>(p, sm, t, stage, ab); break;
-    case 6: gemv_body<MT, 6, NB>(p, sm, t, stage, ab); break;
-    case 7: gemv_body<MT, 7, NB>(p, sm, t, stage, ab); break;
-    default: gemv_body<MT, 8, NB>(p, sm, t, stage, ab); break;
+    case 1: gemv_body<MT, 1, NB, TRI>(p, sm, t, stage, ab); break;
+    case 2: gemv_body<MT, 2, NB, TRI>(p, sm, t, stage, ab); break;
+    case 3: gemv_body<MT, 3, NB, TRI>(p, sm, t, stage, ab); break;
+    case 4: gemv_body<MT, 4, NB, TRI>(p, sm, t, stage, ab); break;
+    case 5: gemv_body<MT, 5, NB, TRI>(p, sm, t, stage, ab); break;
+    case 6: gemv_body<MT, 6, NB, TRI>(p, sm, t, stage, ab); break;
+    case 7: gemv_body<MT, 7, NB, TRI>(p, sm, t, stage, ab); break;
+    default: gemv_body<MT, 8, NB, TRI>(p, sm, t, stage, ab); break;
   }
 }
 
@@ -928,9 +944,10 @@ __device__ void gemv_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_
     inv_inst = inst;
   }
   const int G = t.nunits * rows_per_unit(t.op) / 8;
+  static_assert(kFmaRows == 2, "the FMA path is instantiated for 1 and 2 rows");
   if (p.b == 1) gemv_dispatch<0, 1>(p, sm, t, stage, ab, G);
   else if (p.b == 2) gemv_dispatch<0, 2>(p, sm, t, stage, ab, G);
-  else if (p.b <= kFmaRows) gemv_dispatch<0, 4>(p, sm, t, stage, ab, G);
+  else if (p.b <= kTriRows) gemv_dispatch<1, 1, true>(p, sm, t, stage, ab, G);
   else if (p.b <= 8) gemv_dispatch<1>(p, sm, t, stage, ab, G);
   else gemv_dispatch<2>(p, sm, t, stage, ab, G);
   const long long te0 = (p.trace && threadIdx.x == 0) ? clock64() : 0ll;
@@ -1400,9 +1417,15 @@ __device__ uint64_t warp_kth_largest(Get get, int n, int k, uint32_t* hist) {
   for (int shift = 56; shift >= 0; shift -= 8) {
     for (int i = lane; i < 256; i += 32) hist[i] = 0u;
     __syncwarp();
-    for (int j = lane; j < n; j += 32) {
-      const uint64_t key = get(j);
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    for (int j0 = 0; j0 < n; j0 += 32) {
+      // lanes with the same digit add once (keys of one row bunch into few bins)
+      const int j = j0 + lane;
+      const uint64_t key = j < n ? get(j) : 0ull;
+      const bool in = j < n && (key & mask) == prefix;
+      const unsigned act = __ballot_sync(0xffffffffu, in);
+      const unsigned digit = (unsigned)(key >> shift) & 255u;
+      const unsigned peers = __match_any_sync(0xffffffffu, in ? digit : 256u + (unsigned)lane);
+      if (in && lane == __ffs(peers & act) - 1) atomicAdd(&hist[digit], (unsigned)__popc(peers & act));
     }
     __syncwarp();
     // lane l holds bins 255-8l .. 248-8l: lanes in order walk the bins from the top
@@ -1484,7 +1507,20 @@ __device__ __noinline__ void sample_top_k(const KParams& p, Smem& sm) {
     uint64_t tau0;
     const int kt = min(k, n);
     if (n <= cap) {
-      for (int j = lane; j < n; j += 32) buf[j] = task_key(j);
+      // eight loads in flight per lane
+      for (int j0 = lane; j0 < n; j0 += 256) {
+        float2 c[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int j = j0 + 32 * u;
+          c[u] = j < n ? __ldcg(mx + (size_t)j * p.max_b) : make_float2(0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int j = j0 + 32 * u;
+          if (j < n) buf[j] = logit_key64(c[u].x, __float_as_int(c[u].y));
+        }
+      }
       __syncwarp();
       tau0 = warp_kth_largest([&](int j) { return buf[j]; }, n, kt, hist);
     } else {
@@ -1499,7 +1535,7 @@ __device__ __noinline__ void sample_top_k(const KParams& p, Smem& sm) {
       bool s = false;
       if (j < n) {
         const uint64_t key = n <= cap ? buf[j] : task_key(j);
-        s = key >= tau0 && isfinite(__ldcg(mx + (size_t)j * p.max_b).x);
+        s = key >= tau0 && isfinite(key64_logit(key));
       }
       const unsigned bal = __ballot_sync(0xffffffffu, s);
       const int at = nsel + __popc(bal & ((1u << lane) - 1u));
@@ -1512,19 +1548,37 @@ __device__ __noinline__ void sample_top_k(const KParams& p, Smem& sm) {
       if (lane == 0) p.argmax[bi] = 0x7fffffff;
       continue;
     }
-    // 2. candidates: the selected tasks' logits with key >= tau0
-    int nc = 0;
-    for (int s = 0; s < nsel; ++s) {
+    // 2. candidates: the selected tasks' logits with key >= tau0.  The tasks' row ranges go to
+    // shared memory first (in the space `top` takes later); then (task, row) pairs are walked
+    // flat, eight loads in flight per lane
+    int* row0 = reinterpret_cast<int*>(top);
+    int* nrow = row0 + kMaxTopK;
+    for (int s = lane; s < nsel; s += 32) {
       const int2 rr = __ldcg(p.lmrows + sel[s]);
-      for (int r0 = 0; r0 < rr.y; r0 += 32) {
-        const int r = r0 + lane;
-        uint64_t key = 0;
-        bool c = false;
-        if (r < rr.y) {
-          const int idx = rr.x + r;
-          key = logit_key64(__ldcg(p.logits + (size_t)bi * p.V + idx), idx);
-          c = key >= tau0;
+      row0[s] = rr.x;
+      nrow[s] = rr.y;
+    }
+    __syncwarp();
+    int nc = 0;
+    const int nflat = 64 * nsel;
+    for (int j0 = 0; j0 < nflat; j0 += 256) {
+      float v[8];
+      int idx[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int j = j0 + 32 * u + lane;
+        const int s = j >> 6, r = j & 63;
+        idx[u] = -1;
+        v[u] = 0.f;
+        if (j < nflat && r < nrow[s]) {
+          idx[u] = row0[s] + r;
+          v[u] = __ldcg(p.logits + (size_t)bi * p.V + idx[u]);
         }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint64_t key = idx[u] >= 0 ? logit_key64(v[u], idx[u]) : 0ull;
+        const bool c = idx[u] >= 0 && key >= tau0;
         const unsigned bal = __ballot_sync(0xffffffffu, c);
         const int at = nc + __popc(bal & ((1u << lane) - 1u));
         if (c && at < cap) buf[at] = key;

@@ -45,7 +45,8 @@ def parse():
     ap.add_argument("--no-secondary", action="store_true", help="skip the batch-1 line of the same model")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-all-configs", action="store_true", help="skip timing the other named shapes")
-    ap.add_argument("--no-multi-step", action="store_true", help="skip timing the on-device multi-step loop")
+    ap.add_argument("--no-multi-step", action="store_true",
+                    help="skip timing the on-device multi-step loop, its sampling variant and the multi-token step")
     ap.add_argument("--max-blocks", type=int, default=0, help="schedule option: 8-row blocks per GEMV task")
     ap.add_argument("--attn-slots", type=int, default=0, help="schedule option: attention slots per SM")
     ap.add_argument("--trace", default="", help="write a per-task timeline summary of one step to this file")
@@ -430,6 +431,10 @@ def run_mk(args, world, rank, local):
                              "achieved_gbs": B1 / (ms1 / 1e3) / 1e9}
     if not args.no_multi_step:
         line["multi_step"] = time_multi_step(mk, h, m, tok_d, pos_d, kv, lens, logits, stream, world, ms, flush)
+        line["multi_step_top_k"] = time_multi_step(mk, h, m, tok_d, pos_d, kv, lens, logits, stream, world, ms, flush,
+                                                   top_k=50)
+        if world == 1 and not args.layers:
+            line["verify"] = [time_verify(mk, m, wts, kv, lens[0], t, stream, flush) for t in (4, 8)]
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = {k: v for k, v in cpu_baseline(w, wts, kv, toks, lens).items()
                                 if k != "seconds_per_step"}
@@ -453,16 +458,20 @@ def run_mk(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
-def time_multi_step(mk, h, m, tok_d, pos_d, kv, lens, logits, stream, world, single_ms, flush) -> dict:
-    """The on-device greedy loop: MULTI_STEPS steps per call (each step's greedy token is the
-    next step's input, at the next position), the host waiting once per call.  Per call the
-    context of every sequence grows by MULTI_STEPS, so the bytes are summed step by step."""
+def time_multi_step(mk, h, m, tok_d, pos_d, kv, lens, logits, stream, world, single_ms, flush, top_k=1) -> dict:
+    """The on-device loop: MULTI_STEPS steps per call (each step's token is the next step's
+    input, at the next position), the host waiting once per call; greedy, or top-k sampling
+    (temperature 0.8, seeded uniforms) fused into the step.  Per call the context of every
+    sequence grows by MULTI_STEPS, so the bytes are summed step by step."""
     n, runs = MULTI_STEPS, 5
     b = len(lens)
     toks_out = torch.empty((n, b), dtype=torch.int32, device="cuda")
+    g = torch.Generator(device="cpu").manual_seed(11)
+    uni = torch.rand((n, b), generator=g).to("cuda")
 
     def run():
-        h.steps(n, tok_d, pos_d, kv, toks_out, logits, stream=stream, check=False)
+        h.steps(n, tok_d, pos_d, kv, toks_out, logits, stream=stream, check=False, top_k=top_k, temperature=0.8,
+                uniforms=uni)
 
     for _ in range(2):
         run()
@@ -472,10 +481,38 @@ def time_multi_step(mk, h, m, tok_d, pos_d, kv, lens, logits, stream, world, sin
     assert h.status() == mk.MK_OK, f"device status {h.status()}"
     ms = max_over_ranks(world, total) / (runs * n)
     B = sum(mk.step_bytes(m, [s + k for s in lens]) for k in range(n)) / n
-    return {"n_steps_per_call": n, "calls": runs, "ms_per_step": ms, "tokens_per_s": world * b / (ms / 1e3),
+    return {"n_steps_per_call": n, "calls": runs, "top_k": top_k, "ms_per_step": ms,
+            "tokens_per_s": world * b / (ms / 1e3),
             "mbu": B / (ms / 1e3) / (NOMINAL_HBM_GBS * 1e9), "single_step_ms": single_ms,
             "launches_per_call": n, "host_waits_per_call": 1,
             "l2": "no flush between the steps of one call" + ("; L2 flushed between calls" if flush else "")}
+
+
+def time_verify(mk, m, wts, kv, prior: int, t: int, stream, flush, runs: int = 50) -> dict:
+    """A multi-token step: one sequence with `prior` cached entries and t new (draft) tokens
+    as t rows of one launch on a handle built for t rows; the rows share the sequence's
+    page-table row.  Against t single-token steps, which read every weight t times."""
+    h = mk.Megakernel(m, wts, t, prior + t + 1)
+    table = kv.page_table[torch.zeros(t, dtype=torch.long, device=kv.page_table.device)].contiguous()
+    gkv = synth.KVCache(kv.k_pool, kv.v_pool, table, kv.num_pages, kv.max_pages_per_seq, [prior + j for j in range(t)])
+    tok = torch.tensor(synth.token_ids(m, t, tag="verify"), dtype=torch.int32, device="cuda")
+    pos = torch.arange(prior, prior + t, dtype=torch.int32, device="cuda")
+    first = torch.zeros(t, dtype=torch.int32, device="cuda")
+    lg = torch.empty((t, m.vocab), dtype=torch.float32, device="cuda")
+    am = torch.empty((t,), dtype=torch.int32, device="cuda")
+
+    def run():
+        h.verify(tok, pos, pos + 1, first, gkv, lg, am, stream=stream, check=False)
+
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    total, _ = time_steps(run, runs, stream, flush)
+    assert h.status() == mk.MK_OK, f"device status {h.status()}"
+    h.close()
+    ms = total / runs
+    return {"workload": f"{m.name}: 1 sequence, {prior} cached entries, {t} new tokens in one launch",
+            "tokens": t, "ms_per_step": ms, "tokens_per_s": t / (ms / 1e3)}
 
 
 def time_config(mk, name: str, stream, steps: int, warmup: int, peaks: dict) -> list:

@@ -85,10 +85,16 @@ def _static_step(c, tok, pos, logits, am=None, max_batch=None, max_ctx=None, che
                                  c.kv, logits, am, check=check)
 
 
+QWEN_SMALL = synth.scaled_model(synth.QWEN3_0_6B, name="qwen3-small", n_layers=2, hidden=256, n_heads=4,
+                                n_kv_heads=2, head_dim=128, ffn=512, vocab=4096)
+MODELS = {"tiny": synth.TINY, "smollm2": synth.SMOLLM2_135M, "qwen3-small": QWEN_SMALL}
+
+
 @pytest.mark.parametrize("name, lens, max_ctx", [("tiny", [5, 70, 130], 256),
-                                                  ("smollm2", [1000], 2048)])
+                                                  ("smollm2", [1000], 2048),
+                                                  ("qwen3-small", [40, 0, 17], 64)])
 def test_static_entry_point_matches_oracle_and_handle_entry_point(name, lens, max_ctx):
-    m = synth.TINY if name == "tiny" else synth.SMOLLM2_135M
+    m = MODELS[name]
     c = make_case(m, lens, gain_std=0.1, max_ctx=max_ctx, tag="static-" + name)
     kv_handle = _clone_kv(c.kv)
     kb, vb = c.kv.k_pool.cpu(), c.kv.v_pool.cpu()
