@@ -28,12 +28,16 @@ def needs_build() -> bool:
     return any(os.path.getmtime(d) > t for d in deps if os.path.exists(d))
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not needs_build():
+def build(force: bool = False, verbose: bool = False, trace_detail: bool = False) -> str:
+    """trace_detail: record in-task cycle counts in the per-task timeline (a diagnostic build;
+    the stamps cost a few percent of the step)."""
+    if not force and not trace_detail and not needs_build():
         return LIB
     cmd = [nvcc_path(), "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
            "-Xcompiler", "-fPIC,-fvisibility=hidden", "-shared", "-cudart", "static",
            "-o", LIB + ".tmp"] + [os.path.join(CSRC, s) for s in SOURCES]
+    if trace_detail:
+        cmd.insert(1, "-DMK_TRACE_DETAIL=1")
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), file=sys.stderr)
@@ -43,5 +47,5 @@ def build(force: bool = False, verbose: bool = False) -> str:
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True)
+    build(force="--force" in sys.argv, verbose=True, trace_detail="--trace-detail" in sys.argv)
     print(LIB)

@@ -22,6 +22,14 @@
 
 #include "mk_kernel.h"
 
+// Cycle accounting inside a task (per-stage compute and slot waits, reduce and epilogue
+// time) for the per-task timeline.  Off by default: the stamps sit in the hot loops and cost
+// ~2-3 % of the step.  Timestamps per task (start, dependency met, end) are always recorded
+// when a timeline buffer is set.
+#ifndef MK_TRACE_DETAIL
+#define MK_TRACE_DETAIL 0
+#endif
+
 namespace mk {
 
 typedef __nv_bfloat16 bf16;
@@ -699,13 +707,13 @@ __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDes
     const int slot = stage % kNumSlots;
     const uint32_t par = (stage / kNumSlots) & 1;
     if (!ab && !__shfl_sync(0xffffffffu, ready, 0)) {
-      unsigned long long* wacc = (p.trace && threadIdx.x == 0) ? &sm.wait_cyc : nullptr;
+      unsigned long long* wacc = (MK_TRACE_DETAIL && p.trace && threadIdx.x == 0) ? &sm.wait_cyc : nullptr;
       ab = !mbar_wait_warp(p, &sm.wfull[slot], par, wacc);
       if (!ab) ab = !mbar_wait_warp(p, &sm.ofull[slot], par, wacc);
     }
     if (ab) continue;
     ready = (lane == 0 && s + 1 < nst) ? stage_landed(sm, stage + 1) : 0u;
-    const long long tc0 = (p.trace && threadIdx.x == 0) ? clock64() : 0ll;
+    const long long tc0 = (MK_TRACE_DETAIL && p.trace && threadIdx.x == 0) ? clock64() : 0ll;
     const uint8_t* tile = sm.pool[slot];
     const uint8_t* opnd = tile + (size_t)R * kc * 2;
     const int nb = 2 * ((min(kc, kend - kbeg - s * kc) + kBoxCols - 1) / kBoxCols);
@@ -760,11 +768,11 @@ __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDes
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.empty[slot]);
-    if (p.trace && threadIdx.x == 0) sm.tm[0] += (unsigned long long)(clock64() - tc0);
+    if (MK_TRACE_DETAIL && p.trace && threadIdx.x == 0) sm.tm[0] += (unsigned long long)(clock64() - tc0);
   }
 
   // cross-warp reduction, one 8-row batch tile at a time: red[warp][block][batch g][8 rows]
-  const long long tr0 = (p.trace && threadIdx.x == 0) ? clock64() : 0ll;
+  const long long tr0 = (MK_TRACE_DETAIL && p.trace && threadIdx.x == 0) ? clock64() : 0ll;
   float* red = sm.red;
 #pragma unroll
   for (int mt = 0; mt < NMT; ++mt) {
@@ -804,7 +812,7 @@ __device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDes
     }
     cbar();
   }
-  if (p.trace && threadIdx.x == 0) sm.tm[1] += (unsigned long long)(clock64() - tr0);
+  if (MK_TRACE_DETAIL && p.trace && threadIdx.x == 0) sm.tm[1] += (unsigned long long)(clock64() - tr0);
 }
 
 // TRI (MT = 1 only): the activations are in three parts (batches up to kTriRows, put_operand).
@@ -950,7 +958,7 @@ __device__ void gemv_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_
   else if (p.b <= kTriRows) gemv_dispatch<1, 1, true>(p, sm, t, stage, ab, G);
   else if (p.b <= 8) gemv_dispatch<1>(p, sm, t, stage, ab, G);
   else gemv_dispatch<2>(p, sm, t, stage, ab, G);
-  const long long te0 = (p.trace && threadIdx.x == 0) ? clock64() : 0ll;
+  const long long te0 = (MK_TRACE_DETAIL && p.trace && threadIdx.x == 0) ? clock64() : 0ll;
 
   const int nthr = kConsumerWarps * 32;
   const int n = t.nunits;
@@ -988,7 +996,7 @@ __device__ void gemv_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_
       if (!ab && t.op == OP_LMHEAD && p.argmax)
         for (int bi = threadIdx.x; bi < p.b; bi += nthr)
           p.lmpart[(size_t)t.task_idx * p.max_b + bi] = make_float2(-INFINITY, __int_as_float(0x7fffffff));
-      if (p.trace && threadIdx.x == 0) sm.tm[2] += (unsigned long long)(clock64() - te0);
+      if (MK_TRACE_DETAIL && p.trace && threadIdx.x == 0) sm.tm[2] += (unsigned long long)(clock64() - te0);
       return;
     }
     if (!ab)
@@ -1079,7 +1087,7 @@ __device__ void gemv_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_
       if (threadIdx.x == 0) p.lmrows[t.task_idx] = make_int2(8 * (int)t.u0, min(8 * n, p.V - 8 * (int)t.u0));
     }
   }
-  if (p.trace && threadIdx.x == 0) sm.tm[2] += (unsigned long long)(clock64() - te0);
+  if (MK_TRACE_DETAIL && p.trace && threadIdx.x == 0) sm.tm[2] += (unsigned long long)(clock64() - te0);
 }
 
 __device__ void embed_task(const KParams& p, Smem& sm, const TaskDesc& t, bool ab) {
@@ -1152,7 +1160,7 @@ __device__ __noinline__ void attn_task(const KParams& p, Smem& sm, const TaskDes
   const int grp = warp % WPS, wsel = warp / WPS;
   const int G = p.g;
   const float sc = 1.4426950408889634f / sqrtf((float)HD);
-  const bool tr = p.trace && threadIdx.x == 0;
+  const bool tr = MK_TRACE_DETAIL && p.trace && threadIdx.x == 0;
   uint32_t ks = 0;  // stage count within the task: picks the warp group
   AttnPiece a;
   for (int j = 0; attn_piece(p, sm, (int)t.u0, j, a); ++j) {

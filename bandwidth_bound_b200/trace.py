@@ -6,7 +6,9 @@ layer << 8 | sm << 24 | slot_wait << 40, and the durations in SM clock cycles (t
 globaltimer is too coarse for sub-microsecond intervals), converted here with the SM
 clock.  The summary answers where a step's time goes: waiting on dependency counters
 (another SM's work not done), waiting on pool slots (HBM bytes not yet landed), or
-computing.
+computing.  The in-task durations (compute, reduce, epilogue, slot_wait) are recorded only
+by a library built with MK_TRACE_DETAIL=1 (`build.py --trace-detail`); the default build
+leaves them 0 and records the timestamps and the signal time.
 """
 from __future__ import annotations
 
