@@ -263,27 +263,46 @@ __device__ __forceinline__ int gemv_K_dev(const KParams& p, int op) {
 // Issue the TMA box(es) of 64-column chunk c of one GEMV stage.  Chunk layout in the
 // slot: rows of the task, 128 bytes each, swizzled; QKV: first-half rows then the
 // matching second-half rows of one head; gate/up: gate rows then up rows.
-__device__ __forceinline__ void issue_gemv_chunk(const KParams& p, const TaskDesc& t, int k, uint8_t* dst,
-                                                 uint64_t* bar, uint64_t pol) {
+struct GemvBoxes {
+  const void* m0;         // tensor map of the (first) matrix
+  const void* m1;         // gate/up: the up matrix (its rows follow the gate rows in a chunk)
+  int c1, c2;             // row coordinate; 3-D maps (QKV): head-half coordinate
+  bool three_d;
+  uint32_t chunk_bytes;   // one 64-column chunk of all the task's rows (128 bytes per row)
+  uint32_t second_off;    // gate/up: offset of the up rows within a chunk
+};
+
+// The TMA boxes of a GEMV task's stages.  Chunk layout in the slot: the task's rows, 128
+// bytes each, swizzled; QKV: first-half rows then the matching second-half rows of one head;
+// gate/up: gate rows then up rows.
+__device__ __forceinline__ GemvBoxes gemv_boxes(const KParams& p, const TaskDesc& t) {
   const CUtensorMapLike* maps = reinterpret_cast<const CUtensorMapLike*>(p.tmaps);
   const int n = t.nunits;
+  GemvBoxes b{};
+  b.chunk_bytes = (uint32_t)(n * rows_per_unit(t.op) * 128);
+  b.c1 = 8 * (int)t.u0;
   switch (t.op) {
     case OP_QKV: {
       const int per_head = p.hd >> 4;
       const int hh = (int)t.u0 / per_head, m0 = (int)t.u0 - hh * per_head;
       const int mat = hh < p.nq ? 0 : (hh < p.nq + p.nkv ? 1 : 2);
       const int lh = mat == 0 ? hh : (mat == 1 ? hh - p.nq : hh - p.nq - p.nkv);
-      tma_3d(dst, maps + tmap_index(t.layer, mat, n), k, 8 * m0, 2 * lh, bar, pol);
+      b.m0 = maps + tmap_index(t.layer, mat, n);
+      b.c1 = 8 * m0;
+      b.c2 = 2 * lh;
+      b.three_d = true;
       break;
     }
     case OP_GATEUP:
-      tma_2d(dst, maps + tmap_index(t.layer, 4, n), k, 8 * (int)t.u0, bar, pol);
-      tma_2d(dst + 8 * n * 128, maps + tmap_index(t.layer, 5, n), k, 8 * (int)t.u0, bar, pol);
+      b.m0 = maps + tmap_index(t.layer, 4, n);
+      b.m1 = maps + tmap_index(t.layer, 5, n);
+      b.second_off = (uint32_t)(8 * n * 128);
       break;
-    case OP_OPROJ: tma_2d(dst, maps + tmap_index(t.layer, 3, n), k, 8 * (int)t.u0, bar, pol); break;
-    case OP_DOWN: tma_2d(dst, maps + tmap_index(t.layer, 6, n), k, 8 * (int)t.u0, bar, pol); break;
-    default: tma_2d(dst, maps + tmap_index(p.L, 0, n), k, 8 * (int)t.u0, bar, pol); break;
+    case OP_OPROJ: b.m0 = maps + tmap_index(t.layer, 3, n); break;
+    case OP_DOWN: b.m0 = maps + tmap_index(t.layer, 6, n); break;
+    default: b.m0 = maps + tmap_index(p.L, 0, n); break;
   }
+  return b;
 }
 
 // Split-K attention work, partitioned at run time from this step's lengths in one of two ways.
@@ -429,20 +448,6 @@ __device__ __forceinline__ int gemv_stages(const KParams& p, const TaskDesc& t) 
   return (kend - kbeg + t.kc - 1) / t.kc;
 }
 
-// Weights of stage s of GEMV task t into slot `slot`: one tiled box per 64 columns.
-__device__ void issue_weights(const KParams& p, Smem& sm, const TaskDesc& t, int s, int slot, uint64_t pol) {
-  const int lane = threadIdx.x & 31;
-  int kbeg, kend;
-  gemv_krange(p, t, kbeg, kend);
-  const int R = t.nunits * rows_per_unit(t.op);
-  const int kc0 = kbeg + s * t.kc;
-  const int nch = (min((int)t.kc, kend - kc0) + kBoxCols - 1) / kBoxCols;
-  if (lane == 0) mbar_expect_tx(&sm.wfull[slot], (uint32_t)(nch * R * 128));
-  __syncwarp();
-  for (int c = lane; c < nch; c += 32)
-    issue_gemv_chunk(p, t, kc0 + c * kBoxCols, sm.pool[slot] + (size_t)c * R * 128, &sm.wfull[slot], pol);
-}
-
 // K and V pages of stage k of attention piece a into slot `slot`: whole 16-token pages as
 // tiled boxes (128-byte swizzle; head_dim 128 as [2 halves][16 rows][64]), K pages at the
 // slot's start and V pages at half the slot.  Returns false on a page id out of range.
@@ -452,21 +457,19 @@ __device__ bool issue_kv(const KParams& p, Smem& sm, const TaskDesc& t, const At
   const int T = attn_stage_tokens(p.hd);
   const int s0 = a.t0 + k * T, s1 = min(s0 + T, a.t1);
   const int pg0 = s0 / kPage, npg = (s1 - 1) / kPage - pg0 + 1;
-  bool bad = false;
-  for (int q = lane; q < npg; q += 32) {
-    const int id = p.ptable[a.i * p.mpps + pg0 + q];
-    if (id < 0 || id >= p.num_pages) bad = true;
-  }
-  if (__any_sync(0xffffffffu, bad)) return false;
+  // a stage spans at most T / 16 <= 8 pages (ranges and stages start on page boundaries):
+  // lanes 2q and 2q + 1 take the K and V box of page q, each reading its page id once
+  const int q = lane >> 1;
+  const bool act = q < npg;
+  const int id = act ? p.ptable[a.i * p.mpps + pg0 + q] : 0;
+  if (__any_sync(0xffffffffu, act && (id < 0 || id >= p.num_pages))) return false;
   const uint32_t page_bytes = (uint32_t)kPage * p.hd * 2u;
   if (lane == 0) mbar_expect_tx(&sm.wfull[slot], 2u * npg * page_bytes);
   __syncwarp();
-  for (int e = lane; e < 2 * npg; e += 32) {
-    const int q = e >> 1;
-    const int id = p.ptable[a.i * p.mpps + pg0 + q];
+  if (act) {
     const int row = ((t.layer * p.num_pages + id) * p.nkv + a.h) * kPage;
-    uint8_t* dst = sm.pool[slot] + (size_t)(e & 1) * T * p.hd * 2 + (size_t)q * page_bytes;
-    const void* map = (e & 1) ? (const void*)&p.vmap : (const void*)&p.kmap;
+    uint8_t* dst = sm.pool[slot] + (size_t)(lane & 1) * T * p.hd * 2 + (size_t)q * page_bytes;
+    const void* map = (lane & 1) ? (const void*)&p.vmap : (const void*)&p.kmap;
     if (p.hd == 64) tma_2d(dst, map, 0, row, &sm.wfull[slot], pol);
     else tma_3d(dst, map, 0, row, 0, &sm.wfull[slot], pol);
   }
@@ -500,11 +503,29 @@ __device__ void producer(const KParams& p, Smem& sm, const TaskDesc* ts, int nt)
       }
       continue;
     }
+    // The task's boxes: map(s) and every coordinate but K are the same for all its stages,
+    // so they are worked out once; a released slot then costs only its K coordinate.
     const int wn = gemv_stages(p, t);
+    int kbeg, kend;
+    gemv_krange(p, t, kbeg, kend);
+    const GemvBoxes bx = gemv_boxes(p, t);
     for (int ws = 0; ws < wn; ++ws, ++wk) {
       const int slot = wk % kNumSlots;
       if (!mbar_wait_warp(p, &sm.empty[slot], ((wk / kNumSlots) & 1) ^ 1)) { fail = true; break; }
-      issue_weights(p, sm, t, ws, slot, pol);
+      const int kc0 = kbeg + ws * t.kc;
+      const int nch = (min((int)t.kc, kend - kc0) + kBoxCols - 1) / kBoxCols;
+      if (lane == 0) mbar_expect_tx(&sm.wfull[slot], (uint32_t)nch * bx.chunk_bytes);
+      __syncwarp();
+      for (int c = lane; c < nch; c += 32) {
+        uint8_t* dst = sm.pool[slot] + (size_t)c * bx.chunk_bytes;
+        const int kk = kc0 + c * kBoxCols;
+        if (bx.three_d) {
+          tma_3d(dst, bx.m0, kk, bx.c1, bx.c2, &sm.wfull[slot], pol);
+        } else {
+          tma_2d(dst, bx.m0, kk, bx.c1, &sm.wfull[slot], pol);
+          if (bx.m1) tma_2d(dst + bx.second_off, bx.m1, kk, bx.c1, &sm.wfull[slot], pol);
+        }
+      }
     }
   }
   if (fail) {
