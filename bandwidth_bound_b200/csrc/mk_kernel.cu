@@ -588,37 +588,39 @@ __device__ void operand_loader(const KParams& p, Smem& sm, const TaskDesc* ts, i
         __syncwarp();
       }
     }
+    // Everything but the K coordinate and the slot is the same for all of the task's stages:
+    // worked out once.  fp32 rows (batches up to kFmaRows): per chunk c, row r's 256 bytes at
+    // (c * NB + r) * 256, box e = c * NB + r.  bf16 tiles: (tile, part) q's 1024-byte box of
+    // chunk c at q * kc * 16 + c * 1024, box e = q * nch + c.
     const int kind = operand_kind(t.op);
     int kbeg, kend;
     gemv_krange(p, t, kbeg, kend);
     const int R = t.nunits * rows_per_unit(t.op);
     const int nst = gemv_stages(p, t);
+    const bool f32 = p.b <= kFmaRows;
+    const int NB = fma_rows(p.b);
+    const int rows_per_row = (kind == 0 ? p.ld_x : (kind == 1 ? p.ld_a : p.ld_h)) / 32;
+    const int per_chunk = f32 ? NB : 2 * ntile;             // boxes per 64-column chunk
+    const uint32_t box_bytes = f32 ? 256u : 1024u;
+    const CUtensorMapLike* kmaps = maps + opmap_index(p.L, kind, 0);
+    const int off0 = R * t.kc * 2;
     for (int ws = 0; ws < nst; ++ws, ++wk) {
       const int slot = wk % kNumSlots;
       if (!mbar_wait_warp(p, &sm.empty[slot], ((wk / kNumSlots) & 1) ^ 1)) { fail = true; break; }
-      uint8_t* dst = sm.pool[slot] + (size_t)R * t.kc * 2;
+      uint8_t* dst = sm.pool[slot] + off0;
       const int k0 = kbeg + ws * t.kc;
       const int nch = (min((int)t.kc, kend - k0) + kBoxCols - 1) / kBoxCols;
-      if (p.b <= kFmaRows) {
-        // fp32 rows 0..NB-1: per chunk c, row r's 256 bytes at (c * NB + r) * 256
-        const int NB = fma_rows(p.b);
-        const int rows_per_row = (kind == 0 ? p.ld_x : (kind == 1 ? p.ld_a : p.ld_h)) / 32;
-        const int nbox = NB * nch;
-        if (lane == 0) mbar_expect_tx(&sm.ofull[slot], (uint32_t)nbox * 256u);
-        __syncwarp();
-        for (int e = lane; e < nbox; e += 32) {
+      const int nbox = per_chunk * nch;
+      if (lane == 0) mbar_expect_tx(&sm.ofull[slot], (uint32_t)nbox * box_bytes);
+      __syncwarp();
+      for (int e = lane; e < nbox; e += 32) {
+        if (f32) {
           const int c = e / NB, r = e - c * NB;
-          tma_2d(dst + (size_t)e * 256, maps + opmap_index(p.L, kind, kOpMapsPerKind - 1), 0,
-                 r * rows_per_row + k0 / 32 + 2 * c, &sm.ofull[slot], pol);
-        }
-      } else {
-        const int nbox = 2 * ntile * nch;
-        if (lane == 0) mbar_expect_tx(&sm.ofull[slot], (uint32_t)nbox * 1024u);
-        __syncwarp();
-        for (int e = lane; e < nbox; e += 32) {
-          const int q = e / nch, c = e - q * nch;
-          tma_2d(dst + (size_t)q * t.kc * 16 + (size_t)c * 1024, maps + opmap_index(p.L, kind, q), 0, k0 / 8 + 8 * c,
+          tma_2d(dst + (size_t)e * 256, kmaps + (kOpMapsPerKind - 1), 0, r * rows_per_row + k0 / 32 + 2 * c,
                  &sm.ofull[slot], pol);
+        } else {
+          const int q = e / nch, c = e - q * nch;
+          tma_2d(dst + (size_t)q * t.kc * 16 + (size_t)c * 1024, kmaps + q, 0, k0 / 8 + 8 * c, &sm.ofull[slot], pol);
         }
       }
       __syncwarp();
