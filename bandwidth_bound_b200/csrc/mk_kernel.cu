@@ -615,11 +615,13 @@ __device__ void operand_loader(const KParams& p, Smem& sm, const TaskDesc* ts, i
       __syncwarp();
       for (int e = lane; e < nbox; e += 32) {
         if (f32) {
-          const int c = e / NB, r = e - c * NB;
+          const int c = NB == 1 ? e : (e >> 1), r = e - c * NB;
           tma_2d(dst + (size_t)e * 256, kmaps + (kOpMapsPerKind - 1), 0, r * rows_per_row + k0 / 32 + 2 * c,
                  &sm.ofull[slot], pol);
         } else {
-          const int q = e / nch, c = e - q * nch;
+          // q = e / nch for q < 2 * kMaxTiles <= 4, without a division
+          static_assert(kMaxTiles <= 2, "operand boxes of at most four (tile, part) pairs");
+          const int q = (e >= nch) + (e >= 2 * nch) + (e >= 3 * nch), c = e - q * nch;
           tma_2d(dst + (size_t)q * t.kc * 16 + (size_t)c * 1024, kmaps + q, 0, k0 / 8 + 8 * c, &sm.ofull[slot], pol);
         }
       }
