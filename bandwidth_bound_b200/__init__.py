@@ -101,6 +101,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "mk_router_step": (ctypes.c_int, [vp, vp, vp, vp, i32, i32, ctypes.POINTER(KvCache), vp, vp,
                                           ctypes.POINTER(i32), vp]),
         "mk_router_destroy": (ctypes.c_int, [vp]),
+        "mk_kpo_create": (ctypes.c_int, [ctypes.POINTER(ModelCfg), ctypes.POINTER(WeightPtrs), ctypes.POINTER(vp)]),
+        "mk_kpo_step": (ctypes.c_int, [vp, vp, vp, vp, i32, ctypes.POINTER(KvCache), vp, vp, i32,
+                                       ctypes.POINTER(ctypes.c_float), vp]),
+        "mk_kpo_launches_per_step": (ctypes.c_int, [vp]),
+        "mk_kpo_destroy": (ctypes.c_int, [vp]),
+        "mk_kpo_last_error": (ctypes.c_char_p, [vp]),
         "mk_get_status": (ctypes.c_int, [vp]),
         "mk_reset": (ctypes.c_int, [vp]),
         "mk_set_debug": (ctypes.c_int, [vp, vp]),
@@ -384,6 +390,49 @@ class Router:
     def close(self):
         if self.ptr:
             self.lib.mk_router_destroy(self.ptr)
+            self.ptr = ctypes.c_void_p()
+
+
+KPO_GRAPH, KPO_STREAM, KPO_TIMED, KPO_EMPTY = 0, 1, 2, 3
+
+
+class KernelPerOp:
+    """The same decode step as one kernel per operation (mk_kpo_*): a comparison for the
+    single-launch step.  mode: KPO_GRAPH (CUDA graph replay), KPO_STREAM (launches on the
+    stream), KPO_TIMED (no overlap; step() then returns the summed kernel time in ms),
+    KPO_EMPTY (the same launches doing nothing: the cost of the launches alone)."""
+
+    def __init__(self, m, weights: dict, max_batch: int, max_ctx: int):
+        import torch
+
+        self.lib = load_library()
+        self._torch = torch
+        self.cfg = model_cfg(m, max_batch, max_ctx)
+        w, self._arrays = weight_struct(m, weights)
+        self.weights = weights
+        self.ptr = ctypes.c_void_p()
+        rc = self.lib.mk_kpo_create(ctypes.byref(self.cfg), ctypes.byref(w), ctypes.byref(self.ptr))
+        if rc != MK_OK:
+            raise MkError(rc, "mk_kpo_create: " + (self.lib.mk_kpo_last_error(None) or b"").decode())
+
+    def step(self, token_ids, positions, seq_lens, kv, logits, argmax=None, mode: int = KPO_GRAPH, stream=None):
+        if stream is None:
+            stream = self._torch.cuda.current_stream()
+        busy = ctypes.c_float(0.0)
+        kvs = Megakernel.kv_struct(kv)
+        rc = self.lib.mk_kpo_step(self.ptr, _ptr(token_ids), _ptr(positions), _ptr(seq_lens), int(token_ids.numel()),
+                                  ctypes.byref(kvs), _ptr(logits), _ptr(argmax), int(mode), ctypes.byref(busy),
+                                  ctypes.c_void_p(stream.cuda_stream))
+        if rc != MK_OK:
+            raise MkError(rc, "mk_kpo_step: " + (self.lib.mk_kpo_last_error(self.ptr) or b"").decode())
+        return busy.value
+
+    def launches_per_step(self) -> int:
+        return self.lib.mk_kpo_launches_per_step(self.ptr)
+
+    def close(self):
+        if self.ptr:
+            self.lib.mk_kpo_destroy(self.ptr)
             self.ptr = ctypes.c_void_p()
 
 

@@ -8,7 +8,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmk.so")
-SOURCES = ["mk_api.cu", "mk_kernel.cu", "mk_plan.cpp"]
+SOURCES = ["mk_api.cu", "mk_kernel.cu", "mk_plan.cpp", "kpo.cu"]
 HEADERS = ["mk_common.h", "mk_kernel.h", "mk_plan.h"]
 PUBLIC_HEADER = os.path.join(os.path.dirname(HERE), "include", "mk.h")
 

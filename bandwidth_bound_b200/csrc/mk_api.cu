@@ -245,7 +245,7 @@ static int check_device(int dev, const char* who) {
 
 // RoPE inverse frequencies, in double: theta^(-2j/hd), then the Llama-3.x frequency scaling
 // when rope_scale_factor > 1 (the rule in mk.h's mk_model_cfg).
-static mk::RopeFreq rope_freq(const mk_model_cfg& c) {
+mk::RopeFreq mk_rope_freq(const mk_model_cfg& c) {
   mk::RopeFreq f{};
   const int half = c.head_dim / 2;
   const double pi = 3.14159265358979323846;
@@ -364,7 +364,7 @@ static int upload_tables(const mk_plan_s& plan, const mk_weight_ptrs* w, const s
                          cudaMemcpyHostToDevice, stream);
   if (ce == cudaSuccess)
     ce = cudaMemcpyAsync(A + L.maps, maps.data(), sizeof(CUtensorMap) * maps.size(), cudaMemcpyHostToDevice, stream);
-  if (ce == cudaSuccess) ce = mk::launch_rope_table((float2*)(A + L.rope), c.max_ctx, G.hd, rope_freq(c), stream);
+  if (ce == cudaSuccess) ce = mk::launch_rope_table((float2*)(A + L.rope), c.max_ctx, G.hd, mk_rope_freq(c), stream);
   if (ce == cudaSuccess) ce = cudaStreamSynchronize(stream);
   if (ce != cudaSuccess) return cuda_fail(nullptr, ce, (std::string(who) + ": upload").c_str());
   return MK_OK;

@@ -81,6 +81,11 @@ struct RopeFreq {
   double inv_freq[64];  // per rotation pair j < hd / 2
 };
 cudaError_t launch_rope_table(float2* table, int max_ctx, int hd, const RopeFreq& f, cudaStream_t s);
+
 cudaError_t kernel_attributes(int* regs, int* local_bytes, int* max_threads);
 
 }  // namespace mk
+
+// RoPE inverse frequencies of a model cfg (the scaling rule of mk_model_cfg), in double.
+struct mk_model_cfg;
+mk::RopeFreq mk_rope_freq(const mk_model_cfg& c);

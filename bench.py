@@ -45,6 +45,7 @@ def parse():
     ap.add_argument("--no-secondary", action="store_true", help="skip the batch-1 line of the same model")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-all-configs", action="store_true", help="skip timing the other named shapes")
+    ap.add_argument("--no-kernel-per-op", action="store_true", help="skip timing the kernel-per-op comparison step")
     ap.add_argument("--no-multi-step", action="store_true",
                     help="skip timing the on-device multi-step loop, its sampling variant and the multi-token step")
     ap.add_argument("--max-blocks", type=int, default=0, help="schedule option: 8-row blocks per GEMV task")
@@ -435,6 +436,9 @@ def run_mk(args, world, rank, local):
                                                    top_k=50)
         if world == 1 and not args.layers:
             line["verify"] = [time_verify(mk, m, wts, kv, lens[0], t, stream, flush) for t in (4, 8)]
+    if world == 1 and not args.layers and not args.no_kernel_per_op:
+        line["kernel_per_op"] = [time_kernel_per_op(mk, m, wts, kv, lens, bb, max_ctx, stream, flush, steps)
+                                 for bb, steps in ((b, ms), (1, line.get("secondary", {}).get("ms_per_step")))]
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = {k: v for k, v in cpu_baseline(w, wts, kv, toks, lens).items()
                                 if k != "seconds_per_step"}
@@ -513,6 +517,38 @@ def time_verify(mk, m, wts, kv, prior: int, t: int, stream, flush, runs: int = 5
     ms = total / runs
     return {"workload": f"{m.name}: 1 sequence, {prior} cached entries, {t} new tokens in one launch",
             "tokens": t, "ms_per_step": ms, "tokens_per_s": t / (ms / 1e3)}
+
+
+def time_kernel_per_op(mk, m, wts, kv, lens, b, max_ctx, stream, flush, mk_ms, runs: int = 30) -> dict:
+    """The same step as one kernel per operation (10 per layer + 4), on the same weights and
+    cache: replayed as a CUDA graph with programmatic dependent launch, launched on the
+    stream, and the same launches with kernels that do nothing: that graph's time is what
+    the 10 L + 4 kernel boundaries cost by themselves."""
+    k = mk.KernelPerOp(m, wts, b, max_ctx)
+    tok = torch.tensor(synth.token_ids(m, b, tag="kpo"), dtype=torch.int32, device="cuda")
+    pos = torch.tensor(lens[:b], dtype=torch.int32, device="cuda")
+    lg = torch.empty((b, m.vocab), dtype=torch.float32, device="cuda")
+    am = torch.empty((b,), dtype=torch.int32, device="cuda")
+    out = {"workload": f"{m.name} b{b}", "launches_per_step": k.launches_per_step()}
+    for name, mode in (("graph_pdl", mk.KPO_GRAPH), ("stream_pdl", mk.KPO_STREAM)):
+        run = lambda: k.step(tok, pos, pos + 1, kv, lg, am, mode=mode, stream=stream)  # noqa: E731
+        for _ in range(3):
+            run()
+        torch.cuda.synchronize()
+        total, _ = time_steps(run, runs, stream, flush)
+        out[f"ms_per_step_{name}"] = total / runs
+    run = lambda: k.step(tok, pos, pos + 1, kv, lg, am, mode=mk.KPO_EMPTY, stream=stream)  # noqa: E731
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    total, _ = time_steps(run, runs, stream, None)
+    out["ms_per_step_launches_only"] = total / runs
+    out["us_per_launch"] = 1e3 * out["ms_per_step_launches_only"] / out["launches_per_step"]
+    if mk_ms:
+        out["megakernel_ms_per_step"] = mk_ms
+        out["graph_vs_megakernel"] = out["ms_per_step_graph_pdl"] / mk_ms
+    k.close()
+    return out
 
 
 def time_config(mk, name: str, stream, steps: int, warmup: int, peaks: dict) -> list:

@@ -303,6 +303,39 @@ MK_API int mk_launches_per_step(mk_handle_t h);
 
 MK_API int mk_destroy(mk_handle_t h);
 
+/* ---- the kernel-per-op step ------------------------------------------------------------ */
+
+/* The same decode step run the way a conventional engine runs it: one kernel per operation
+ * (per layer RMSNorm, QKV GEMV, RoPE + KV append, split-K attention, its combine, O GEMV +
+ * residual, RMSNorm, gate/up GEMV, SwiGLU, down GEMV + residual; then the final norm, the
+ * LM head and the argmax: 10 * n_layers + 4 launches), each launch allowed to overlap its
+ * predecessor's tail (programmatic dependent launch).  A comparison for the single-launch
+ * step (ForgeMegakernel §1: engines launch 280-448 kernels per token; §2.3): the launches
+ * per token, and the device time the kernel boundaries add.  Plain CUDA-core kernels
+ * (fp32 arithmetic on bf16 weights and cache); batches up to 8, no QK-norm.
+ *   mk_kpo_create: cfg and weights as for mk_create; allocates its buffers.
+ *   mk_kpo_step: arguments as for mk_decode_step (the same cache layout and page table),
+ *     plus mode: MK_KPO_GRAPH replays a CUDA graph of the launches (captured on the first
+ *     call and again when the batch or the cache changes); MK_KPO_STREAM launches them on
+ *     the stream; MK_KPO_TIMED launches them without overlap with an event after each and
+ *     synchronises, writing the sum of the kernels' own times to *busy_ms (the events add
+ *     their own cost); MK_KPO_EMPTY replays a graph of the same launches, same grids, with
+ *     a kernel that does nothing but wait for its predecessor: its time is that of the
+ *     launches and kernel boundaries alone (no results are written).  In the other modes the
+ *     logits and argmax are copied to the caller's buffers at the end of the step. */
+typedef struct mk_kpo_s *mk_kpo_t;
+#define MK_KPO_GRAPH 0
+#define MK_KPO_STREAM 1
+#define MK_KPO_TIMED 2
+#define MK_KPO_EMPTY 3
+MK_API int mk_kpo_create(const mk_model_cfg *cfg, const mk_weight_ptrs *weights, mk_kpo_t *out);
+MK_API int mk_kpo_step(mk_kpo_t k, const int32_t *token_ids, const int32_t *positions,
+                       const int32_t *seq_lens, int32_t batch, const mk_kv_cache *kv, float *logits_out,
+                       int32_t *argmax_out, int32_t mode, float *busy_ms, mk_stream_t stream);
+MK_API int mk_kpo_launches_per_step(mk_kpo_t k);
+MK_API int mk_kpo_destroy(mk_kpo_t k);
+MK_API const char *mk_kpo_last_error(mk_kpo_t k);
+
 /* ---- routing among handles specialised by bounds ------------------------------------ */
 
 /* A handle is built for bounds (cfg.max_batch, cfg.max_ctx); its schedule is specialised to
