@@ -624,7 +624,6 @@ __device__ void operand_loader(const KParams& p, Smem& sm, const TaskDesc* ts, i
           tma_2d(dst + (size_t)q * t.kc * 16 + (size_t)c * 1024, kmaps + q, 0, k0 / 8 + 8 * c, &sm.wfull[slot], pol);
         }
       }
-      __syncwarp();
     }
   }
   if (fail) {
