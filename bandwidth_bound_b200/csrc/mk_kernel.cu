@@ -215,9 +215,10 @@ __device__ __forceinline__ uint32_t stage_landed(Smem& sm, uint32_t st) {
   return mbar_test(&sm.wfull[slot], par) ? 1u : 0u;
 }
 
-// Warp-wide wait for the copy warps: every lane tests the barrier (one shared-memory request),
-// a vote makes the answer uniform; the polling loop, with its abort and time-limit checks
-// (decided by vote too), is out of line.
+// Warp-wide wait, taken by whole warps (copy warps, consumer stage waits, signal warp): every
+// lane tests the barrier (one shared-memory request) and a vote makes the answer uniform, so
+// no lane waits alone and then broadcasts; the polling loop, with its abort and time-limit
+// checks (decided by vote too), is out of line.
 __device__ __noinline__ bool mbar_wait_all_slow(const KParams& p, uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = gtimer();
   for (uint32_t it = 1;; ++it) {
@@ -234,7 +235,6 @@ __device__ __noinline__ bool mbar_wait_all_slow(const KParams& p, uint64_t* bar,
 __device__ __forceinline__ bool mbar_wait_all(const KParams& p, uint64_t* bar, uint32_t parity) {
   return __all_sync(0xffffffffu, mbar_try(bar, parity)) || mbar_wait_all_slow(p, bar, parity);
 }
-
 
 // Wait until counter c has received count*epoch signals (wrap-around safe).
 __device__ bool wait_counter(const KParams& p, int c, uint32_t count) {

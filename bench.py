@@ -171,19 +171,29 @@ def job_throughput(world: int, total_ms_this_rank: float, steps: int, batch: int
     return ms, world * batch / (ms / 1e3)
 
 
+def kernel_source_hash(root: str = ROOT) -> str:
+    """Hash of the kernel's source code, comments and layout left out: a summary taken on a
+    kernel stays valid through edits of its comments, and no longer after any code change."""
+    import hashlib
+    import re
+
+    code = ""
+    for f in ("mk_kernel.cu", "mk_common.h", "mk_kernel.h"):
+        with open(os.path.join(root, "bandwidth_bound_b200", "csrc", f)) as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        code += " ".join(text.split()) + "\n"
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
+
+
 def traffic_from_profile(workload: str):
     """Per-launch DRAM bytes recorded by the committed ncu summary, if it covers this
-    workload and the kernel sources it was taken on are unchanged."""
-    import hashlib
-
+    workload and the kernel code it was taken on is unchanged."""
     p = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(p):
         return None
-    src = b""
-    for f in ("mk_kernel.cu", "mk_common.h", "mk_kernel.h"):
-        with open(os.path.join(ROOT, "bandwidth_bound_b200", "csrc", f), "rb") as fh:
-            src += fh.read()
-    h = hashlib.sha256(src).hexdigest()[:16]
+    h = kernel_source_hash()
     with open(p) as f:
         for line in f:
             parts = line.split()
