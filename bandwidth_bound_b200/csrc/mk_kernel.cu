@@ -730,8 +730,11 @@ __device__ __forceinline__ void put_operand(const KParams& p, bf16* tiles, float
 // MT = 0: CUDA-core FMA on fp32 activations for NB (1 or 2 = batch) rows, the operands of
 // chunk c row r at (c * NB + r) * 256 bytes; MT = 1, 2: mma.sync with MT tiles of 8 batch
 // rows, the M = 16 tile holding the bf16 parts of the activations (put_operand).
+// Inlined into the consumer loop like the attention body: as called functions, the two cost
+// each task ~0.5-1 µs on entry (call, spills of live registers, a cold code path) and the
+// step 4.7 % (b8) / 4.3 % (b1).
 template <int MT, int G, int NB = 1, bool TRI = false>
-__device__ __noinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDesc t, uint32_t& stage, bool& ab) {
+__device__ __forceinline__ void gemv_body(const KParams& p, Smem& sm, const TaskDesc t, uint32_t& stage, bool& ab) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, tq = lane & 3;
   int kbeg, kend;
@@ -1198,7 +1201,7 @@ __device__ __forceinline__ uint32_t split_pair(float x, float y, bool lo) {
 // normalised and stored here.  A template argument, so that models without QK-norm run code
 // with none of it.
 template <int HD, bool QKN>
-__device__ __noinline__ void attn_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_t& stage, bool& ab) {
+__device__ __forceinline__ void attn_task(const KParams& p, Smem& sm, const TaskDesc& t, uint32_t& stage, bool& ab) {
   constexpr int T = HD == 64 ? 128 : 96;      // tokens per stage (K then V: 32 / 48 KB)
   constexpr int WPS = T / 16;                 // warps per stage, one 16-token group each
   constexpr int NG = kConsumerWarps / WPS;    // stages in flight across warp groups
