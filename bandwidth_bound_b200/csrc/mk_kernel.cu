@@ -217,9 +217,11 @@ __device__ __forceinline__ uint32_t stage_landed(Smem& sm, uint32_t st) {
 
 // Warp-wide wait, taken by whole warps (copy warps, consumer stage waits, signal warp): every
 // lane tests the barrier (one shared-memory request) and a vote makes the answer uniform, so
-// no lane waits alone and then broadcasts; the polling loop, with its abort and time-limit
-// checks (decided by vote too), is out of line.
-__device__ __noinline__ bool mbar_wait_all_slow(const KParams& p, uint64_t* bar, uint32_t parity) {
+// no lane waits alone and then broadcasts; the polling loop checks the abort flag and the
+// time limit (decided by vote too).  Inlined, like every function on the step's paths but
+// the error report and the sampler: a call costs a warp its live registers' spills and
+// refills after the wait (out of line, the waits and the QK-norm epilogue cost 1.5 % at b8).
+__device__ __forceinline__ bool mbar_wait_all_slow(const KParams& p, uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = gtimer();
   for (uint32_t it = 1;; ++it) {
     if (__all_sync(0xffffffffu, mbar_try(bar, parity))) return true;
@@ -255,7 +257,7 @@ __device__ bool wait_counter(const KParams& p, int c, uint32_t count) {
   }
 }
 
-__device__ __noinline__ bool wait_counter_all_slow(const KParams& p, const uint32_t* ptr, uint32_t target) {
+__device__ __forceinline__ bool wait_counter_all_slow(const KParams& p, const uint32_t* ptr, uint32_t target) {
   const uint64_t t0 = gtimer();
   for (uint32_t it = 1;; ++it) {
     __nanosleep(64);
@@ -942,7 +944,7 @@ __device__ __forceinline__ void qkv_epilogue(const KParams& p, Smem& sm, const T
 // sum of squares (its units' rows of both halves, added in row order) to one slot per unit.
 // Where the whole head is read (attention) the slots are added and the factor applied; the
 // key is stored into the cache there.  Values are appended here as usual.
-__device__ __noinline__ void qkv_epilogue_qk_norm(const KParams& p, Smem& sm, const TaskDesc& t) {
+__device__ __forceinline__ void qkv_epilogue_qk_norm(const KParams& p, Smem& sm, const TaskDesc& t) {
   const int nthr = kConsumerWarps * 32;
   const int n = t.nunits;
   const int half = p.hd / 2, per_head = p.hd >> 4;
